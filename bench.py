@@ -1,0 +1,448 @@
+"""Benchmark of the NVFP4 W4A4 linear-layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode|prefill]
+
+Prints ONE JSON line (rank 0).  Default workload ("decode"): the decode GEMV
+configuration -- M in {1,2,4,8,16}, (N,K) in {(4096,4096), (14336,4096),
+(4096,14336)}, bf16 activations N(0,1) with 1% of channels x50 quantized online
+(per-tensor amax, block scales, codes) and multiplied by pre-quantized NVFP4
+weights N(0,0.02).  One step = all 15 (M, shape) linear calls, each
+nvfp4_quantize + nvfp4_gemm.  Weights rotate through 4 copies per shape
+(302 MB) so each call streams its weights from HBM, not L2.
+
+value = aggregate algorithmic GB/s of a step (per call N*K*9/16 + M*K*(2+9/16)
++ 4*M*N bytes), device-timed with CUDA events around K graph-replayed steps.
+Multi-GPU: replicas only (the decode path has no data-path exchange); value is
+the bytes all ranks processed over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 linear µs/call & GB/s at M=1–16, TFLOP/s at M=8192; % of roofline"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled in the background."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            pass
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "100", *sel], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.15)
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                frac = float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                rows.append((ts + frac, float(parts[2]), float(parts[3]), parts[6:10]))
+            except Exception:
+                continue
+        os.unlink(self.f.name)
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.05 <= r[0] <= (self.t1 or 1e18) + 0.05]
+        use = inside or rows
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(inside), "samples_total": len(rows)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ decode workload
+
+def decode_bytes(M, N, K):
+    """Algorithmic bytes of one online-quantized linear call: W codes+scales, X bf16
+    read, X NVFP4 written/read once, Y fp32 written."""
+    return N * K * 9 // 16 + M * K * 2 + M * K * 9 // 16 + 4 * M * N
+
+
+def gemv_bytes(M, N, K):
+    return N * K * 9 // 16 + M * K * 9 // 16 + 4 * M * N
+
+
+class DecodeWorkload:
+    COPIES = 4
+
+    def __init__(self, dev):
+        import nvfp4_block_scaled_18_b200 as nv
+        from nvfp4_block_scaled_18_b200 import workloads as wl
+        self.nv, self.wl, self.dev = nv, wl, dev
+        self.shapes = list(wl.DECODE_SHAPES)
+        self.Ms = list(wl.DECODE_M)
+        self.calls = [(M, N, K) for M in self.Ms for (N, K) in self.shapes]
+        self.W = {}
+        for (N, K) in self.shapes:
+            w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
+            q0 = nv.NVFP4Tensor.empty(N, K, device=dev)
+            nv.nvfp4_quantize(w, q0, workspace=nv.Workspace(N, K, dev))
+            del w
+            copies = [q0]
+            for _ in range(self.COPIES - 1):
+                copies.append(nv.NVFP4Tensor(q0.codes.clone(), q0.scales.clone(), q0.tensor_scale.clone(), N, K))
+            self.W[(N, K)] = copies
+        self.X, self.Xhost, self.QX, self.WS, self.Y, self.Yhost = {}, {}, {}, {}, {}, {}
+        for M in self.Ms:
+            for K in sorted({k for _, k in self.shapes}):
+                x = wl.to_bf16(wl.decode_x(M, K))
+                self.Xhost[(M, K)] = x.pin_memory()
+                self.X[(M, K)] = x.to(dev)
+                self.QX[(M, K)] = nv.NVFP4Tensor.empty(M, K, device=dev)
+                self.WS[(M, K)] = nv.Workspace(M, K, dev)
+            for (N, K) in self.shapes:
+                self.Y[(M, N, K)] = torch.empty((M, N), dtype=torch.float32, device=dev)
+                self.Yhost[(M, N, K)] = torch.empty((M, N), dtype=torch.float32).pin_memory()
+        self.step_bytes = sum(decode_bytes(*c) for c in self.calls)
+        self.launches_per_step = 3 * len(self.calls)  # amax + quantize + GEMV per call
+        torch.cuda.synchronize()
+
+    def copy_index(self, step, i):
+        return ((step * len(self.calls) + i) // len(self.shapes)) % self.COPIES
+
+    def run_step(self, step, e2e=False):
+        nv = self.nv
+        for i, (M, N, K) in enumerate(self.calls):
+            if e2e:
+                self.X[(M, K)].copy_(self.Xhost[(M, K)], non_blocking=True)
+            nv.nvfp4_quantize(self.X[(M, K)], self.QX[(M, K)], workspace=self.WS[(M, K)])
+            nv.nvfp4_gemm(self.QX[(M, K)], self.W[(N, K)][self.copy_index(step, i)], self.Y[(M, N, K)])
+            if e2e:
+                self.Yhost[(M, N, K)].copy_(self.Y[(M, N, K)], non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(M * K * 2 for (M, N, K) in self.calls)
+
+    def d2h_bytes(self):
+        return sum(M * N * 4 for (M, N, K) in self.calls)
+
+
+def capture_graphs(wk, phases, e2e=False):
+    graphs = []
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for p in range(phases):      # eager warm-up of every phase (sets kernel attributes)
+            wk.run_step(p, e2e)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for p in range(phases):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            wk.run_step(p, e2e)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs
+
+
+def time_graphs(graphs, steps, warmup, world, sampler=None):
+    n = len(graphs)
+    for i in range(warmup):
+        graphs[i % n].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.mark_start()
+    start.record()
+    for i in range(steps):
+        graphs[i % n].replay()
+    end.record()
+    end.synchronize()
+    if sampler:
+        sampler.mark_end()
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(end)
+
+
+def time_gemv_launches(wk, reps=24):
+    """Per-launch device time of the GEMV kernel for every (M, shape), events
+    recorded inside a CUDA graph around each launch (weights rotating)."""
+    nv = wk.nv
+    out = {}
+    for (M, N, K) in wk.calls:
+        qx, y = wk.QX[(M, K)], wk.Y[(M, N, K)]
+        nv.nvfp4_quantize(wk.X[(M, K)], qx, workspace=wk.WS[(M, K)])
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            nv.nvfp4_gemm(qx, wk.W[(N, K)][0], y)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            for r in range(reps):
+                ev[r][0].record()
+                nv.nvfp4_gemm(qx, wk.W[(N, K)][r % wk.COPIES], y)
+                ev[r][1].record()
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(3):
+            g.replay()
+            torch.cuda.synchronize()
+            times += [a.elapsed_time(b) for a, b in ev[wk.COPIES:]]
+        out[(M, N, K)] = statistics.median(times)
+    return out
+
+
+# ------------------------------------------------------------ CPU baseline
+
+def cpu_oracle_sample(budget_s: float = 12.0, n_rows_w: int = 4096):
+    """Time the CPU oracle (as it stands) on the decode workload: (N,K)=(4096,4096),
+    M in {1,16}; quantize X online, fp64 GEMM on the dequantized operands."""
+    import oracle
+    from nvfp4_block_scaled_18_b200 import workloads as wl
+    oracle.build()
+    N, K = 4096, 4096
+    w = wl.weights_normal(N, K)
+    qw = oracle.quantize(w)
+    done_bytes, t_total, calls = 0, 0.0, 0
+    Ms = [1, 16]
+    t_start = time.perf_counter()
+    while time.perf_counter() - t_start < budget_s or calls < 2:
+        M = Ms[calls % 2]
+        x = wl.decode_x(M, K)
+        t0 = time.perf_counter()
+        qx = oracle.quantize(x)
+        oracle.gemm(qx, qw)
+        t_total += time.perf_counter() - t0
+        done_bytes += decode_bytes(M, N, K)
+        calls += 1
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {"value": round(done_bytes / t_total / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{calls} linear calls on (N,K)=(4096,4096), M alternating 1/16: oracle quantize "
+                      f"+ fp64 dequantized GEMM, {t_total:.1f} s"}
+
+
+def reference_arm(args):
+    """--impl reference: the CPU oracle timed as the comparison arm (rank 0 only)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import oracle
+    from nvfp4_block_scaled_18_b200 import workloads as wl
+    oracle.build()
+    budget = 150.0
+    per_step = max(0.02, min(1.0, budget / max(1, args.steps + args.warmup)))
+    shapes = list(wl.DECODE_SHAPES)
+    Ms = list(wl.DECODE_M)
+    cache = {}
+
+    def sample(i):
+        M, (N, K) = Ms[i % len(Ms)], shapes[(i // len(Ms)) % len(shapes)]
+        if (N, K) not in cache:
+            w = wl.weights_normal(N, K)
+            cache[(N, K)] = (oracle.quantize(w), w.shape[0])
+        qw, _ = cache[(N, K)]
+        # bound the work of a step: a row subset of W sized to the per-step budget
+        rows = max(8, min(N, int(per_step * 4e5 / max(1, K / 4096))))
+        sub = oracle.QTensor(qw.codes[:rows], qw.scales[:rows], qw.s)
+        x = wl.decode_x(M, K)
+        t0 = time.perf_counter()
+        oracle.gemm(oracle.quantize(x), sub)
+        return time.perf_counter() - t0, decode_bytes(M, rows, K)
+
+    for i in range(args.warmup):
+        sample(i)
+    t, b = 0.0, 0
+    for i in range(args.steps):
+        dt, db = sample(i)
+        t += dt
+        b += db
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    value = b / t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "decode GEMV, M=1..16, (N,K)=(4096,4096),(14336,4096),(4096,14336); "
+                                   "CPU oracle on a bounded row sample of W per step"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} steps, each one linear call on a W row subset"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    import nvfp4_block_scaled_18_b200 as nv
+    nv.load_library()
+    peaks = load_peaks()
+
+    wk = DecodeWorkload(dev)
+    phases = DecodeWorkload.COPIES
+    graphs = capture_graphs(wk, phases)
+    sampler = ClockSampler(torch.cuda.current_device())
+    ms = time_graphs(graphs, args.steps, args.warmup, world, sampler)
+    clocks = sampler.stop()
+    ms_max = max_over_ranks(ms, world)
+    total_bytes = sum_over_ranks(wk.step_bytes * args.steps, world)
+    value = total_bytes / (ms_max * 1e-3) / 1e9
+    ms_per_step = ms_max / args.steps
+
+    # end to end: pinned host X -> device, quantize + GEMV, Y -> pinned host, every step
+    e2e_steps = max(4 * phases, min(args.steps, 400))
+    e2e_graphs = capture_graphs(wk, phases, e2e=True)
+    ms_e2e = max_over_ranks(time_graphs(e2e_graphs, e2e_steps, args.warmup, world), world)
+    e2e_value = sum_over_ranks(wk.step_bytes * e2e_steps, world) / (ms_e2e * 1e-3) / 1e9
+
+    # per-launch GEMV timing for the roofline of the dominant kernel
+    per = time_gemv_launches(wk)
+    g_bytes = sum(gemv_bytes(*c) for c in wk.calls)
+    g_ms = sum(per.values())
+    achieved = g_bytes / (g_ms * 1e-3) / 1e9
+    detail = {f"M{M}_N{N}_K{K}": {"gemv_us": round(per[(M, N, K)] * 1e3, 3),
+                                  "gemv_GBps": round(gemv_bytes(M, N, K) / (per[(M, N, K)] * 1e-3) / 1e9, 1)}
+              for (M, N, K) in wk.calls}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "us_per_call": round(ms_per_step * 1e3 / len(wk.calls), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
+        "data": "synthetic",
+        "config": {"workload": "decode GEMV (M in 1,2,4,8,16; (N,K) in (4096,4096),(14336,4096),(4096,14336)); "
+                               "online bf16->NVFP4 activation quantization + CUDA-core NVFP4 GEMV, fp32 out",
+                   "calls_per_step": len(wk.calls), "l2": "weights rotate through 4 copies per shape (302 MB > L2)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                     "kernel": "k_gemv (all 15 decode launches)", "peak_source": peaks["source"]},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": wk.h2d_bytes(),
+                "d2h_bytes_per_step": wk.d2h_bytes()},
+        "gpu_launches": wk.launches_per_step * args.steps,
+        "clocks": clocks,
+        "detail": detail,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graphs, e2e_graphs
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,157 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 block-scaled W4A4 linear-layer
+ * library.
+ *
+ * NVFP4 (Replay the Curvature ... NVFP4 Quantization, abstract; ARCQuant blog
+ * post, section 1): a tensor of 4-bit E2M1 values in which every 16
+ * consecutive values along a row share one E4M3 block scale, under one FP32
+ * per-tensor scale.  An element decodes to v(code) * d(block) * s(tensor).
+ *
+ * Conventions for every entry point
+ *  - Pointers marked "device" are CUDA device (or managed) memory owned by the
+ *    caller; the library allocates nothing and keeps no state between calls
+ *    except the caller-owned workspace described below.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t, NULL = legacy default
+ *    stream).  A return of NVFP4_OK means the work was enqueued.
+ *  - Argument errors are detected on the host, before any launch, and returned
+ *    synchronously; nothing is enqueued then.
+ *  - Data-dependent errors (a NaN/Inf input, a device-side wait that timed out)
+ *    are written to `*dev_status` (device int, may be NULL) as an
+ *    nvfp4_status value; the first error written sticks.  Zero it before use.
+ *  - Row-major matrices; `ld*` arguments are row strides in elements.
+ *  - Activations and weights are quantized by the same entry points: weights
+ *    are simply quantized once, offline.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad enum value        */
+  NVFP4_ERR_ALIGNMENT = 2,   /* pointer or row stride not 16-byte aligned     */
+  NVFP4_ERR_UNSUPPORTED = 3, /* valid but not implemented shape/layout combo  */
+  NVFP4_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed             */
+  NVFP4_ERR_NONFINITE = 5,   /* device: an input element was NaN or Inf       */
+  NVFP4_ERR_TIMEOUT = 6,     /* device: a bounded wait gave up                */
+  NVFP4_ERR_WORKSPACE = 7    /* workspace missing or smaller than required    */
+} nvfp4_status;
+
+typedef enum { NVFP4_F32 = 0, NVFP4_BF16 = 1 } nvfp4_dtype;
+
+/* Block-scale storage.
+ *  ROWMAJOR: scale of (row r, block b) at byte r * (cols/16) + b.
+ *  TILED:    the 128-row x 4-block atom layout that tcgen05 block-scaled MMAs
+ *            consume: rows padded to a multiple of 128, blocks to a multiple
+ *            of 4; atom (rt, kt) = rows [128rt, 128rt+128) x blocks [4kt, 4kt+4)
+ *            starts at byte (rt * ceil(cols/64) + kt) * 512 and holds
+ *            (r, b) at (r % 32) * 16 + ((r / 32) % 4) * 4 + (b % 4).
+ *            Padding entries are never written: zero the buffer once after
+ *            allocating it. */
+typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_TILED = 1 } nvfp4_sf_layout;
+
+/* An NVFP4 matrix of rows x cols (cols a multiple of 16). */
+typedef struct {
+  uint8_t* codes;        /* device, rows x cols/2 bytes, row-major; element 2j of a
+                            row in the low nibble of byte j, element 2j+1 in the
+                            high nibble; nibble = sign(bit 3) | E2M1 magnitude   */
+  uint8_t* scales;       /* device, E4M3 block scales in sf_layout              */
+  float* tensor_scale;   /* device, one FP32 per-tensor scale                   */
+  int64_t rows;
+  int64_t cols;
+  nvfp4_sf_layout sf_layout;
+} nvfp4_tensor;
+
+/* Bytes of block-scale storage for a rows x cols NVFP4 matrix. */
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout);
+
+/* Bytes of workspace the quantizers need for an M x K input (RMSNorm variant
+ * included).  The workspace is device memory that must be zero-filled once
+ * after allocation; every successful call leaves it zero-filled again.  Calls
+ * sharing one workspace must be ordered (same stream).  After a call that
+ * reported an error through dev_status, zero it again. */
+size_t nvfp4_workspace_size(int64_t M, int64_t K);
+
+/* Quantize X (M x K, dtype dt, row stride ldx) to NVFP4 into q.
+ * Definition (ARCQuant post section 1; per-tensor scale as s_aug in section 3.1):
+ *   s = scale_in ? *scale_in : fl32(amax|X| / 2688)     (2688 = 6 * 448)
+ *   per 16-block: d = E4M3_RNE_satfinite(fl32(amax_block / fl32(6 s)))
+ *   per element:  code = E2M1_RNE_satfinite(fl32(x * fl32(1 / fl32(d s))))
+ *   (d = 0 or s < 2^-110 gives all-zero magnitudes).  *q->tensor_scale = s.
+ * x: device, 16-byte aligned, ldx * sizeof(dt) a multiple of 16; K % 16 == 0.
+ * q: rows == M, cols == K; codes 16-byte aligned.
+ * scale_in: device float or NULL (NULL = computed from X on the device).
+ * workspace: device, >= nvfp4_workspace_size(M, K) bytes (used when
+ *            scale_in == NULL).  */
+nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                            const float* scale_in, nvfp4_tensor* q, void* workspace,
+                            size_t ws_bytes, int* dev_status, void* stream);
+
+/* ResServe-style full residue (ResServe abstract: an FP4 activation base plus
+ * an FP4-quantized residue of what quantization lost):
+ *   q = Q(X) as nvfp4_quantize;  R = fl32(X - fl32(fl32(v d) s));
+ *   r = Q(R) with its own tensor scale s_R = rscale_in ? *rscale_in
+ *       : fl32(amax|R| / 2688).
+ * q and r are both M x K.  Other arguments as nvfp4_quantize. */
+nvfp4_status nvfp4_quantize_residue(const void* x, nvfp4_dtype dt, int64_t M, int64_t K,
+                                    int64_t ldx, const float* scale_in, const float* rscale_in,
+                                    nvfp4_tensor* q, nvfp4_tensor* r, void* workspace,
+                                    size_t ws_bytes, int* dev_status, void* stream);
+
+/* ARCQuant fused quantizer (ARCQuant post sections 3.1-3.2): RMSNorm, channel
+ * reorder, main quantization and residue quantization of the outlier channels
+ * in one pass, producing X_aug (M x (K+S)):
+ *   y[:,c]  = gamma ? fl32(fl32(x[:,c] * rinv_row) * gamma[c]) : x[:,c]
+ *             rinv_row = fl32(1 / sqrt(mean_row(x^2) + eps)), the mean square
+ *             formed exactly (squares truncated at 2^-34 of the row's largest
+ *             power of two, summed as integers, finished in binary64);
+ *   y'[:,j] = y[:, perm[j]]  (perm NULL = identity; outlier channels first);
+ *   s_aug   = scale_in ? *scale_in : fl32(amax|y'| / 2688);
+ *   X_aug[:, 0..K)    = Q(y') under s_aug;
+ *   X_aug[:, K..K+S)  = Q(y'[:, :S] - deq(Q(y'))[:, :S]) under the same s_aug.
+ * gamma: device, K elements of dtype dt, or NULL (no normalisation).
+ * perm: device int32[K], a permutation of 0..K-1, or NULL.
+ * S: 0 <= S <= K, S % 16 == 0.  x_aug: rows == M, cols == K + S.
+ * workspace: device, >= nvfp4_workspace_size(M, K) bytes. */
+nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K,
+                                            int64_t ldx, const void* gamma, float eps,
+                                            const int32_t* perm, int64_t S, const float* scale_in,
+                                            nvfp4_tensor* x_aug, void* workspace, size_t ws_bytes,
+                                            int* dev_status, void* stream);
+
+/* Block-scaled W4A4 linear: Y = s_a s_w * A W^T with A (M x K) and W (N x K)
+ * NVFP4, fp32 accumulation, output dtype out_dt (row stride ldy).
+ * ARCQuant's K -> K+S compensation is this call with K+S columns
+ * (ARCQuant post section 3.1-3.2: "unified GEMM call").
+ * Kernel choice: M <= 16 runs the CUDA-core decode GEMV (needs ROWMAJOR scales
+ * on both operands and K % 64 == 0); larger M runs the tcgen05 block-scaled
+ * tensor-core GEMM (needs TILED scales on both operands and K % 64 == 0).
+ * y: device, aligned to sizeof(out_dt), row stride ldy >= N elements. */
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y,
+                        nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
+
+/* ResServe compensated linear (ResServe abstract):
+ *   Y = s_a s_w * A W^T + s_r s_w * R W^T,
+ * both products accumulated on-chip and written once.  a and r are M x K,
+ * w is N x K.  Other conventions as nvfp4_gemm. */
+nvfp4_status nvfp4_gemm_residue(const nvfp4_tensor* a, const nvfp4_tensor* r,
+                                const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt, int64_t ldy,
+                                int* dev_status, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* nvfp4_status_string(nvfp4_status status);
+
+/* Library version and target, e.g. "nvfp4 0.1 sm_100a" (static string). */
+const char* nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

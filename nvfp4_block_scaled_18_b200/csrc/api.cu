@@ -1,0 +1,216 @@
+// C-ABI entry points declared in include/nvfp4.h: argument validation on the
+// host, then kernel launches on the caller's stream.  No allocation, no
+// global state beyond a per-device SM-count cache.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "nvfp4.h"
+
+using namespace nvfp4;
+
+namespace {
+
+int num_sms_current_device() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t dt_size(nvfp4_dtype dt) { return dt == NVFP4_BF16 ? 2 : 4; }
+inline bool dt_ok(nvfp4_dtype dt) { return dt == NVFP4_BF16 || dt == NVFP4_F32; }
+
+nvfp4_status check_input(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx) {
+  if (x == nullptr || !dt_ok(dt) || M <= 0 || K <= 0 || ldx < K) return NVFP4_ERR_INVALID_ARG;
+  if (K % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(x) || ((size_t)ldx * dt_size(dt)) % 16 != 0) return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+nvfp4_status check_tensor(const nvfp4_tensor* t, int64_t rows, int64_t cols) {
+  if (t == nullptr || t->codes == nullptr || t->scales == nullptr || t->tensor_scale == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (t->rows != rows || t->cols != cols || cols % 16 != 0 || rows <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (t->sf_layout != NVFP4_SF_ROWMAJOR && t->sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(t->codes) || !aligned16(t->scales) || (reinterpret_cast<uintptr_t>(t->tensor_scale) & 3u))
+    return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+QOut qout(const nvfp4_tensor* t) {
+  return QOut{t->codes, t->scales, t->tensor_scale, t->cols, t->sf_layout == NVFP4_SF_TILED};
+}
+
+nvfp4_status check_ws(const void* ws, size_t ws_bytes, int64_t M, int64_t K) {
+  if (ws == nullptr || ws_bytes < nvfp4_workspace_size(M, K)) return NVFP4_ERR_WORKSPACE;
+  if (!aligned16(ws)) return NVFP4_ERR_ALIGNMENT;
+  return NVFP4_OK;
+}
+
+inline nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+#define NVFP4_TRY(expr)                       \
+  do {                                        \
+    nvfp4_status _s = (expr);                 \
+    if (_s != NVFP4_OK) return _s;            \
+  } while (0)
+
+nvfp4_status check_gemm_operands(const nvfp4_tensor* a, const nvfp4_tensor* r, const nvfp4_tensor* w,
+                                 const void* y, nvfp4_dtype out_dt, int64_t ldy) {
+  if (a == nullptr || w == nullptr || y == nullptr || !dt_ok(out_dt)) return NVFP4_ERR_INVALID_ARG;
+  const int64_t M = a->rows, K = a->cols, N = w->rows;
+  NVFP4_TRY(check_tensor(a, M, K));
+  NVFP4_TRY(check_tensor(w, N, K));
+  if (r != nullptr) {
+    NVFP4_TRY(check_tensor(r, M, K));
+    if (r->sf_layout != a->sf_layout) return NVFP4_ERR_UNSUPPORTED;
+  }
+  if (ldy < N) return NVFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(y) % dt_size(out_dt)) != 0) return NVFP4_ERR_ALIGNMENT;
+  if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
+  return NVFP4_OK;
+}
+
+nvfp4_status run_gemm(const nvfp4_tensor* a, const nvfp4_tensor* r, const nvfp4_tensor* w, void* y,
+                      nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream) {
+  NVFP4_TRY(check_gemm_operands(a, r, w, y, out_dt, ldy));
+  GemmArgs g{};
+  g.a_codes = a->codes; g.a_scales = a->scales; g.a_s = a->tensor_scale;
+  if (r) { g.r_codes = r->codes; g.r_scales = r->scales; g.r_s = r->tensor_scale; }
+  g.w_codes = w->codes; g.w_scales = w->scales; g.w_s = w->tensor_scale;
+  g.y = y; g.ldy = ldy; g.y_bf16 = out_dt == NVFP4_BF16;
+  g.M = a->rows; g.N = w->rows; g.K = a->cols; g.st = dev_status;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (g.M <= 16) {
+    if (a->sf_layout != NVFP4_SF_ROWMAJOR || w->sf_layout != NVFP4_SF_ROWMAJOR)
+      return NVFP4_ERR_UNSUPPORTED;
+    return cuda_status(launch_gemv(g, num_sms_current_device(), s));
+  }
+  if (a->sf_layout != NVFP4_SF_TILED || w->sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_gemm_tc(g, num_sms_current_device(), s);
+  if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout) {
+  if (rows <= 0 || cols <= 0) return 0;
+  if (layout == NVFP4_SF_TILED) return (size_t)((rows + 127) / 128) * (size_t)((cols + 63) / 64) * 512;
+  return (size_t)rows * (size_t)((cols + 15) / 16);
+}
+
+size_t nvfp4_workspace_size(int64_t M, int64_t K) {
+  (void)K;
+  if (M <= 0) return kWsHeaderBytes;
+  return kWsHeaderBytes + (((size_t)M * 4 + 255) / 256) * 256;
+}
+
+nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                            const float* scale_in, nvfp4_tensor* q, void* workspace,
+                            size_t ws_bytes, int* dev_status, void* stream) {
+  NVFP4_TRY(check_input(x, dt, M, K, ldx));
+  NVFP4_TRY(check_tensor(q, M, K));
+  if (scale_in == nullptr) NVFP4_TRY(check_ws(workspace, ws_bytes, M, K));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = num_sms_current_device();
+  WsHeader* ws = static_cast<WsHeader*>(workspace);
+  const QOut qo = qout(q);
+  const float* s_ptr = scale_in;
+  if (s_ptr == nullptr) {
+    NVFP4_TRY(cuda_status(launch_amax(x, dt, M, K, ldx, ws, 0, q->tensor_scale, dev_status, sms, s)));
+    s_ptr = q->tensor_scale;
+  }
+  return cuda_status(launch_quant(Q_PLAIN, x, dt, M, K, ldx, s_ptr, nullptr, qo, qo, ws, dev_status, sms, s));
+}
+
+nvfp4_status nvfp4_quantize_residue(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                    const float* scale_in, const float* rscale_in, nvfp4_tensor* q,
+                                    nvfp4_tensor* r, void* workspace, size_t ws_bytes,
+                                    int* dev_status, void* stream) {
+  NVFP4_TRY(check_input(x, dt, M, K, ldx));
+  NVFP4_TRY(check_tensor(q, M, K));
+  NVFP4_TRY(check_tensor(r, M, K));
+  if (scale_in == nullptr || rscale_in == nullptr) NVFP4_TRY(check_ws(workspace, ws_bytes, M, K));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = num_sms_current_device();
+  WsHeader* ws = static_cast<WsHeader*>(workspace);
+  const QOut qo = qout(q), ro = qout(r);
+  const float* s_ptr = scale_in;
+  if (s_ptr == nullptr) {
+    NVFP4_TRY(cuda_status(launch_amax(x, dt, M, K, ldx, ws, 0, q->tensor_scale, dev_status, sms, s)));
+    s_ptr = q->tensor_scale;
+  }
+  if (rscale_in != nullptr)
+    return cuda_status(launch_quant(Q_BOTH, x, dt, M, K, ldx, s_ptr, rscale_in, qo, ro, ws, dev_status, sms, s));
+  NVFP4_TRY(cuda_status(launch_quant(Q_MAIN_AMAXR, x, dt, M, K, ldx, s_ptr, nullptr, qo, ro, ws, dev_status, sms, s)));
+  return cuda_status(launch_quant(Q_RES_ONLY, x, dt, M, K, ldx, s_ptr, r->tensor_scale, qo, ro, ws, dev_status, sms, s));
+}
+
+nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K,
+                                            int64_t ldx, const void* gamma, float eps,
+                                            const int32_t* perm, int64_t S, const float* scale_in,
+                                            nvfp4_tensor* x_aug, void* workspace, size_t ws_bytes,
+                                            int* dev_status, void* stream) {
+  NVFP4_TRY(check_input(x, dt, M, K, ldx));
+  if (S < 0 || S > K || S % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  NVFP4_TRY(check_tensor(x_aug, M, K + S));
+  if (gamma != nullptr && !aligned16(gamma)) return NVFP4_ERR_ALIGNMENT;
+  if (gamma != nullptr && !(eps >= 0.0f)) return NVFP4_ERR_INVALID_ARG;
+  if (gamma != nullptr || scale_in == nullptr) NVFP4_TRY(check_ws(workspace, ws_bytes, M, K));
+  if (reorder_smem_bytes(dt, K, gamma != nullptr) > 200 * 1024) return NVFP4_ERR_UNSUPPORTED;
+  if (K > 65536) return NVFP4_ERR_UNSUPPORTED;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = num_sms_current_device();
+  WsHeader* ws = static_cast<WsHeader*>(workspace);
+  float* rinv = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeaderBytes) : nullptr;
+  if (gamma != nullptr) {
+    NVFP4_TRY(cuda_status(launch_rms_stats(x, dt, M, K, ldx, gamma, eps, ws, rinv, x_aug->tensor_scale,
+                                           scale_in == nullptr, dev_status, sms, s)));
+  } else if (scale_in == nullptr) {
+    NVFP4_TRY(cuda_status(launch_amax(x, dt, M, K, ldx, ws, 0, x_aug->tensor_scale, dev_status, sms, s)));
+  }
+  const float* s_ptr = scale_in ? scale_in : x_aug->tensor_scale;
+  return cuda_status(launch_reorder_quant(x, dt, M, K, ldx, gamma, rinv, perm, S, s_ptr, qout(x_aug),
+                                          dev_status, sms, s));
+}
+
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt,
+                        int64_t ldy, int* dev_status, void* stream) {
+  return run_gemm(a, nullptr, w, y, out_dt, ldy, dev_status, stream);
+}
+
+nvfp4_status nvfp4_gemm_residue(const nvfp4_tensor* a, const nvfp4_tensor* r, const nvfp4_tensor* w,
+                                void* y, nvfp4_dtype out_dt, int64_t ldy, int* dev_status,
+                                void* stream) {
+  if (r == nullptr) return NVFP4_ERR_INVALID_ARG;
+  return run_gemm(a, r, w, y, out_dt, ldy, dev_status, stream);
+}
+
+const char* nvfp4_status_string(nvfp4_status st) {
+  switch (st) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported shape or layout";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_NONFINITE: return "non-finite input";
+    case NVFP4_ERR_TIMEOUT: return "device wait timed out";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* nvfp4_version(void) { return "nvfp4 0.1 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "nvfp4.h"
+
+namespace nvfp4 {
+
+struct WsHeader;
+
+// Output NVFP4 tensor as the quantizer kernels see it.
+struct QOut {
+  uint8_t* codes;
+  uint8_t* scales;
+  float* s;       // tensor scale (device)
+  int64_t cols;   // columns of the whole tensor (row pitch = cols/2 bytes of codes)
+  bool tiled;     // scale layout
+};
+
+enum QuantMode { Q_PLAIN = 0, Q_MAIN_AMAXR = 1, Q_RES_ONLY = 2, Q_BOTH = 3 };
+
+cudaError_t launch_amax(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                        WsHeader* ws, int slot, float* s_out, int* st, int num_sms,
+                        cudaStream_t stream);
+cudaError_t launch_quant(int mode, const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                         const float* s_ptr, const float* sr_ptr, const QOut& q, const QOut& r,
+                         WsHeader* ws, int* st, int num_sms, cudaStream_t stream);
+cudaError_t launch_rms_stats(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                             const void* gamma, float eps, WsHeader* ws, float* rinv, float* s_out,
+                             bool want_scale, int* st, int num_sms, cudaStream_t stream);
+size_t reorder_smem_bytes(nvfp4_dtype dt, int64_t K, bool has_gamma);
+cudaError_t launch_reorder_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                 const void* gamma, const float* rinv, const int32_t* perm,
+                                 int64_t S, const float* s_ptr, const QOut& q, int* st, int num_sms,
+                                 cudaStream_t stream);
+
+// Operands of the decode GEMV / tensor-core GEMM.
+struct GemmArgs {
+  const uint8_t* a_codes; const uint8_t* a_scales; const float* a_s;   // M x K
+  const uint8_t* r_codes; const uint8_t* r_scales; const float* r_s;   // M x K (residue) or null
+  const uint8_t* w_codes; const uint8_t* w_scales; const float* w_s;   // N x K
+  void* y; int64_t ldy; bool y_bf16;
+  int64_t M, N, K;
+  int* st;
+};
+
+cudaError_t launch_gemv(const GemmArgs& g, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);
+
+}  // namespace nvfp4

@@ -1,0 +1,388 @@
+// NVFP4 activation quantizers for sm_100a.
+//
+//  k_amax          per-tensor |x| maximum -> s = fl32(amax / 2688)      (tensor scale)
+//  k_quant         block amax, E4M3 block scale, E2M1 codes; optional
+//                  ResServe residue R = X - deq(Q(X)) with its own scale
+//  k_rms_stats     ARCQuant fused path, pass 1: exact per-row mean square,
+//                  rinv, and the tensor amax of the normalised rows
+//  k_reorder_quant ARCQuant fused path, pass 2: normalise, gather by the
+//                  channel permutation, quantize, append the outlier residue
+//
+// Sources: ARCQuant blog post (zizhi168.cn) sections 1 and 3.1-3.2 (format,
+// two-stage quantization, fused reorder/RMSNorm/quantize kernel, reorder
+// indices cached in shared memory); ResServe abstract (FP4 residue).
+//
+// Every rounding step uses an explicit _rn intrinsic so that no multiply-add
+// is contracted: the codes and scales are bit-identical to the definition in
+// include/nvfp4.h.  Thread mapping: one thread owns 8 consecutive elements
+// (one 16-byte bf16 vector); the two threads of an even/odd lane pair own one
+// 16-element block and exchange their half-block maxima with one shuffle.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+// Quantize the 8 values this thread owns (half of a 16-block; the partner lane
+// lane^1 owns the other half).  All 32 lanes must call it together.
+// Returns 8 packed E2M1 nibbles; d_byte receives the block's E4M3 scale; when
+// deq != nullptr it receives fl32(fl32(v(c) * d) * s) per element.
+__device__ __forceinline__ uint32_t quant_half_block(const float v[8], float s, uint32_t& d_byte,
+                                                     float* deq) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+  a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+  uint32_t db = 0;
+  if (s >= NVFP4_MIN_TENSOR_SCALE) db = f32_to_e4m3(__fdiv_rn(a, __fmul_rn(6.0f, s)));
+  const float d = e4m3_value(db);
+  const float inv = (d != 0.0f) ? __frcp_rn(__fmul_rn(d, s)) : 0.0f;
+  const uint32_t codes =
+      f32x8_to_e2m1(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
+                    __fmul_rn(v[3], inv), __fmul_rn(v[4], inv), __fmul_rn(v[5], inv),
+                    __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+  if (deq != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) deq[i] = __fmul_rn(__fmul_rn(e2m1_value(codes >> (4 * i)), d), s);
+  }
+  d_byte = db;
+  return codes;
+}
+
+__device__ __forceinline__ void store_half_block(const QOut& q, int64_t row, int64_t col8,
+                                                 uint32_t codes, uint32_t d_byte) {
+  *reinterpret_cast<uint32_t*>(q.codes + row * (q.cols >> 1) + col8 * 4) = codes;
+  if ((col8 & 1) == 0) q.scales[scale_offset(row, col8 >> 1, q.cols >> 4, q.tiled)] = (uint8_t)d_byte;
+}
+
+// Last-CTA-finishes reduction of a running |.| maximum into a tensor scale.
+// Every thread of every CTA calls it; `key` is the thread's local maximum.
+__device__ void finish_tensor_scale(uint32_t key, unsigned int* amax_cell, unsigned int* arrive,
+                                    float* s_out, int* st) {
+  __shared__ uint32_t red[32];
+  __shared__ bool last;
+  const uint32_t m = block_max_u32(key, red);
+  if (threadIdx.x == 0) {
+    if (m != 0u) atomicMax(amax_cell, m);
+    __threadfence();
+    const unsigned int total = gridDim.x * gridDim.y;
+    last = (atomicAdd(arrive, 1u) == total - 1u);
+  }
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t a = atomicAdd(amax_cell, 0u);
+    float s = 0.0f;
+    if (a >= 0x7F800000u) {
+      report_status(st, NVFP4_ERR_NONFINITE);
+    } else {
+      s = __fdiv_rn(__uint_as_float(a), 2688.0f);
+    }
+    *s_out = s;
+    *amax_cell = 0u;  // leave the workspace zeroed for the next call
+    *arrive = 0u;
+    __threadfence();
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_amax(const T* __restrict__ x, int64_t M, int64_t K,
+                                              int64_t ldx, WsHeader* ws, int slot, float* s_out,
+                                              int* st) {
+  const int64_t upr = K >> 3;
+  uint32_t key = 0;
+  for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
+    for (int64_t c8 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c8 < upr;
+         c8 += (int64_t)gridDim.x * blockDim.x) {
+      float v[8];
+      load8(x + row * ldx + c8 * 8, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
+    }
+  }
+  finish_tensor_scale(key, &ws->amax_bits[slot], &ws->arrive[slot], s_out, st);
+}
+
+template <typename T, int MODE>
+__global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t M, int64_t K,
+                                               int64_t ldx, const float* s_ptr,
+                                               const float* sr_ptr, QOut q, QOut r, WsHeader* ws,
+                                               int* st) {
+  const int64_t upr = K >> 3;
+  const float s = *s_ptr;
+  const float s_r = (MODE == Q_RES_ONLY || MODE == Q_BOTH) ? *sr_ptr : 0.0f;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    if (MODE != Q_RES_ONLY && q.s != s_ptr) *q.s = s;
+    if (MODE == Q_BOTH && r.s != sr_ptr) *r.s = s_r;
+  }
+  uint32_t bad = 0, rkey = 0;
+  for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < upr;
+         base += (int64_t)gridDim.x * blockDim.x) {
+      const int64_t c8 = base + threadIdx.x;
+      const bool act = c8 < upr;
+      float v[8];
+      if (act) {
+        load8(x + row * ldx + c8 * 8, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) bad = max(bad, abs_key(v[i]));
+      uint32_t db;
+      float deq[8];
+      const uint32_t codes = quant_half_block(v, s, db, MODE == Q_PLAIN ? nullptr : deq);
+      if (act && MODE != Q_RES_ONLY) store_half_block(q, row, c8, codes, db);
+      if (MODE != Q_PLAIN) {
+        float rv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rv[i] = __fsub_rn(v[i], deq[i]);
+        if (MODE == Q_MAIN_AMAXR) {
+          if (act) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) rkey = max(rkey, abs_key(rv[i]));
+          }
+        } else {
+          uint32_t dr;
+          const uint32_t rc = quant_half_block(rv, s_r, dr, nullptr);
+          if (act) store_half_block(r, row, c8, rc, dr);
+        }
+      }
+    }
+  }
+  if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
+  if (MODE == Q_MAIN_AMAXR) finish_tensor_scale(rkey, &ws->amax_bits[1], &ws->arrive[1], r.s, st);
+}
+
+// ----------------------------------------------------------- ARCQuant path
+
+// Binary64 power of two 2^e for -1022 <= e <= 1023.
+__device__ __forceinline__ double pow2_f64(int e) {
+  return __longlong_as_double((long long)(1023 + e) << 52);
+}
+
+// floor(log2(a)) for a finite positive fp32 bit pattern.
+__device__ __forceinline__ int ilog2_key(uint32_t key) {
+  return key >= 0x00800000u ? (int)(key >> 23) - 127 : (31 - __clz((int)key)) - 149;
+}
+
+// Pass 1, one CTA per row (grid-stride): rinv of the row and the running
+// maximum of |y| = |fl32(fl32(x * rinv) * gamma)| over the tensor.
+template <typename T>
+__global__ void __launch_bounds__(256) k_rms_stats(const T* __restrict__ x, int64_t M, int64_t K,
+                                                   int64_t ldx, const T* __restrict__ gamma,
+                                                   float eps, WsHeader* ws, float* rinv_out,
+                                                   float* s_out, bool want_scale, int* st) {
+  __shared__ uint32_t redu[32];
+  __shared__ double redd[32];
+  const int64_t upr = K >> 3;
+  uint32_t ykey = 0, bad = 0;
+  for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+    const T* xr = x + row * ldx;
+    uint32_t key = 0;
+    for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+      float v[8];
+      load8(xr + c8 * 8, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
+    }
+    key = block_max_u32(key, redu);
+    bad = max(bad, key);
+    double qsum = 0.0;
+    int e = 0;
+    if (key != 0u && key < 0x7F800000u) {
+      e = ilog2_key(key);
+      const double c = pow2_f64(17 - e);  // z = x * 2^(17-e), |z| < 2^18
+      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+        float v[8];
+        load8(xr + c8 * 8, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const double z = __dmul_rn((double)v[i], c);
+          qsum = __dadd_rn(qsum, floor(__dmul_rn(z, z)));
+        }
+      }
+    }
+    qsum = block_sum_f64(qsum, redd);  // exact: integers with total < 2^53
+    const double mean = __ddiv_rn(__dmul_rn(qsum, pow2_f64(2 * e - 34)), (double)K);
+    const float rinv = __double2float_rn(__drcp_rn(__dsqrt_rn(__dadd_rn(mean, (double)eps))));
+    if (threadIdx.x == 0) rinv_out[row] = rinv;
+    if (want_scale) {
+      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+        float v[8], g[8];
+        load8(xr + c8 * 8, v);
+        load8(gamma + c8 * 8, g);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ykey = max(ykey, abs_key(__fmul_rn(__fmul_rn(v[i], rinv), g[i])));
+      }
+    }
+  }
+  if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
+  if (want_scale) finish_tensor_scale(ykey, &ws->amax_bits[0], &ws->arrive[0], s_out, st);
+}
+
+// Pass 2, persistent CTAs looping over rows.  Shared memory holds the channel
+// permutation (loaded once per CTA), gamma, and the current row of x.
+template <typename T>
+__global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, int64_t M,
+                                                       int64_t K, int64_t ldx,
+                                                       const T* __restrict__ gamma,
+                                                       const float* __restrict__ rinv,
+                                                       const int32_t* __restrict__ perm, int64_t S,
+                                                       const float* s_ptr, QOut q, int* st) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int32_t* sperm = reinterpret_cast<int32_t*>(smem);
+  float* sgamma = reinterpret_cast<float*>(smem + K * 4);
+  T* srow = reinterpret_cast<T*>(smem + K * 4 + (gamma ? K * 4 : 0));
+  const float s = *s_ptr;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && q.s != s_ptr) *q.s = s;
+  for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
+    int32_t p = perm ? perm[k] : (int32_t)k;
+    if (p < 0 || (int64_t)p >= K) {  // not a permutation of 0..K-1: report, never index out of range
+      report_status(st, NVFP4_ERR_INVALID_ARG);
+      p = 0;
+    }
+    sperm[k] = p;
+    if (gamma) sgamma[k] = load1(gamma + k);
+  }
+  const int64_t upr = K >> 3;
+  const int64_t rupr = S >> 3;
+  uint32_t bad = 0;
+  for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+    __syncthreads();  // previous row fully consumed (and sperm/sgamma ready)
+    const T* xr = x + row * ldx;
+    for (int64_t c = threadIdx.x; c < (K * (int64_t)sizeof(T)) / 16; c += blockDim.x)
+      reinterpret_cast<uint4*>(srow)[c] = __ldg(reinterpret_cast<const uint4*>(xr) + c);
+    __syncthreads();
+    const float ri = gamma ? rinv[row] : 1.0f;
+    for (int64_t base = 0; base < upr; base += blockDim.x) {
+      const int64_t c8 = base + threadIdx.x;
+      const bool act = c8 < upr;
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float y = 0.0f;
+        if (act) {
+          const int32_t p = sperm[c8 * 8 + i];
+          y = load1(srow + p);
+          bad = max(bad, abs_key(y));
+          if (gamma) y = __fmul_rn(__fmul_rn(y, ri), sgamma[p]);
+        }
+        v[i] = y;
+      }
+      uint32_t db;
+      float deq[8];
+      const uint32_t codes = quant_half_block(v, s, db, deq);
+      if (act) store_half_block(q, row, c8, codes, db);
+      if (base < rupr) {  // uniform across the CTA: every lane takes part in the shuffle
+        float rv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rv[i] = __fsub_rn(v[i], deq[i]);
+        uint32_t dr;
+        const uint32_t rc = quant_half_block(rv, s, dr, nullptr);
+        if (c8 < rupr) store_half_block(q, row, upr + c8, rc, dr);
+      }
+    }
+  }
+  if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
+}
+
+// ------------------------------------------------------------ launchers
+
+static inline dim3 quant_grid(int64_t M, int64_t K, int num_sms) {
+  const int64_t upr = K >> 3;
+  const int64_t gx = std::min<int64_t>((upr + 255) / 256, 65535);
+  const int64_t target = (int64_t)num_sms * 8;
+  const int64_t gy = std::max<int64_t>(1, std::min<int64_t>({M, 65535, (target + gx - 1) / gx}));
+  return dim3((unsigned)gx, (unsigned)gy);
+}
+
+template <typename T>
+cudaError_t launch_amax_t(const void* x, int64_t M, int64_t K, int64_t ldx, WsHeader* ws, int slot,
+                          float* s_out, int* st, int num_sms, cudaStream_t stream) {
+  k_amax<T><<<quant_grid(M, K, num_sms), 256, 0, stream>>>(static_cast<const T*>(x), M, K, ldx, ws,
+                                                           slot, s_out, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                        WsHeader* ws, int slot, float* s_out, int* st, int num_sms,
+                        cudaStream_t stream) {
+  return dt == NVFP4_BF16
+             ? launch_amax_t<__nv_bfloat16>(x, M, K, ldx, ws, slot, s_out, st, num_sms, stream)
+             : launch_amax_t<float>(x, M, K, ldx, ws, slot, s_out, st, num_sms, stream);
+}
+
+template <typename T>
+cudaError_t launch_quant_t(int mode, const void* x, int64_t M, int64_t K, int64_t ldx,
+                           const float* s_ptr, const float* sr_ptr, const QOut& q, const QOut& r,
+                           WsHeader* ws, int* st, int num_sms, cudaStream_t stream) {
+  const dim3 g = quant_grid(M, K, num_sms);
+  const T* xp = static_cast<const T*>(x);
+  switch (mode) {
+    case Q_PLAIN: k_quant<T, Q_PLAIN><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
+    case Q_MAIN_AMAXR: k_quant<T, Q_MAIN_AMAXR><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
+    case Q_RES_ONLY: k_quant<T, Q_RES_ONLY><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
+    default: k_quant<T, Q_BOTH><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant(int mode, const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                         const float* s_ptr, const float* sr_ptr, const QOut& q, const QOut& r,
+                         WsHeader* ws, int* st, int num_sms, cudaStream_t stream) {
+  return dt == NVFP4_BF16
+             ? launch_quant_t<__nv_bfloat16>(mode, x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream)
+             : launch_quant_t<float>(mode, x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream);
+}
+
+template <typename T>
+cudaError_t launch_rms_stats_t(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                               float eps, WsHeader* ws, float* rinv, float* s_out, bool want_scale,
+                               int* st, int num_sms, cudaStream_t stream) {
+  const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * 8));
+  k_rms_stats<T><<<g, 256, 0, stream>>>(static_cast<const T*>(x), M, K, ldx,
+                                        static_cast<const T*>(gamma), eps, ws, rinv, s_out,
+                                        want_scale, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rms_stats(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                             const void* gamma, float eps, WsHeader* ws, float* rinv, float* s_out,
+                             bool want_scale, int* st, int num_sms, cudaStream_t stream) {
+  return dt == NVFP4_BF16
+             ? launch_rms_stats_t<__nv_bfloat16>(x, M, K, ldx, gamma, eps, ws, rinv, s_out, want_scale, st, num_sms, stream)
+             : launch_rms_stats_t<float>(x, M, K, ldx, gamma, eps, ws, rinv, s_out, want_scale, st, num_sms, stream);
+}
+
+size_t reorder_smem_bytes(nvfp4_dtype dt, int64_t K, bool has_gamma) {
+  return (size_t)K * 4 + (has_gamma ? (size_t)K * 4 : 0) + (size_t)K * (dt == NVFP4_BF16 ? 2 : 4);
+}
+
+template <typename T>
+cudaError_t launch_reorder_quant_t(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                                   const float* rinv, const int32_t* perm, int64_t S,
+                                   const float* s_ptr, const QOut& q, int* st, int num_sms,
+                                   cudaStream_t stream) {
+  const size_t smem = reorder_smem_bytes(sizeof(T) == 2 ? NVFP4_BF16 : NVFP4_F32, K, gamma != nullptr);
+  cudaError_t e = cudaFuncSetAttribute(k_reorder_quant<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int per_sm = smem <= 72 * 1024 ? 3 : (smem <= 110 * 1024 ? 2 : 1);
+  const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * per_sm));
+  k_reorder_quant<T><<<g, 256, smem, stream>>>(static_cast<const T*>(x), M, K, ldx,
+                                               static_cast<const T*>(gamma), rinv, perm, S, s_ptr,
+                                               q, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reorder_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                 const void* gamma, const float* rinv, const int32_t* perm,
+                                 int64_t S, const float* s_ptr, const QOut& q, int* st, int num_sms,
+                                 cudaStream_t stream) {
+  return dt == NVFP4_BF16
+             ? launch_reorder_quant_t<__nv_bfloat16>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms, stream)
+             : launch_reorder_quant_t<float>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms, stream);
+}
+
+}  // namespace nvfp4

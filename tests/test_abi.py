@@ -1,0 +1,74 @@
+"""The C-ABI library loads and exports every function include/nvfp4.h declares;
+host-side validation answers without touching a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_block_scaled_18_b200 as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_block_scaled_18_b200 import build
+    build.build()
+    return nv.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = header_functions()
+    assert len(names) >= 9
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(nv.EXPORTED_SYMBOLS)
+
+
+def test_host_only_queries(lib):
+    assert nv.nvfp4_version().startswith("nvfp4")
+    assert nv.nvfp4_scales_bytes(4, 256, nv.SF_ROWMAJOR) == 64
+    assert nv.nvfp4_scales_bytes(4, 256, nv.SF_TILED) == 4 * 512        # 1 row-atom x 4 k-atoms
+    assert nv.nvfp4_scales_bytes(129, 80, nv.SF_TILED) == 2 * 2 * 512
+    assert nv.nvfp4_workspace_size(1, 4096) >= 256
+    assert nv.nvfp4_workspace_size(2048, 4096) >= 256 + 4 * 2048
+    for code, name in nv.STATUS_NAMES.items():
+        assert isinstance(nv.status_string(code), str) and nv.status_string(code)
+
+
+def _tensor(rows, cols, codes=16, scales=16, ts=16, layout=0):
+    return nv._CTensor(codes, scales, ts, rows, cols, layout)
+
+
+def test_validation_before_launch(lib):
+    # fake, never-dereferenced device addresses: validation must reject before any CUDA call
+    good = 1 << 20
+    q = _tensor(4, 64, good, good, good)
+    f = lib.nvfp4_quantize
+    assert f(None, 1, 4, 64, 64, good, ctypes.byref(q), None, 0, None, None) == 1      # null x
+    assert f(good + 2, 1, 4, 64, 64, good, ctypes.byref(q), None, 0, None, None) == 2  # misaligned x
+    assert f(good, 1, 4, 60, 64, good, ctypes.byref(q), None, 0, None, None) == 1      # K % 16
+    assert f(good, 1, 4, 64, 68, good, ctypes.byref(q), None, 0, None, None) == 2      # ldx*2 % 16
+    assert f(good, 7, 4, 64, 64, good, ctypes.byref(q), None, 0, None, None) == 1      # bad dtype
+    bad_rows = _tensor(5, 64, good, good, good)
+    assert f(good, 1, 4, 64, 64, good, ctypes.byref(bad_rows), None, 0, None, None) == 1
+    assert f(good, 1, 4, 64, 64, None, ctypes.byref(q), None, 0, None, None) == 7      # no workspace
+    xa = _tensor(4, 64 + 16, good, good, good)
+    g = lib.nvfp4_rmsnorm_reorder_quantize
+    assert g(good, 1, 4, 64, 64, None, ctypes.c_float(1e-5), None, 8, good, ctypes.byref(xa), None, 0,
+             None, None) == 1                                                           # S % 16
+    a, w = _tensor(4, 64, good, good, good), _tensor(32, 64, good, good, good)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(w), None, 0, 32, None, None) == 1
+    w_bad = _tensor(32, 128, good, good, good)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(w_bad), good, 0, 32, None, None) == 1
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(w), good, 0, 30, None, None) == 1  # ldy < N
+    a_tiled = _tensor(4, 64, good, good, good, layout=1)
+    assert lib.nvfp4_gemm(ctypes.byref(a_tiled), ctypes.byref(w), good, 0, 32, None, None) == 3
+    assert lib.nvfp4_gemm_residue(ctypes.byref(a), None, ctypes.byref(w), good, 0, 32, None, None) == 1
