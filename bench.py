@@ -256,32 +256,24 @@ def time_graphs(graphs, steps, warmup, world, sampler=None):
 
 
 def time_gemv_launches(wk, reps=24):
-    """Per-launch device time of the GEMV kernel for every (M, shape), events
-    recorded inside a CUDA graph around each launch (weights rotating)."""
+    """Per-launch device time of the GEMV kernel for every (M, shape): CUDA events
+    around each launch on the launching stream, weights rotating.  The stream is
+    first held by a sleep kernel so that all event/launch triplets are queued
+    before any runs, and host launch gaps never enter the measured intervals."""
     nv = wk.nv
     out = {}
     for (M, N, K) in wk.calls:
         qx, y = wk.QX[(M, K)], wk.Y[(M, N, K)]
         nv.nvfp4_quantize(wk.X[(M, K)], qx, workspace=wk.WS[(M, K)])
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        g = torch.cuda.CUDAGraph()
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            nv.nvfp4_gemm(qx, wk.W[(N, K)][0], y)
-        torch.cuda.current_stream().wait_stream(s)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g):
+        times = []
+        for _ in range(3):
+            torch.cuda.synchronize()
+            torch.cuda._sleep(20_000_000)
             for r in range(reps):
                 ev[r][0].record()
                 nv.nvfp4_gemm(qx, wk.W[(N, K)][r % wk.COPIES], y)
                 ev[r][1].record()
-        for _ in range(2):
-            g.replay()
-        torch.cuda.synchronize()
-        times = []
-        for _ in range(3):
-            g.replay()
             torch.cuda.synchronize()
             times += [a.elapsed_time(b) for a, b in ev[wk.COPIES:]]
         out[(M, N, K)] = statistics.median(times)

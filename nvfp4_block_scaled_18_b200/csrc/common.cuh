@@ -103,6 +103,12 @@ __device__ __forceinline__ float load1(const __nv_bfloat16* p) {
 }
 __device__ __forceinline__ float load1(const float* p) { return *p; }
 
+// Two fp32 -> packed bf16x2 (round to nearest even); `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 // ------------------------------------------------------------ scale layout
 
 // Byte offset of block scale (row r, block b) of a matrix with nblk = cols/16 blocks.

@@ -1,9 +1,367 @@
-// tcgen05 block-scaled FP4 GEMM (large M).  Not built yet: the entry point
-// reports "not supported" so nvfp4_gemm returns NVFP4_ERR_UNSUPPORTED.
+// Large-M NVFP4 W4A4 GEMM on the 5th-generation tensor cores (tcgen05), sm_100a.
+//
+// Y = s_a s_w * A W^T with A (M x K) and W (N x K) NVFP4, both K-major with
+// block scales in the 128-row x 4-block atom layout (NVFP4_SF_TILED).  Each
+// tcgen05.mma.kind::mxf4nvf4.block_scale.block16 multiplies a 128 x 64 slice of
+// A by a 256 x 64 slice of W, applying one E4M3 scale per 16 elements of both
+// operands, and accumulates in fp32 in tensor memory.  ARCQuant's K -> K+S
+// compensation (ARCQuant blog post, section 3.1-3.2: one GEMM over the
+// augmented K) runs through this kernel unchanged.
+//
+// Structure (persistent, one CTA per SM, 192 threads):
+//   warp 0     one lane issues TMA loads of A/W code tiles (128 B K-slices,
+//              128-byte swizzle) and bulk copies of the matching scale atoms
+//              into a 4-stage shared-memory ring;
+//   warp 1     allocates 512 TMEM columns; one lane copies each stage's scale
+//              atoms into TMEM (tcgen05.cp 32x128b.warpx4) and issues 4 MMAs
+//              (K = 64 each) per stage; tcgen05.commit frees the stage and, at
+//              the end of a tile, signals the epilogue;
+//   warps 2-5  read the 128 x 256 fp32 accumulator (tcgen05.ld 32x32b.x32, one
+//              TMEM lane quadrant per warp), scale by s_a s_w and store Y.
+// Tiles are 128 x 256 x 256 (M x N x K); tile order walks M fastest so that the
+// CTAs in flight share W tiles through L2.  Every mbarrier wait is bounded: on
+// timeout the kernel records NVFP4_ERR_TIMEOUT, every role leaves its loop, and
+// TMEM is still released.
+#include <cuda.h>
+
+#include "common.cuh"
 #include "kernels.h"
 
 namespace nvfp4 {
+namespace {
 
-cudaError_t launch_gemm_tc(const GemmArgs&, int, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int BM = 128, BN = 256, BK = 256;
+constexpr int BK_BYTES = BK / 2;                 // one 128-byte swizzle row per k-tile
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK_BYTES;           // 16 KB
+constexpr int B_BYTES = BN * BK_BYTES;           // 32 KB
+constexpr int SFA_BYTES = 4 * 512;               // 4 k-atoms of one 128-row group
+constexpr int SFB_BYTES = 2 * 4 * 512;           // 2 row groups x 4 k-atoms
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
+constexpr int OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;    // + alignment slack
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;                  // 256 fp32 columns
+constexpr uint32_t SFA_COL = 256;                // 4 k-blocks x 4 columns
+constexpr uint32_t SFB_COL = 272;                // 4 k-blocks x 8 columns
+constexpr int NUM_THREADS = 192;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+
+static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for 128B swizzle");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct TcParams {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const float* a_s;
+  const float* w_s;
+  void* y;
+  int64_t ldy;
+  int y_bf16;
+  int M, N, K;
+  int katoms;      // scale atoms along K per 128-row group = ceil(K / 64)
+  int b_groups;    // 128-row groups of W = ceil(N / 128)
+  int m_blocks, n_blocks, num_tiles, k_tiles;
+  int* st;
+};
+
+// ----------------------------------------------------------------- PTX
+
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when this or another role gave up.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* st) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      *abort_flag = 1;
+      report_status(st, NVFP4_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_cp_scales(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand tile, 128-byte swizzle,
+// 8-row groups 1024 bytes apart (sm_100 descriptor version 1).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Descriptor of one 512-byte scale atom (32 rows of 16 bytes, no swizzle) as
+// the tcgen05.cp source.
+__device__ __forceinline__ uint64_t desc_sf_atom(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(512 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
+         ((uint64_t)1 << 46);
+}
+// Instruction descriptor: kind::mxf4nvf4, A and B E2M1, K-major, UE4M3 scales,
+// fp32 accumulator, M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc_nvf4(int n) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// --------------------------------------------------------------- kernel
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const TcParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;               // [STAGES] TMA -> MMA
+  uint64_t* empty = bars + STAGES;     // [STAGES] MMA -> TMA
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(saddr(&full[s]), 1);
+      mbar_init(saddr(&empty[s]), 1);
+    }
+    mbar_init(saddr(acc_full), 1);
+    mbar_init(saddr(acc_empty), 4);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer
+    int s = 0;
+    uint32_t ph = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
+      const int ngroups = min(2, p.b_groups - nb * 2);
+      for (int kt = 0; kt < p.k_tiles; ++kt) {
+        if (!mbar_wait(saddr(&empty[s]), ph ^ 1u, abort_flag, p.st)) goto producer_done;
+        const int jmax = min(4, (p.K - kt * BK) / 64);
+        const uint32_t sf_bytes = (uint32_t)jmax * 512u;
+        const uint32_t bar = saddr(&full[s]);
+        uint8_t* st_base = smem + s * STAGE_BYTES;
+        mbar_expect_tx(bar, A_BYTES + B_BYTES + sf_bytes * (1 + ngroups));
+        tma_load_2d(saddr(st_base), &tmA, kt * BK_BYTES, mb * BM, bar);
+        tma_load_2d(saddr(st_base + OFF_B), &tmB, kt * BK_BYTES, nb * BN, bar);
+        bulk_load(saddr(st_base + OFF_SFA), p.sfa + ((size_t)mb * p.katoms + kt * 4) * 512, sf_bytes, bar);
+        for (int g = 0; g < ngroups; ++g)
+          bulk_load(saddr(st_base + OFF_SFB + g * 2048),
+                    p.sfb + ((size_t)(nb * 2 + g) * p.katoms + kt * 4) * 512, sf_bytes, bar);
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+    }
+  producer_done:;
+  } else if (warp == 1 && lane == 0) {
+    // -------------------------------------------------------- MMA issuer
+    const uint32_t idesc = idesc_nvf4(BN);
+    int s = 0;
+    uint32_t ph = 0;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+      const int nb = tile / p.m_blocks;
+      const int ngroups = min(2, p.b_groups - nb * 2);
+      if (!mbar_wait(saddr(acc_empty), (uint32_t)(local & 1) ^ 1u, abort_flag, p.st)) break;
+      tc_fence_after();
+      for (int kt = 0; kt < p.k_tiles; ++kt) {
+        if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) goto mma_done;
+        tc_fence_after();
+        const int jmax = min(4, (p.K - kt * BK) / 64);
+        const uint8_t* st_base = smem + s * STAGE_BYTES;
+        const uint32_t a0 = saddr(st_base), b0 = saddr(st_base + OFF_B);
+        for (int j = 0; j < jmax; ++j) {
+          tc_cp_scales(tmem + SFA_COL + 4 * j, desc_sf_atom(saddr(st_base + OFF_SFA + j * 512)));
+          for (int g = 0; g < ngroups; ++g)
+            tc_cp_scales(tmem + SFB_COL + 8 * j + 4 * g,
+                         desc_sf_atom(saddr(st_base + OFF_SFB + g * 2048 + j * 512)));
+        }
+        for (int j = 0; j < jmax; ++j) {
+          tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a0) + (uint64_t)(2 * j), desc_sw128(b0) + (uint64_t)(2 * j),
+                      idesc, tmem + SFA_COL + 4 * j, tmem + SFB_COL + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+        }
+        tc_commit(saddr(&empty[s]));  // stage reusable once these MMAs have read it
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+      tc_commit(saddr(acc_full));     // accumulator complete
+    }
+  mma_done:;
+  } else if (warp >= 2) {
+    // ----------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    int local = 0;
+    const float alpha = (*p.a_s) * (*p.w_s);
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+      const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
+      if (!mbar_wait(saddr(acc_full), (uint32_t)(local & 1), abort_flag, p.st)) break;
+      tc_fence_after();
+      const int row = mb * BM + q * 32 + lane;
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + c * 32, r);
+        tmem_ld_wait();
+        const int col0 = nb * BN + c * 32;
+        if (row >= p.M || col0 >= p.N) continue;
+        if (p.y_bf16) {
+          __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (int64_t)row * p.ldy + col0;
+          const bool vec = col0 + 32 <= p.N && ((reinterpret_cast<uintptr_t>(yr) & 15u) == 0);
+          if (vec) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(r[i]) * alpha, __uint_as_float(r[i + 1]) * alpha);
+              v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * alpha, __uint_as_float(r[i + 3]) * alpha);
+              v.z = pack_bf16x2(__uint_as_float(r[i + 4]) * alpha, __uint_as_float(r[i + 5]) * alpha);
+              v.w = pack_bf16x2(__uint_as_float(r[i + 6]) * alpha, __uint_as_float(r[i + 7]) * alpha);
+              *reinterpret_cast<uint4*>(yr + i) = v;
+            }
+          } else {
+            for (int i = 0; i < 32 && col0 + i < p.N; ++i) yr[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * alpha);
+          }
+        } else {
+          float* yr = reinterpret_cast<float*>(p.y) + (int64_t)row * p.ldy + col0;
+          const bool vec = col0 + 32 <= p.N && ((reinterpret_cast<uintptr_t>(yr) & 15u) == 0);
+          if (vec) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(yr + i) =
+                  make_float4(__uint_as_float(r[i]) * alpha, __uint_as_float(r[i + 1]) * alpha,
+                              __uint_as_float(r[i + 2]) * alpha, __uint_as_float(r[i + 3]) * alpha);
+          } else {
+            for (int i = 0; i < 32 && col0 + i < p.N; ++i) yr[i] = __uint_as_float(r[i]) * alpha;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(saddr(acc_empty));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)BK_BYTES, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return cuTensorMapEncodeTiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims,
+                                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) {
+  if (g.r_codes != nullptr) return cudaErrorNotSupported;  // own-scale residue: small-M paths only
+  if (g.K % 64 != 0 || g.K < BK) return cudaErrorNotSupported;
+  CUtensorMap tmA, tmB;
+  if (!encode_codes_map(&tmA, g.a_codes, g.M, g.K, BM) || !encode_codes_map(&tmB, g.w_codes, g.N, g.K, BN))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.sfa = g.a_scales; p.sfb = g.w_scales; p.a_s = g.a_s; p.w_s = g.w_s;
+  p.y = g.y; p.ldy = g.ldy; p.y_bf16 = g.y_bf16 ? 1 : 0;
+  p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K;
+  p.katoms = (int)((g.K + 63) / 64);
+  p.b_groups = (int)((g.N + 127) / 128);
+  p.m_blocks = (int)((g.M + BM - 1) / BM);
+  p.n_blocks = (int)((g.N + BN - 1) / BN);
+  p.num_tiles = p.m_blocks * p.n_blocks;
+  p.k_tiles = (int)((g.K + BK - 1) / BK);
+  p.st = g.st;
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_nvf4, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int grid = std::max(1, std::min(p.num_tiles, num_sms));
+  k_gemm_nvf4<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+  return cudaGetLastError();
+}
 
 }  // namespace nvfp4

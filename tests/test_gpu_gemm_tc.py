@@ -1,0 +1,165 @@
+"""GPU parity: the tcgen05 block-scaled GEMM (M > 16, TILED scales) against the
+fp64 oracle on the same quantized operands, relative Frobenius error <= 1e-5.
+
+One-hot operands pin the code/scale placement (tile rows, TMEM lane quadrants,
+k-blocks inside a k-tile, both 128-row groups of a 256-wide W tile); ragged
+shapes exercise the M, N and K tails; the large configurations are checked on
+sampled rows and columns that the oracle evaluates."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_block_scaled_18_b200 as nv
+from nvfp4_block_scaled_18_b200 import workloads as wl
+
+from gpu_util import REL_FRO_TOL, assert_same_q, rel_fro, run_quantize, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    nv.load_library()
+
+
+def tiled_from_rowmajor(scales: np.ndarray) -> np.ndarray:
+    """Place row-major block scales (rows x nb) into the TILED atom layout (layout only)."""
+    rows, nb = scales.shape
+    katoms = (nb + 3) // 4
+    out = np.zeros(((rows + 127) // 128) * katoms * 512, np.uint8)
+    r = np.arange(rows)[:, None]
+    b = np.arange(nb)[None, :]
+    off = ((r // 128) * katoms + b // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + (b % 4)
+    out[off] = scales
+    return out
+
+
+def gpu_tensor(codes, scales_rowmajor, s, layout=nv.SF_TILED):
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    sc = tiled_from_rowmajor(scales_rowmajor) if layout == nv.SF_TILED else scales_rowmajor.reshape(-1)
+    return nv.NVFP4Tensor(torch.from_numpy(np.ascontiguousarray(codes)).cuda(), torch.from_numpy(sc).cuda(),
+                          torch.tensor([s], dtype=torch.float32, device="cuda"), rows, cols, layout)
+
+
+def run_gemm(a, w, out_dtype=torch.float32):
+    y = torch.full((a.rows, w.rows), float("nan"), dtype=out_dtype, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_gemm(a, w, y, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, nv.status_string(st.item())
+    return y
+
+
+@pytest.mark.parametrize("m,n,k", [(0, 0, 0), (33, 131, 17), (77, 255, 95), (127, 128, 130), (64, 200, 255),
+                                   (5, 17, 64), (96, 250, 191)])
+def test_one_hot_placement(orc, m, n, k):
+    M, N, K = 128, 256, 256
+    ca = np.zeros((M, K // 2), np.uint8)
+    cw = np.zeros((N, K // 2), np.uint8)
+    sa = np.zeros((M, K // 16), np.uint8)
+    sw = np.zeros((N, K // 16), np.uint8)
+    ca[m, k // 2] = 0x7 << (4 * (k & 1))      # +6
+    cw[n, k // 2] = 0xB << (4 * (k & 1))      # -1.5
+    sa[m, k // 16] = 0x40                     # 2.0
+    sw[n, k // 16] = 0x31                     # 0.5625
+    # decoys: other blocks of the same rows carry different scales and zero codes
+    sa[m, (k // 16 + 1) % 16] = 0x7E
+    sw[n, (k // 16 + 3) % 16] = 0x7E
+    a, w = gpu_tensor(ca, sa, 0.5), gpu_tensor(cw, sw, 0.25)
+    y = run_gemm(a, w).cpu().numpy()
+    expect = np.zeros((M, N))
+    expect[m, n] = 6 * 2.0 * 0.5 * (-1.5) * 0.5625 * 0.25
+    np.testing.assert_array_equal(y, expect)
+    ref = orc.gemm(orc.QTensor(ca, sa, 0.5), orc.QTensor(cw, sw, 0.25))
+    np.testing.assert_array_equal(ref, expect)
+
+
+def _random_case(orc, M, N, K, seed, out_dtype=torch.float32):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((M, K)) * 2).astype(np.float32)
+    x[:, rng.choice(K, max(1, K // 64), replace=False)] *= 30
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    qa = run_quantize(to_dev(x, torch.float32), nv.SF_TILED)
+    qw = run_quantize(to_dev(w, torch.float32), nv.SF_TILED)
+    y = run_gemm(qa, qw, out_dtype)
+    return y, orc.gemm(orc.quantize(x), orc.quantize(w))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (256, 512, 1024), (200, 300, 320), (129, 1000, 4224),
+                                   (17, 64, 256), (1000, 130, 576), (384, 768, 2048)])
+def test_random_shapes(orc, M, N, K):
+    y, ref = _random_case(orc, M, N, K, M + N + K)
+    err = rel_fro(y.cpu().numpy(), ref)
+    assert err <= REL_FRO_TOL, err
+
+
+def test_bf16_output(orc):
+    y, ref = _random_case(orc, 256, 512, 512, 5, torch.bfloat16)
+    y = y.float().cpu().numpy()
+    assert np.all(np.abs(y - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)
+
+
+def test_exact_sums_exact(orc):
+    """Power-of-two tensor scales and scales in [0.5, 2): every partial sum of a
+    K = 256 product is a small multiple of 2^-8, so the fp32 result must be exact."""
+    M, N, K = 128, 256, 256
+    rng = np.random.default_rng(9)
+    ca = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    cw = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sa = rng.integers(0x30, 0x40, (M, K // 16), dtype=np.uint8)
+    sw = rng.integers(0x30, 0x40, (N, K // 16), dtype=np.uint8)
+    y = run_gemm(gpu_tensor(ca, sa, 0.5), gpu_tensor(cw, sw, 0.25)).cpu().numpy().astype(np.float64)
+    ref = orc.gemm(orc.QTensor(ca, sa, 0.5), orc.QTensor(cw, sw, 0.25))
+    np.testing.assert_array_equal(y, ref)
+
+
+def _sampled_check(orc, x, w, qa, qw, n_rows=96, n_cols=384, seed=0):
+    """Compare Y on a sample of rows and columns, the oracle quantizing only those
+    rows of X and W (under the full tensors' scales, so they are bit-identical)."""
+    M, N = x.shape[0], w.shape[0]
+    y = run_gemm(qa, qw)
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, n_rows, replace=False)]))
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, n_cols, replace=False)]))
+    ox = orc.quantize(x[rows], orc.tensor_scale(np.abs(x).max()))
+    ow = orc.quantize(w[cols], orc.tensor_scale(np.abs(w).max()))
+    ys = y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].cpu().numpy()
+    err = rel_fro(ys, orc.gemm(ox, ow))
+    assert err <= REL_FRO_TOL, err
+    return err
+
+
+@pytest.mark.parametrize("N,K", wl.PREFILL_SHAPES)
+def test_large_prefill_sampled(orc, N, K):
+    M = wl.PREFILL_M
+    x = wl.prefill_x(M, K)
+    w = wl.weights_normal(N, K)
+    qa = run_quantize(to_dev(x), nv.SF_TILED)
+    qw = run_quantize(to_dev(w, torch.float32), nv.SF_TILED)
+    _sampled_check(orc, x, w, qa, qw)
+
+
+@pytest.mark.parametrize("S", [128, 256, 512])
+def test_arcquant_augmented_gemm(orc, S):
+    """ARCQuant: fused quantizer to X_aug (K+S) and W_aug = [W' | W'_o], one GEMM."""
+    x, gamma, perm = wl.arc_inputs()
+    M, K = x.shape
+    N = wl.ARC_N
+    w = wl.weights_normal(N, K)
+    xa = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED)
+    nv.nvfp4_rmsnorm_reorder_quantize(to_dev(x), xa, gamma=to_dev(gamma), eps=1e-5,
+                                      perm=torch.from_numpy(perm).cuda(), S=S, workspace=nv.Workspace(M, K))
+    w_aug = orc.augment_weight(w, perm, S)
+    qw = run_quantize(to_dev(w_aug, torch.float32), nv.SF_TILED)
+    y = run_gemm(xa, qw)
+    rng = np.random.default_rng(S)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 64, replace=False)]))
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 256, replace=False)]))
+    ref_xa = orc.rmsnorm_reorder_quantize(x, gamma, 1e-5, perm, S)
+    assert_same_q(xa, ref_xa)
+    ox = orc.QTensor(ref_xa.codes[rows], ref_xa.scales[rows], ref_xa.s)
+    ow = orc.quantize(w_aug[cols], orc.tensor_scale(np.abs(w_aug).max()))
+    ys = y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].cpu().numpy()
+    err = rel_fro(ys, orc.gemm(ox, ow))
+    assert err <= REL_FRO_TOL, err
