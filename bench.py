@@ -280,14 +280,168 @@ def time_gemv_launches(wk, reps=24):
     return out
 
 
+# ------------------------------------------------------------ prefill workload
+
+def fp4_peak_tflops(peaks, sustained=False):
+    """Dense FP4 peak: the measured bf16 GEMM peak x 4 (nominal 9 / 2.25 PFLOP/s)."""
+    return 4.0 * (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
+
+
+class PrefillWorkload:
+    """Large prefill W4A4: M = 8192, (N,K) in {(14336,4096), (4096,14336), (28672,8192)},
+    bf16 N(0,1) activations with 1% channels x50 quantized online (TILED scales),
+    each shape with and without the S = 256 outlier-residue K extension
+    (reorder + residue quantizer with no normalisation, W_aug of K+S columns)."""
+
+    S = 256
+
+    def __init__(self, dev):
+        import nvfp4_block_scaled_18_b200 as nv
+        from nvfp4_block_scaled_18_b200 import workloads as wl
+        self.nv, self.dev = nv, dev
+        self.M = wl.PREFILL_M
+        self.shapes = list(wl.PREFILL_SHAPES)
+        self.calls = []   # (name, M, N, Keff, S)
+        self.buf = {}
+        g = torch.Generator(device="cpu").manual_seed(0)
+        for (N, K) in self.shapes:
+            x = wl.to_bf16(wl.prefill_x(self.M, K)).to(dev)
+            perm = torch.from_numpy(wl.calibrated_perm(wl.prefill_x(64, K))).to(dev)
+            w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
+            qw = nv.NVFP4Tensor.empty(N, K, nv.SF_TILED, device=dev)
+            nv.nvfp4_quantize(w, qw, workspace=nv.Workspace(N, K, dev))
+            w_aug = torch.cat([w[:, perm.long()], w[:, perm[: self.S].long()]], dim=1).contiguous()
+            del w
+            qwa = nv.NVFP4Tensor.empty(N, K + self.S, nv.SF_TILED, device=dev)
+            nv.nvfp4_quantize(w_aug, qwa, workspace=nv.Workspace(N, K + self.S, dev))
+            del w_aug
+            self.buf[(N, K)] = dict(
+                x=x, perm=perm, qw=qw, qwa=qwa,
+                qx=nv.NVFP4Tensor.empty(self.M, K, nv.SF_TILED, device=dev),
+                qxa=nv.NVFP4Tensor.empty(self.M, K + self.S, nv.SF_TILED, device=dev),
+                ws=nv.Workspace(self.M, K, dev),
+                y=torch.empty((self.M, N), dtype=torch.float32, device=dev))
+            self.calls.append(("plain", self.M, N, K, 0))
+            self.calls.append(("k+s", self.M, N, K + self.S, self.S))
+        torch.cuda.synchronize()
+
+    def quantize(self, N, K, S):
+        b = self.buf[(N, K)]
+        if S == 0:
+            self.nv.nvfp4_quantize(b["x"], b["qx"], workspace=b["ws"])
+        else:
+            self.nv.nvfp4_rmsnorm_reorder_quantize(b["x"], b["qxa"], perm=b["perm"], S=S, workspace=b["ws"])
+
+    def gemm(self, N, K, S):
+        b = self.buf[(N, K)]
+        self.nv.nvfp4_gemm(b["qxa"] if S else b["qx"], b["qwa"] if S else b["qw"], b["y"])
+
+    def run_step(self, step=0, e2e=False):
+        for (_, M, N, Keff, S) in self.calls:
+            K = Keff - S
+            self.quantize(N, K, S)
+            self.gemm(N, K, S)
+
+    def h2d_bytes(self):
+        return sum(M * (Keff - S) * 2 for (_, M, N, Keff, S) in self.calls)
+
+    def d2h_bytes(self):
+        return sum(M * N * 4 for (_, M, N, Keff, S) in self.calls)
+
+
+def prefill_e2e(wk, steps):
+    """End-to-end prefill step time (ms): each call's X copied from pinned host
+    memory, quantized, multiplied, and Y copied back to pinned host memory."""
+    host_x = {k: b["x"].cpu().pin_memory() for k, b in wk.buf.items()}
+    host_y = {k: torch.empty(b["y"].shape, dtype=torch.float32).pin_memory() for k, b in wk.buf.items()}
+
+    def step():
+        for (_, M, N, Keff, S) in wk.calls:
+            K = Keff - S
+            b = wk.buf[(N, K)]
+            b["x"].copy_(host_x[(N, K)], non_blocking=True)
+            wk.quantize(N, K, S)
+            wk.gemm(N, K, S)
+            host_y[(N, K)].copy_(b["y"], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+def time_launches(fn, reps=8, rounds=3):
+    """Median device time (ms) of fn() launches: CUDA events around each launch,
+    all queued behind a sleep kernel so host gaps never enter the intervals."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    fn()
+    times = []
+    for _ in range(rounds):
+        torch.cuda.synchronize()
+        torch.cuda._sleep(20_000_000)
+        for r in range(reps):
+            ev[r][0].record()
+            fn()
+            ev[r][1].record()
+        torch.cuda.synchronize()
+        times += [a.elapsed_time(b) for a, b in ev]
+    return statistics.median(times)
+
+
+def measure_prefill_from(wk, peaks):
+    """Per-launch GEMM and quantizer times on the prefill workload."""
+    out, flops_total, gemm_ms_total = {}, 0.0, 0.0
+    for (name, M, N, Keff, S) in wk.calls:
+        K = Keff - S
+        wk.quantize(N, K, S)
+        g_ms = time_launches(lambda: wk.gemm(N, K, S))
+        q_ms = time_launches(lambda: wk.quantize(N, K, S))
+        flops = 2.0 * M * N * Keff
+        q_bytes = 2 * M * K + M * Keff * 9 // 16
+        flops_total += flops
+        gemm_ms_total += g_ms
+        out[f"M{M}_N{N}_K{K}" + (f"+S{S}" if S else "")] = {
+            "gemm_us": round(g_ms * 1e3, 2), "gemm_TFLOPs": round(flops / (g_ms * 1e-3) / 1e12, 1),
+            "gemm_frac_fp4_peak": round(flops / (g_ms * 1e-3) / 1e12 / fp4_peak_tflops(peaks), 4),
+            "quant_us": round(q_ms * 1e3, 2), "quant_GBps": round(q_bytes / (q_ms * 1e-3) / 1e9, 1)}
+    achieved = flops_total / (gemm_ms_total * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak_tflops(peaks), 1),
+            "unit": "TFLOP/s", "frac": round(achieved / fp4_peak_tflops(peaks), 4), "traffic": None,
+            "kernel": "k_gemm_nvf4 (6 prefill launches)",
+            "peak_source": peaks["source"] + " bf16 x4 (dense FP4 / bf16 nominal ratio)"}
+    return out, roof
+
+
 # ------------------------------------------------------------ CPU baseline
 
-def cpu_oracle_sample(budget_s: float = 12.0, n_rows_w: int = 4096):
+def cpu_oracle_sample(workload: str = "decode", budget_s: float = 12.0):
     """Time the CPU oracle (as it stands) on the decode workload: (N,K)=(4096,4096),
     M in {1,16}; quantize X online, fp64 GEMM on the dequantized operands."""
     import oracle
     from nvfp4_block_scaled_18_b200 import workloads as wl
     oracle.build()
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    if workload == "prefill":
+        # a 128-row slice of the M = 8192 activations against the full (14336, 4096) weight
+        N, K, rows = 14336, 4096, 128
+        qw = oracle.quantize(wl.weights_normal(N, K))
+        x = wl.prefill_x(rows, K)
+        flops, t_total, calls = 0.0, 0.0, 0
+        t_start = time.perf_counter()
+        while time.perf_counter() - t_start < budget_s or calls < 1:
+            t0 = time.perf_counter()
+            oracle.gemm(oracle.quantize(x), qw)
+            t_total += time.perf_counter() - t0
+            flops += 2.0 * rows * N * K
+            calls += 1
+        return {"value": round(flops / t_total / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": f"{calls} x (128 rows of X, M=8192 workload) against W (14336,4096): oracle quantize "
+                          f"+ fp64 dequantized GEMM, {t_total:.1f} s"}
     N, K = 4096, 4096
     w = wl.weights_normal(N, K)
     qw = oracle.quantize(w)
@@ -303,7 +457,6 @@ def cpu_oracle_sample(budget_s: float = 12.0, n_rows_w: int = 4096):
         t_total += time.perf_counter() - t0
         done_bytes += decode_bytes(M, N, K)
         calls += 1
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     return {"value": round(done_bytes / t_total / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{calls} linear calls on (N,K)=(4096,4096), M alternating 1/16: oracle quantize "
                       f"+ fp64 dequantized GEMM, {t_total:.1f} s"}
@@ -367,8 +520,9 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="decode line without the prefill sub-measurement")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -380,58 +534,80 @@ def main():
     nv.load_library()
     peaks = load_peaks()
 
-    wk = DecodeWorkload(dev)
-    phases = DecodeWorkload.COPIES
+    if args.workload == "decode":
+        wk = DecodeWorkload(dev)
+        phases = DecodeWorkload.COPIES
+        unit, work_per_step = "GB/s", float(wk.step_bytes)
+        scale = 1e9
+        steps = args.steps
+    else:
+        wk = PrefillWorkload(dev)
+        phases = 1
+        unit, work_per_step = "TFLOP/s", float(sum(2.0 * M * N * Keff for (_, M, N, Keff, _) in wk.calls))
+        scale = 1e12
+        steps = max(1, min(args.steps, 40))
     graphs = capture_graphs(wk, phases)
     sampler = ClockSampler(torch.cuda.current_device())
-    ms = time_graphs(graphs, args.steps, args.warmup, world, sampler)
+    ms = time_graphs(graphs, steps, args.warmup, world, sampler)
     clocks = sampler.stop()
     ms_max = max_over_ranks(ms, world)
-    total_bytes = sum_over_ranks(wk.step_bytes * args.steps, world)
-    value = total_bytes / (ms_max * 1e-3) / 1e9
-    ms_per_step = ms_max / args.steps
+    value = sum_over_ranks(work_per_step * steps, world) / (ms_max * 1e-3) / scale
+    ms_per_step = ms_max / steps
 
-    # end to end: pinned host X -> device, quantize + GEMV, Y -> pinned host, every step
-    e2e_steps = max(4 * phases, min(args.steps, 400))
-    e2e_graphs = capture_graphs(wk, phases, e2e=True)
-    ms_e2e = max_over_ranks(time_graphs(e2e_graphs, e2e_steps, args.warmup, world), world)
-    e2e_value = sum_over_ranks(wk.step_bytes * e2e_steps, world) / (ms_e2e * 1e-3) / 1e9
+    # end to end: pinned host X -> device, quantize + GEMM, Y -> pinned host, every step
+    e2e_steps = max(4 * phases, min(steps, 400)) if args.workload == "decode" else max(2, min(steps, 5))
+    if args.workload == "decode":
+        e2e_graphs = capture_graphs(wk, phases, e2e=True)
+        ms_e2e = max_over_ranks(time_graphs(e2e_graphs, e2e_steps, args.warmup, world), world)
+        h2d, d2h = wk.h2d_bytes(), wk.d2h_bytes()
+    else:
+        ms_e2e, h2d, d2h = prefill_e2e(wk, e2e_steps), wk.h2d_bytes(), wk.d2h_bytes()
+        ms_e2e = max_over_ranks(ms_e2e, world)
+        e2e_graphs = []
+    e2e_value = sum_over_ranks(work_per_step * e2e_steps, world) / (ms_e2e * 1e-3) / scale
 
-    # per-launch GEMV timing for the roofline of the dominant kernel
-    per = time_gemv_launches(wk)
-    g_bytes = sum(gemv_bytes(*c) for c in wk.calls)
-    g_ms = sum(per.values())
-    achieved = g_bytes / (g_ms * 1e-3) / 1e9
-    detail = {f"M{M}_N{N}_K{K}": {"gemv_us": round(per[(M, N, K)] * 1e3, 3),
-                                  "gemv_GBps": round(gemv_bytes(M, N, K) / (per[(M, N, K)] * 1e-3) / 1e9, 1)}
-              for (M, N, K) in wk.calls}
-
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-        "us_per_call": round(ms_per_step * 1e3 / len(wk.calls), 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
-        "data": "synthetic",
-        "config": {"workload": "decode GEMV (M in 1,2,4,8,16; (N,K) in (4096,4096),(14336,4096),(4096,14336)); "
-                               "online bf16->NVFP4 activation quantization + CUDA-core NVFP4 GEMV, fp32 out",
-                   "calls_per_step": len(wk.calls), "l2": "weights rotate through 4 copies per shape (302 MB > L2)",
-                   "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
-                     "kernel": "k_gemv (all 15 decode launches)", "peak_source": peaks["source"]},
-        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": wk.h2d_bytes(),
-                "d2h_bytes_per_step": wk.d2h_bytes()},
-        "gpu_launches": wk.launches_per_step * args.steps,
-        "clocks": clocks,
-        "detail": detail,
-    }
+    line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5)}
+    if args.workload == "decode":
+        per = time_gemv_launches(wk)
+        g_bytes = sum(gemv_bytes(*c) for c in wk.calls)
+        achieved = g_bytes / (sum(per.values()) * 1e-3) / 1e9
+        line["us_per_call"] = round(ms_per_step * 1e3 / len(wk.calls), 3)
+        detail = {f"M{M}_N{N}_K{K}": {"gemv_us": round(per[(M, N, K)] * 1e3, 3),
+                                      "gemv_GBps": round(gemv_bytes(M, N, K) / (per[(M, N, K)] * 1e-3) / 1e9, 1)}
+                  for (M, N, K) in wk.calls}
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                    "kernel": "k_gemv (all 15 decode launches)", "peak_source": peaks["source"]}
+        config = {"workload": "decode GEMV (M in 1,2,4,8,16; (N,K) in (4096,4096),(14336,4096),(4096,14336)); "
+                              "online bf16->NVFP4 activation quantization + NVFP4 GEMV, fp32 out",
+                  "calls_per_step": len(wk.calls), "l2": "weights rotate through 4 copies per shape (302 MB > L2)",
+                  "parallelism": f"replicas x{world}"}
+        launches = wk.launches_per_step * steps
+    else:
+        detail, roofline = measure_prefill_from(wk, peaks)
+        config = {"workload": "large prefill W4A4 GEMM, M=8192, (N,K) in (14336,4096),(4096,14336),(28672,8192), "
+                              "each without and with the S=256 outlier-residue K extension; online quantization",
+                  "calls_per_step": len(wk.calls), "l2": "inputs > L2 (X 67-235 MB, Y 134-940 MB per call)",
+                  "parallelism": f"replicas x{world}"}
+        launches = 3 * len(wk.calls) * steps
+    line.update({"higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
+                 "data": "synthetic", "config": config, "roofline": roofline,
+                 "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d,
+                         "d2h_bytes_per_step": d2h},
+                 "gpu_launches": launches, "clocks": clocks, "detail": detail})
+    if args.workload == "decode" and not args.no_prefill:
+        del graphs, e2e_graphs
+        pw = PrefillWorkload(dev)
+        pdetail, proof = measure_prefill_from(pw, peaks)
+        line["prefill"] = {"roofline": proof, "detail": pdetail}
+        del pw
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_sample()
+        line["cpu_baseline"] = cpu_oracle_sample(args.workload)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del graphs, e2e_graphs
         dist.destroy_process_group()
     return 0
 
