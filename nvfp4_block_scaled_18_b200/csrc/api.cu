@@ -89,13 +89,18 @@ nvfp4_status run_gemm(const nvfp4_tensor* a, const nvfp4_tensor* r, const nvfp4_
   g.y = y; g.ldy = ldy; g.y_bf16 = out_dt == NVFP4_BF16;
   g.M = a->rows; g.N = w->rows; g.K = a->cols; g.st = dev_status;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (g.M <= 16) {
-    if (a->sf_layout != NVFP4_SF_ROWMAJOR || w->sf_layout != NVFP4_SF_ROWMAJOR)
-      return NVFP4_ERR_UNSUPPORTED;
-    return cuda_status(launch_gemv(g, num_sms_current_device(), s));
+  const bool tiled = a->sf_layout == NVFP4_SF_TILED && w->sf_layout == NVFP4_SF_TILED;
+  const bool rowmajor = a->sf_layout == NVFP4_SF_ROWMAJOR && w->sf_layout == NVFP4_SF_ROWMAJOR;
+  cudaError_t e;
+  if (rowmajor && g.M <= 16) {
+    e = launch_gemv(g, num_sms_current_device(), s);              // CUDA-core decode GEMV
+  } else if (tiled && g.M <= 128) {
+    e = launch_gemv_tc(g, num_sms_current_device(), s);           // tensor cores, operands swapped
+  } else if (tiled && r == nullptr) {
+    e = launch_gemm_tc(g, num_sms_current_device(), s);           // tensor cores, 128x256 tiles
+  } else {
+    return NVFP4_ERR_UNSUPPORTED;
   }
-  if (a->sf_layout != NVFP4_SF_TILED || w->sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_UNSUPPORTED;
-  const cudaError_t e = launch_gemm_tc(g, num_sms_current_device(), s);
   if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
   return cuda_status(e);
 }

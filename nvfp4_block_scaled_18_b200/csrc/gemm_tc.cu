@@ -22,13 +22,11 @@
 // CTAs in flight share W tiles through L2.  Every mbarrier wait is bounded: on
 // timeout the kernel records NVFP4_ERR_TIMEOUT, every role leaves its loop, and
 // TMEM is still released.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace nvfp4 {
+using namespace tc;
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 256;
@@ -47,7 +45,6 @@ constexpr uint32_t ACC_COL = 0;                  // 256 fp32 columns
 constexpr uint32_t SFA_COL = 256;                // 4 k-blocks x 4 columns
 constexpr uint32_t SFB_COL = 272;                // 4 k-blocks x 8 columns
 constexpr int NUM_THREADS = 192;
-constexpr uint64_t kTimeoutNs = 4000000000ull;
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for 128B swizzle");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -66,112 +63,6 @@ struct TcParams {
   int m_blocks, n_blocks, num_tiles, k_tiles;
   int* st;
 };
-
-// ----------------------------------------------------------------- PTX
-
-__device__ __forceinline__ uint32_t saddr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: false when this or another role gave up.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* st) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
-      *abort_flag = 1;
-      report_status(st, NVFP4_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(dst), "l"(map), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void tc_cp_scales(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-__device__ __forceinline__ void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %6, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
-      ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor: K-major operand tile, 128-byte swizzle,
-// 8-row groups 1024 bytes apart (sm_100 descriptor version 1).
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// Descriptor of one 512-byte scale atom (32 rows of 16 bytes, no swizzle) as
-// the tcgen05.cp source.
-__device__ __forceinline__ uint64_t desc_sf_atom(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(512 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
-         ((uint64_t)1 << 46);
-}
-// Instruction descriptor: kind::mxf4nvf4, A and B E2M1, K-major, UE4M3 scales,
-// fp32 accumulator, M = 128, N = n.
-__device__ __forceinline__ uint32_t idesc_nvf4(int n) {
-  return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-}
 
 // --------------------------------------------------------------- kernel
 
@@ -328,6 +219,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+}  // namespace
+
+namespace tc {
+
 // The driver's tensor-map encoder, resolved at run time through the runtime API
 // so that the library does not link against libcuda.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -347,7 +242,7 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
   if (encode == nullptr) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-  const cuuint32_t box[2] = {(cuuint32_t)BK_BYTES, box_rows};
+  const cuuint32_t box[2] = {(cuuint32_t)128, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims,
                                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -355,7 +250,7 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
+}  // namespace tc
 
 cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   if (g.r_codes != nullptr) return cudaErrorNotSupported;  // own-scale residue: small-M paths only

@@ -1,0 +1,306 @@
+// Few-row NVFP4 linear (M <= 128) on the tensor cores with the operands
+// swapped, sm_100a.
+//
+// Y^T = W X^T: W (N x K) is the 128-row A operand of
+// tcgen05.mma.kind::mxf4nvf4.block_scale.block16, the M activation rows (padded
+// to NP = 16/32/64/128) are the B operand, so a decode step costs one pass over
+// W at HBM speed instead of being limited by CUDA-core multiply rates.  With a
+// residue operand R (ResServe abstract: FP4 base plus FP4 residue, combined
+// on-chip) the same W tile feeds a second accumulator, and both are combined in
+// the epilogue with their own tensor scales: Y = s_x s_w acc + s_r s_w acc_r.
+//
+// Grid: (ks, ceil(N/128)); the ks CTAs of one cluster split K between them and
+// each accumulates a 128 x NP fp32 partial in TMEM.  The partials are written
+// to shared memory and summed across the cluster through distributed shared
+// memory; CTA rank r of the cluster writes rows [r*128/ks, (r+1)*128/ks) of the
+// tile.  Roles inside a CTA (128 threads): warp 0 lane 0 issues TMA/bulk copies
+// into a shared-memory ring, warp 1 lane 0 copies scale atoms to TMEM and
+// issues the MMAs, then all four warps drain the accumulators.
+//
+// Safety: every mbarrier wait is bounded; every CTA reaches both cluster
+// barriers on every path; the dynamic shared-memory request caps the CTAs per
+// SM so that their TMEM allocations always fit side by side (no CTA can block
+// in tcgen05.alloc behind a cluster peer).
+#include "kernels.h"
+#include "tcgen05.cuh"
+
+namespace nvfp4 {
+using namespace tc;
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int W_TILE = 128 * 128;   // 128 rows of W x 128 bytes (256 K-elements)
+constexpr int SF4 = 4 * 512;         // 4 scale atoms: one 128-row group x 256 K
+
+template <int NP, bool RES>
+struct Cfg {
+  static constexpr int X_TILE = NP * 128;
+  static constexpr int OFF_X = W_TILE;
+  static constexpr int OFF_R = OFF_X + X_TILE;
+  static constexpr int OFF_SFW = OFF_R + (RES ? X_TILE : 0);
+  static constexpr int OFF_SFX = OFF_SFW + SF4;
+  static constexpr int OFF_SFR = OFF_SFX + SF4;
+  static constexpr int STAGE = ((OFF_SFR + (RES ? SF4 : 0)) + 1023) / 1024 * 1024;
+  // TMEM: acc [0,NP), acc_r [NP,2NP), scales of W, X, R (16 columns each)
+  static constexpr uint32_t ACC = 0, ACC_R = NP;
+  static constexpr uint32_t SFW_COL = 2 * NP, SFX_COL = 2 * NP + 16, SFR_COL = 2 * NP + 32;
+  static constexpr uint32_t COLS_USED = 2 * NP + 48;
+  static constexpr uint32_t TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
+  static constexpr int TMEM_CTAS = 512 / TMEM_COLS;               // CTAs whose TMEM fits on one SM
+  static constexpr int BAR = 256;
+  // stages: as many as keep two CTAs per SM (four when TMEM allows only one CTA)
+  static constexpr int BUDGET = TMEM_CTAS >= 2 ? 114 * 1024 : 224 * 1024;
+  static constexpr int STAGES = (4 * STAGE + BAR + 1024 <= BUDGET) ? 4 : ((3 * STAGE + BAR + 1024 <= BUDGET) ? 3 : 2);
+  static constexpr int PITCH = NP + 4;                            // floats per partial row (padded)
+  static constexpr int PART = 128 * PITCH * 4 * (RES ? 2 : 1);   // overlays the idle stage ring
+  static constexpr int SMEM_NEED = STAGES * STAGE + BAR + 1024;
+  // request that keeps at most TMEM_CTAS CTAs on an SM, so tcgen05.alloc never waits on a peer
+  static constexpr int SMEM_MIN = 233472 / (TMEM_CTAS + 1) + 1024;
+  static constexpr int SMEM = SMEM_NEED > SMEM_MIN ? SMEM_NEED : SMEM_MIN;
+  static constexpr int CTAS_PER_SM = (233472 / (SMEM + 1024)) < TMEM_CTAS ? (233472 / (SMEM + 1024)) : TMEM_CTAS;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(PART <= STAGES * STAGE, "partials overlay the stage ring");
+  static_assert(233472 / (SMEM + 1024) <= TMEM_CTAS, "TMEM must fit every co-resident CTA");
+  static_assert(CTAS_PER_SM >= 1, "residency");
+};
+
+struct SwapParams {
+  const uint8_t* sfw;    // W scales, TILED
+  const uint8_t* sfx;    // X scales, TILED (row group 0)
+  const uint8_t* sfr;    // R scales, TILED (row group 0) or null
+  const float* x_s;
+  const float* w_s;
+  const float* r_s;
+  void* y;
+  int64_t ldy;
+  int M, N, K;
+  int katoms_w, k_tiles;
+  int* st;
+};
+
+template <int NP>
+__device__ __forceinline__ void drain_acc(uint32_t taddr, float* row_out) {
+  if constexpr (NP == 16) {
+    uint32_t r[16];
+    tmem_ld16(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; i += 4)
+      *reinterpret_cast<float4*>(row_out + i) =
+          make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
+                      __uint_as_float(r[i + 3]));
+  } else {
+#pragma unroll
+    for (int c = 0; c < NP; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(row_out + c + i) =
+            make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
+                        __uint_as_float(r[i + 3]));
+    }
+  }
+}
+
+template <int NP, bool RES, bool BF16OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemv_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+              const __grid_constant__ CUtensorMap tmR, const SwapParams p) {
+  using C = Cfg<NP, RES>;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* part = reinterpret_cast<float*>(smem);    // reused once the mainloop is over
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* acc_full = bars + 2 * C::STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank(), ks = cluster_nctarank();
+  const int rt = blockIdx.y;                                       // 128-row tile of W
+  const int kt0 = (int)((rank * (uint32_t)p.k_tiles) / ks);
+  const int kt1 = (int)(((rank + 1) * (uint32_t)p.k_tiles) / ks);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(saddr(&full[s]), 1);
+      mbar_init(saddr(&empty[s]), 1);
+    }
+    mbar_init(saddr(acc_full), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------- TMA producer
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kt = kt0; kt < kt1; ++kt) {
+      if (!mbar_wait(saddr(&empty[s]), ph ^ 1u, abort_flag, p.st)) break;
+      const int jmax = min(4, (p.K - kt * 256) / 64);
+      const uint32_t sf = (uint32_t)jmax * 512u;
+      const uint32_t bar = saddr(&full[s]);
+      uint8_t* sb = smem + s * C::STAGE;
+      mbar_expect_tx(bar, W_TILE + C::X_TILE * (RES ? 2 : 1) + sf * (RES ? 3 : 2));
+      tma_load_2d(saddr(sb), &tmW, kt * 128, rt * 128, bar);
+      tma_load_2d(saddr(sb + C::OFF_X), &tmX, kt * 128, 0, bar);
+      if (RES) tma_load_2d(saddr(sb + C::OFF_R), &tmR, kt * 128, 0, bar);
+      bulk_load(saddr(sb + C::OFF_SFW), p.sfw + ((size_t)rt * p.katoms_w + kt * 4) * 512, sf, bar);
+      bulk_load(saddr(sb + C::OFF_SFX), p.sfx + (size_t)kt * 4 * 512, sf, bar);
+      if (RES) bulk_load(saddr(sb + C::OFF_SFR), p.sfr + (size_t)kt * 4 * 512, sf, bar);
+      if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // --------------------------------------------------------- MMA issuer
+    const uint32_t idesc = idesc_nvf4(NP);
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kt = kt0; kt < kt1; ++kt) {
+      if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) break;
+      tc_fence_after();
+      const int jmax = min(4, (p.K - kt * 256) / 64);
+      const uint8_t* sb = smem + s * C::STAGE;
+      for (int j = 0; j < jmax; ++j) {
+        tc_cp_scales(tmem + C::SFW_COL + 4 * j, desc_sf_atom(saddr(sb + C::OFF_SFW + j * 512)));
+        tc_cp_scales(tmem + C::SFX_COL + 4 * j, desc_sf_atom(saddr(sb + C::OFF_SFX + j * 512)));
+        if (RES) tc_cp_scales(tmem + C::SFR_COL + 4 * j, desc_sf_atom(saddr(sb + C::OFF_SFR + j * 512)));
+      }
+      const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(sb + C::OFF_X));
+      const uint64_t dr = desc_sw128(saddr(sb + C::OFF_R));
+      for (int j = 0; j < jmax; ++j) {
+        const uint32_t acc = (kt > kt0 || j > 0) ? 1u : 0u;
+        tc_mma_nvf4(tmem + C::ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + C::SFW_COL + 4 * j,
+                    tmem + C::SFX_COL + 4 * j, acc);
+        if (RES)
+          tc_mma_nvf4(tmem + C::ACC_R, dw + (uint64_t)(2 * j), dr + (uint64_t)(2 * j), idesc,
+                      tmem + C::SFW_COL + 4 * j, tmem + C::SFR_COL + 4 * j, acc);
+      }
+      tc_commit(saddr(&empty[s]));
+      if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+    }
+    tc_commit(saddr(acc_full));
+  }
+  __syncwarp();
+
+  // ----------------------------------------- drain partials into shared memory
+  const bool ok = mbar_wait(saddr(acc_full), 0u, abort_flag, p.st);
+  tc_fence_after();
+  {
+    const int row = warp * 32 + lane;                              // TMEM lane = W row of the tile
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    if (ok) {
+      drain_acc<NP>(lane_addr + C::ACC, part + row * C::PITCH);
+      if (RES) drain_acc<NP>(lane_addr + C::ACC_R, part + (128 + row) * C::PITCH);
+    } else {
+      for (int i = 0; i < NP; ++i) part[row * C::PITCH + i] = 0.0f;
+    }
+  }
+  tc_fence_before();
+  cluster_sync();
+
+  // -------------------------------- reduce the K-split partials across the cluster
+  {
+    const int r0 = (int)((rank * 128u) / ks), r1 = (int)(((rank + 1) * 128u) / ks);
+    const int nrows = r1 - r0;
+    const float alpha = (*p.x_s) * (*p.w_s);
+    const float alpha_r = RES ? (*p.r_s) * (*p.w_s) : 0.0f;
+    const uint32_t part_base = saddr(part);
+    for (int idx = threadIdx.x; idx < nrows * p.M; idx += kThreads) {
+      const int m = idx / nrows, i = idx - m * nrows;
+      const int n = rt * 128 + r0 + i;
+      if (n >= p.N) continue;
+      const uint32_t off = (uint32_t)(((r0 + i) * C::PITCH + m) * 4);
+      float sum = 0.0f, sum_r = 0.0f;
+      for (uint32_t pr = 0; pr < ks; ++pr) {
+        sum += ld_cluster_f32(mapa_shared(part_base + off, pr));
+        if (RES) sum_r += ld_cluster_f32(mapa_shared(part_base + off + 128u * C::PITCH * 4u, pr));
+      }
+      const float out = RES ? fmaf(sum, alpha, sum_r * alpha_r) : sum * alpha;
+      if (BF16OUT)
+        reinterpret_cast<__nv_bfloat16*>(p.y)[(int64_t)m * p.ldy + n] = __float2bfloat16_rn(out);
+      else
+        reinterpret_cast<float*>(p.y)[(int64_t)m * p.ldy + n] = out;
+    }
+  }
+  cluster_sync();  // peers may still be reading this CTA's partials until here
+
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+template <int NP, bool RES, bool BF16OUT>
+cudaError_t launch_np(const GemmArgs& g, int num_sms, cudaStream_t stream) {
+  using C = Cfg<NP, RES>;
+  CUtensorMap tmW, tmX, tmR;
+  if (!encode_codes_map(&tmW, g.w_codes, g.N, g.K, 128) || !encode_codes_map(&tmX, g.a_codes, g.M, g.K, NP))
+    return cudaErrorInvalidValue;
+  if (RES) {
+    if (!encode_codes_map(&tmR, g.r_codes, g.M, g.K, NP)) return cudaErrorInvalidValue;
+  } else {
+    tmR = tmX;
+  }
+  SwapParams p{};
+  p.sfw = g.w_scales; p.sfx = g.a_scales; p.sfr = g.r_scales;
+  p.x_s = g.a_s; p.w_s = g.w_s; p.r_s = RES ? g.r_s : g.a_s;
+  p.y = g.y; p.ldy = g.ldy;
+  p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K;
+  p.katoms_w = (int)((g.K + 63) / 64);
+  p.k_tiles = (int)((g.K + 255) / 256);
+  p.st = g.st;
+  const int row_tiles = (int)((g.N + 127) / 128);
+  const int want = std::max(1, (C::CTAS_PER_SM * num_sms + row_tiles / 2) / row_tiles);
+  const int ks = std::max(1, std::min({8, p.k_tiles, want}));
+  auto kern = k_gemv_tc<NP, RES, BF16OUT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ks, (unsigned)row_tiles, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, tmR, p);
+}
+
+template <int NP>
+cudaError_t launch_res(const GemmArgs& g, int num_sms, cudaStream_t stream) {
+  if (g.r_codes != nullptr)
+    return g.y_bf16 ? launch_np<NP, true, true>(g, num_sms, stream) : launch_np<NP, true, false>(g, num_sms, stream);
+  return g.y_bf16 ? launch_np<NP, false, true>(g, num_sms, stream) : launch_np<NP, false, false>(g, num_sms, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) {
+  if (g.K % 64 != 0 || g.K < 256 || g.M > 128) return cudaErrorNotSupported;
+  if (g.M <= 16) return launch_res<16>(g, num_sms, stream);
+  if (g.M <= 32) return launch_res<32>(g, num_sms, stream);
+  if (g.M <= 64) return launch_res<64>(g, num_sms, stream);
+  return launch_res<128>(g, num_sms, stream);
+}
+
+}  // namespace nvfp4

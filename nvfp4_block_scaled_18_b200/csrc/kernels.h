@@ -50,5 +50,6 @@ struct GemmArgs {
 
 cudaError_t launch_gemv(const GemmArgs& g, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemv_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);
 
 }  // namespace nvfp4

@@ -43,3 +43,22 @@ def rel_fro(y, ref) -> float:
 def sub_rows(orc, q_full_codes, q_full_scales, s, rows):
     """An oracle QTensor of selected rows (slicing only)."""
     return orc.QTensor(np.ascontiguousarray(q_full_codes[rows]), np.ascontiguousarray(q_full_scales[rows]), s)
+
+
+def tiled_from_rowmajor(scales: np.ndarray) -> np.ndarray:
+    """Place row-major block scales (rows x nb) into the TILED atom layout (layout only)."""
+    rows, nb = scales.shape
+    katoms = (nb + 3) // 4
+    out = np.zeros(((rows + 127) // 128) * katoms * 512, np.uint8)
+    r = np.arange(rows)[:, None]
+    b = np.arange(nb)[None, :]
+    off = ((r // 128) * katoms + b // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + (b % 4)
+    out[off] = scales
+    return out
+
+
+def gpu_tensor(codes, scales_rowmajor, s, layout=nv.SF_TILED):
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    sc = tiled_from_rowmajor(scales_rowmajor) if layout == nv.SF_TILED else scales_rowmajor.reshape(-1)
+    return nv.NVFP4Tensor(torch.from_numpy(np.ascontiguousarray(codes)).cuda(), torch.from_numpy(sc).cuda(),
+                          torch.tensor([s], dtype=torch.float32, device="cuda"), rows, cols, layout)

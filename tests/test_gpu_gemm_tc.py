@@ -12,7 +12,7 @@ import torch
 import nvfp4_block_scaled_18_b200 as nv
 from nvfp4_block_scaled_18_b200 import workloads as wl
 
-from gpu_util import REL_FRO_TOL, assert_same_q, rel_fro, run_quantize, to_dev
+from gpu_util import REL_FRO_TOL, assert_same_q, gpu_tensor, rel_fro, run_quantize, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -21,25 +21,6 @@ pytestmark = pytest.mark.gpu
 def _cuda():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     nv.load_library()
-
-
-def tiled_from_rowmajor(scales: np.ndarray) -> np.ndarray:
-    """Place row-major block scales (rows x nb) into the TILED atom layout (layout only)."""
-    rows, nb = scales.shape
-    katoms = (nb + 3) // 4
-    out = np.zeros(((rows + 127) // 128) * katoms * 512, np.uint8)
-    r = np.arange(rows)[:, None]
-    b = np.arange(nb)[None, :]
-    off = ((r // 128) * katoms + b // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + (b % 4)
-    out[off] = scales
-    return out
-
-
-def gpu_tensor(codes, scales_rowmajor, s, layout=nv.SF_TILED):
-    rows, cols = codes.shape[0], codes.shape[1] * 2
-    sc = tiled_from_rowmajor(scales_rowmajor) if layout == nv.SF_TILED else scales_rowmajor.reshape(-1)
-    return nv.NVFP4Tensor(torch.from_numpy(np.ascontiguousarray(codes)).cuda(), torch.from_numpy(sc).cuda(),
-                          torch.tensor([s], dtype=torch.float32, device="cuda"), rows, cols, layout)
 
 
 def run_gemm(a, w, out_dtype=torch.float32):
