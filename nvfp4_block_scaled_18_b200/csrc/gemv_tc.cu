@@ -10,11 +10,10 @@
 // the epilogue with their own tensor scales: Y = s_x s_w acc + s_r s_w acc_r.
 //
 // Grid: (ks, ceil(N/128)); the ks CTAs of one cluster split K between them and
-// each accumulates a 128 x NP fp32 partial in TMEM.  Every CTA pushes its
-// partial rows into the shared memory of the CTA that owns them (distributed
-// shared memory stores), one cluster barrier later each owner sums its rows
-// and writes Y.  The kernel is launched as a programmatic dependent of the
-// activation quantizer: the W tiles stream in before griddepcontrol.wait.  Roles inside a CTA (128 threads): warp 0 lane 0 issues TMA/bulk copies
+// each accumulates a 128 x NP fp32 partial in TMEM.  The partials are written
+// to shared memory and summed across the cluster through distributed shared
+// memory; CTA rank r of the cluster writes rows [r*128/ks, (r+1)*128/ks) of the
+// tile.  Roles inside a CTA (128 threads): warp 0 lane 0 issues TMA/bulk copies
 // into a shared-memory ring, warp 1 lane 0 copies scale atoms to TMEM and
 // issues the MMAs, then all four warps drain the accumulators.
 //
@@ -49,22 +48,18 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
   static constexpr int TMEM_CTAS = 512 / TMEM_COLS;               // CTAs whose TMEM fits on one SM
   static constexpr int BAR = 256;
-  static constexpr int PITCH = NP + 4;                            // floats per partial row (padded)
-  // partial rows pushed to an owner CTA: ks * ceil(128/ks) <= 135 for ks <= 8
-  static constexpr int PART_ROWS = 136;
-  static constexpr int PART = PART_ROWS * PITCH * 4 * (RES ? 2 : 1);
-  static constexpr bool PART_OWN = PART <= 40 * 1024;            // dedicated area, else overlays the ring
-  static constexpr int PART_DED = PART_OWN ? PART : 0;
   // stages: as many as keep two CTAs per SM (four when TMEM allows only one CTA)
-  static constexpr int BUDGET = (TMEM_CTAS >= 2 ? 114 * 1024 : 224 * 1024) - PART_DED;
+  static constexpr int BUDGET = TMEM_CTAS >= 2 ? 114 * 1024 : 224 * 1024;
   static constexpr int STAGES = (4 * STAGE + BAR + 1024 <= BUDGET) ? 4 : ((3 * STAGE + BAR + 1024 <= BUDGET) ? 3 : 2);
+  static constexpr int PITCH = NP + 4;                            // floats per partial row (padded)
+  static constexpr int PART = 128 * PITCH * 4 * (RES ? 2 : 1);   // overlays the idle stage ring
   static constexpr int SMEM_NEED = STAGES * STAGE + BAR + 1024;
   // request that keeps at most TMEM_CTAS CTAs on an SM, so tcgen05.alloc never waits on a peer
   static constexpr int SMEM_MIN = 233472 / (TMEM_CTAS + 1) + 1024;
   static constexpr int SMEM = SMEM_NEED > SMEM_MIN ? SMEM_NEED : SMEM_MIN;
   static constexpr int CTAS_PER_SM = (233472 / (SMEM + 1024)) < TMEM_CTAS ? (233472 / (SMEM + 1024)) : TMEM_CTAS;
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(PART_OWN || PART <= STAGES * STAGE, "partials overlay the stage ring");
+  static_assert(PART <= STAGES * STAGE, "partials overlay the stage ring");
   static_assert(233472 / (SMEM + 1024) <= TMEM_CTAS, "TMEM must fit every co-resident CTA");
   static_assert(CTAS_PER_SM >= 1, "residency");
 };
@@ -116,8 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<NP, RES>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* part = reinterpret_cast<float*>(C::PART_OWN ? smem + C::STAGES * C::STAGE : smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE + C::PART_DED);
+  float* part = reinterpret_cast<float*>(smem);    // reused once the mainloop is over
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* acc_full = bars + 2 * C::STAGES;
@@ -152,44 +147,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------- TMA producer
-    // W does not depend on the preceding grid (the activation quantizer): the
-    // first stages' W tiles are requested before waiting for it.
-    auto stage_bytes = [&](int kt) {
-      const uint32_t sf = (uint32_t)min(4, (p.K - kt * 256) / 64) * 512u;
-      return (uint32_t)(W_TILE + C::X_TILE * (RES ? 2 : 1)) + sf * (RES ? 3u : 2u);
-    };
-    auto load_w = [&](int kt, int s) {
-      const uint32_t sf = (uint32_t)min(4, (p.K - kt * 256) / 64) * 512u;
-      uint8_t* sb = smem + s * C::STAGE;
-      const uint32_t bar = saddr(&full[s]);
-      tma_load_2d(saddr(sb), &tmW, kt * 128, rt * 128, bar);
-      bulk_load(saddr(sb + C::OFF_SFW), p.sfw + ((size_t)rt * p.katoms_w + kt * 4) * 512, sf, bar);
-    };
-    auto load_x = [&](int kt, int s) {
-      const uint32_t sf = (uint32_t)min(4, (p.K - kt * 256) / 64) * 512u;
-      uint8_t* sb = smem + s * C::STAGE;
-      const uint32_t bar = saddr(&full[s]);
-      tma_load_2d(saddr(sb + C::OFF_X), &tmX, kt * 128, 0, bar);
-      bulk_load(saddr(sb + C::OFF_SFX), p.sfx + (size_t)kt * 4 * 512, sf, bar);
-      if (RES) {
-        tma_load_2d(saddr(sb + C::OFF_R), &tmR, kt * 128, 0, bar);
-        bulk_load(saddr(sb + C::OFF_SFR), p.sfr + (size_t)kt * 4 * 512, sf, bar);
-      }
-    };
-    const int pre = min(kt1 - kt0, C::STAGES);
-    for (int i = 0; i < pre; ++i) {        // first round: every stage is free
-      mbar_expect_tx(saddr(&full[i]), stage_bytes(kt0 + i));
-      load_w(kt0 + i, i);
-    }
-    griddep_wait();
-    for (int i = 0; i < pre; ++i) load_x(kt0 + i, i);
-    int s = pre % C::STAGES;
-    uint32_t ph = (pre == C::STAGES) ? 1u : 0u;
-    for (int kt = kt0 + pre; kt < kt1; ++kt) {
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kt = kt0; kt < kt1; ++kt) {
       if (!mbar_wait(saddr(&empty[s]), ph ^ 1u, abort_flag, p.st)) break;
-      mbar_expect_tx(saddr(&full[s]), stage_bytes(kt));
-      load_w(kt, s);
-      load_x(kt, s);
+      const int jmax = min(4, (p.K - kt * 256) / 64);
+      const uint32_t sf = (uint32_t)jmax * 512u;
+      const uint32_t bar = saddr(&full[s]);
+      uint8_t* sb = smem + s * C::STAGE;
+      mbar_expect_tx(bar, W_TILE + C::X_TILE * (RES ? 2 : 1) + sf * (RES ? 3 : 2));
+      tma_load_2d(saddr(sb), &tmW, kt * 128, rt * 128, bar);
+      tma_load_2d(saddr(sb + C::OFF_X), &tmX, kt * 128, 0, bar);
+      if (RES) tma_load_2d(saddr(sb + C::OFF_R), &tmR, kt * 128, 0, bar);
+      bulk_load(saddr(sb + C::OFF_SFW), p.sfw + ((size_t)rt * p.katoms_w + kt * 4) * 512, sf, bar);
+      bulk_load(saddr(sb + C::OFF_SFX), p.sfx + (size_t)kt * 4 * 512, sf, bar);
+      if (RES) bulk_load(saddr(sb + C::OFF_SFR), p.sfr + (size_t)kt * 4 * 512, sf, bar);
       if (++s == C::STAGES) { s = 0; ph ^= 1u; }
     }
   } else if (warp == 1 && lane == 0) {
@@ -223,63 +195,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_commit(saddr(acc_full));
   }
   __syncwarp();
-  griddep_wait();  // the epilogue reads the activation tensor scale
 
-  // ------------------- push this CTA's partial rows to the CTA that owns them
-  // Row r of the tile is owned by cluster rank o = r*ks/128, which holds rows
-  // [ceil(o*128/ks), ceil((o+1)*128/ks)); every source rank has its own slot.
+  // ----------------------------------------- drain partials into shared memory
   const bool ok = mbar_wait(saddr(acc_full), 0u, abort_flag, p.st);
   tc_fence_after();
-  const int rows_max = (int)((128u + ks - 1) / ks);
-  auto owner_row0 = [&](uint32_t o) { return (int)((o * 128u + ks - 1) / ks); };
-  if (!C::PART_OWN) {            // the partials overlay the ring: wait until every peer's mainloop is over
-    tc_fence_before();
-    cluster_arrive();
-    cluster_wait();
-  }
   {
-    const int row = warp * 32 + lane;
-    const uint32_t o = (uint32_t)(row * (int)ks) / 128u;
-    const int slot = (int)rank * rows_max + (row - owner_row0(o));
-    const uint32_t dst = mapa_shared(saddr(part + slot * C::PITCH), o);
+    const int row = warp * 32 + lane;                              // TMEM lane = W row of the tile
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int acc_i = 0; acc_i < (RES ? 2 : 1); ++acc_i) {
-      const uint32_t dsti = dst + (uint32_t)(acc_i * C::PART_ROWS * C::PITCH * 4);
-      const uint32_t src = lane_addr + (acc_i ? C::ACC_R : C::ACC);
-#pragma unroll
-      for (int c = 0; c < NP; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(src + c, r);
-        tmem_ld_wait();
-        if (!ok) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = 0u;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; i += 4)
-          st_cluster_f32x4(dsti + (uint32_t)((c + i) * 4), __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                           __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-      }
+    if (ok) {
+      drain_acc<NP>(lane_addr + C::ACC, part + row * C::PITCH);
+      if (RES) drain_acc<NP>(lane_addr + C::ACC_R, part + (128 + row) * C::PITCH);
+    } else {
+      for (int i = 0; i < NP; ++i) part[row * C::PITCH + i] = 0.0f;
     }
   }
   tc_fence_before();
-  cluster_sync();  // all partials have landed in their owners' shared memory
+  cluster_sync();
 
-  // ------------------------------------------- owners sum their rows and store
+  // -------------------------------- reduce the K-split partials across the cluster
   {
-    const int r0 = owner_row0(rank), r1 = owner_row0(rank + 1);
+    const int r0 = (int)((rank * 128u) / ks), r1 = (int)(((rank + 1) * 128u) / ks);
     const int nrows = r1 - r0;
     const float alpha = (*p.x_s) * (*p.w_s);
     const float alpha_r = RES ? (*p.r_s) * (*p.w_s) : 0.0f;
+    const uint32_t part_base = saddr(part);
     for (int idx = threadIdx.x; idx < nrows * p.M; idx += kThreads) {
       const int m = idx / nrows, i = idx - m * nrows;
       const int n = rt * 128 + r0 + i;
       if (n >= p.N) continue;
+      const uint32_t off = (uint32_t)(((r0 + i) * C::PITCH + m) * 4);
+      // issue every peer load before the first add so their latencies overlap
+      float v[8], vr[8];
+#pragma unroll
+      for (uint32_t pr = 0; pr < 8; ++pr) {
+        v[pr] = pr < ks ? ld_cluster_f32(mapa_shared(part_base + off, pr)) : 0.0f;
+        if (RES) vr[pr] = pr < ks ? ld_cluster_f32(mapa_shared(part_base + off + 128u * C::PITCH * 4u, pr)) : 0.0f;
+      }
       float sum = 0.0f, sum_r = 0.0f;
-      for (uint32_t src = 0; src < ks; ++src) {
-        const int slot = (int)src * rows_max + i;
-        sum += part[slot * C::PITCH + m];
-        if (RES) sum_r += part[C::PART_ROWS * C::PITCH + slot * C::PITCH + m];
+#pragma unroll
+      for (int pr = 0; pr < 8; ++pr) {
+        sum += v[pr];
+        if (RES) sum_r += vr[pr];
       }
       const float out = RES ? fmaf(sum, alpha, sum_r * alpha_r) : sum * alpha;
       if (BF16OUT)
@@ -288,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         reinterpret_cast<float*>(p.y)[(int64_t)m * p.ldy + n] = out;
     }
   }
+  cluster_sync();  // peers may still be reading this CTA's partials until here
 
   if (warp == 1) {
     __syncwarp();
@@ -327,15 +284,13 @@ cudaError_t launch_np(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the quantizer's tail
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, tmR, p);
 }
 

@@ -107,8 +107,6 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
                                                int64_t ldx, const float* s_ptr,
                                                const float* sr_ptr, QOut q, QOut r, WsHeader* ws,
                                                int* st) {
-  // a programmatically dependent GEMM may start its weight prefetch now
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t upr = K >> 3;
   const float s = *s_ptr;
   const float s_r = (MODE == Q_RES_ONLY || MODE == Q_BOTH) ? *sr_ptr : 0.0f;
@@ -233,7 +231,6 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
                                                        const int32_t* __restrict__ perm, int64_t S,
                                                        const float* s_ptr, QOut q, int* st) {
   extern __shared__ __align__(16) unsigned char smem[];
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   int32_t* sperm = reinterpret_cast<int32_t*>(smem);
   float* sgamma = reinterpret_cast<float*>(smem + K * 4);
   T* srow = reinterpret_cast<T*>(smem + K * 4 + (gamma ? K * 4 : 0));
