@@ -135,11 +135,6 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64
  *     the 128-row MMA operand, K split across a thread-block cluster), K >= 256;
  *   TILED scales, M > 128: tensor-core 128x256-tile GEMM, K >= 256.
  *   Other combinations return NVFP4_ERR_UNSUPPORTED.
- * Ordering: the few-row tensor-core kernel is launched as a programmatic
- * dependent of the preceding kernel on `stream`; it may start reading w (codes
- * and scales) while that kernel is still running.  w must therefore be
- * complete before the preceding kernel starts (weights are normally static);
- * a, r, their tensor scales and y may be produced or consumed by it.
  * y: device, aligned to sizeof(out_dt), row stride ldy >= N elements. */
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y,
                         nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
