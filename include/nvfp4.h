@@ -147,6 +147,31 @@ nvfp4_status nvfp4_gemm_residue(const nvfp4_tensor* a, const nvfp4_tensor* r,
                                 const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt, int64_t ldy,
                                 int* dev_status, void* stream);
 
+/* Largest M accepted by nvfp4_rmsnorm_reorder_quantize_noalloc. */
+#define NVFP4_NOALLOC_MAX_ROWS 65536
+
+/* nvfp4_rmsnorm_reorder_quantize without a caller workspace, for callers that
+ * cannot allocate device memory (code running during CUDA graph capture, hosts
+ * that own every allocation, paths that must never call the allocator).  The
+ * method's pages have no counterpart: this is a deployment variant of the
+ * fused quantizer above, with identical results.
+ * Its scratch (reduction cells + one fp32 per row) is a device array inside the
+ * library, allocated when the library is loaded and held by every GPU that
+ * loads it until the process exits; M > NVFP4_NOALLOC_MAX_ROWS returns
+ * NVFP4_ERR_WORKSPACE.  Every call on a device shares that array and finds it
+ * as the previous call left it: each call first clears the reduction cells on
+ * `stream`, so calls ordered on one stream are safe, while calls that may
+ * overlap on the GPU (unordered streams) race on it.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture begins.
+ * It calls no allocation routine.  Other arguments and errors as
+ * nvfp4_rmsnorm_reorder_quantize. */
+nvfp4_status nvfp4_rmsnorm_reorder_quantize_noalloc(const void* x, nvfp4_dtype dt, int64_t M, int64_t K,
+                                                    int64_t ldx, const void* gamma, float eps,
+                                                    const int32_t* perm, int64_t S,
+                                                    const float* scale_in, nvfp4_tensor* x_aug,
+                                                    int* dev_status, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* nvfp4_status_string(nvfp4_status status);
 

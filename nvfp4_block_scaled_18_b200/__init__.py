@@ -25,7 +25,9 @@ SF_ROWMAJOR, SF_TILED = 0, 1
 
 EXPORTED_SYMBOLS = ("nvfp4_scales_bytes", "nvfp4_workspace_size", "nvfp4_quantize",
                     "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize", "nvfp4_gemm",
-                    "nvfp4_gemm_residue", "nvfp4_status_string", "nvfp4_version")
+                    "nvfp4_gemm_residue", "nvfp4_rmsnorm_reorder_quantize_noalloc",
+                    "nvfp4_status_string", "nvfp4_version")
+NVFP4_NOALLOC_MAX_ROWS = 65536
 
 
 class NVFP4Error(RuntimeError):
@@ -60,10 +62,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.nvfp4_quantize_residue.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, T, T, P, SZ, P, P]
         lib.nvfp4_rmsnorm_reorder_quantize.argtypes = [P, ctypes.c_int, I64, I64, I64, P, F, P, I64, P, T,
                                                        P, SZ, P, P]
+        lib.nvfp4_rmsnorm_reorder_quantize_noalloc.argtypes = [P, ctypes.c_int, I64, I64, I64, P, F, P, I64, P,
+                                                               T, P, P]
         lib.nvfp4_gemm.argtypes = [T, T, P, ctypes.c_int, I64, P, P]
         lib.nvfp4_gemm_residue.argtypes = [T, T, T, P, ctypes.c_int, I64, P, P]
         for fn in ("nvfp4_quantize", "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize",
-                   "nvfp4_gemm", "nvfp4_gemm_residue"):
+                   "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_gemm", "nvfp4_gemm_residue"):
             getattr(lib, fn).restype = ctypes.c_int
         lib.nvfp4_status_string.argtypes = [ctypes.c_int]
         lib.nvfp4_status_string.restype = ctypes.c_char_p
@@ -208,6 +212,22 @@ def nvfp4_rmsnorm_reorder_quantize(x: torch.Tensor, x_aug: NVFP4Tensor,
                                               ctypes.byref(xc), ws_ptr, ws_n, _ptr(dev_status),
                                               _stream(stream)),
            "nvfp4_rmsnorm_reorder_quantize")
+
+
+def nvfp4_rmsnorm_reorder_quantize_noalloc(x: torch.Tensor, x_aug: NVFP4Tensor,
+                                           gamma: Optional[torch.Tensor] = None, eps: float = 1e-5,
+                                           perm: Optional[torch.Tensor] = None, S: int = 0,
+                                           scale_in: Optional[torch.Tensor] = None,
+                                           dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """As nvfp4_rmsnorm_reorder_quantize, with the library's built-in scratch
+    instead of a caller workspace (for callers that cannot allocate)."""
+    lib = load_library()
+    M, K = x.shape
+    xc = x_aug.c()
+    _check(lib.nvfp4_rmsnorm_reorder_quantize_noalloc(x.data_ptr(), _dtype_code(x), M, K, _ldx(x), _ptr(gamma),
+                                                      ctypes.c_float(eps), _ptr(perm), S, _ptr(scale_in),
+                                                      ctypes.byref(xc), _ptr(dev_status), _stream(stream)),
+           "nvfp4_rmsnorm_reorder_quantize_noalloc")
 
 
 def _out_dtype(y: torch.Tensor) -> int:
