@@ -131,6 +131,8 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K,
   const int sms = num_sms_current_device();
   WsHeader* ws = static_cast<WsHeader*>(workspace);
   const QOut qo = qout(q);
+  if (M * (K / 8) <= quant_small_max_units(dt))   // decode-sized: one launch, no workspace traffic
+    return cuda_status(launch_quant_small(false, x, dt, M, K, ldx, scale_in, nullptr, qo, qo, dev_status, s));
   const float* s_ptr = scale_in;
   if (s_ptr == nullptr) {
     NVFP4_TRY(cuda_status(launch_amax(x, dt, M, K, ldx, ws, 0, q->tensor_scale, dev_status, sms, s)));
@@ -151,6 +153,8 @@ nvfp4_status nvfp4_quantize_residue(const void* x, nvfp4_dtype dt, int64_t M, in
   const int sms = num_sms_current_device();
   WsHeader* ws = static_cast<WsHeader*>(workspace);
   const QOut qo = qout(q), ro = qout(r);
+  if (M * (K / 8) <= quant_small_max_units(dt))
+    return cuda_status(launch_quant_small(true, x, dt, M, K, ldx, scale_in, rscale_in, qo, ro, dev_status, s));
   const float* s_ptr = scale_in;
   if (s_ptr == nullptr) {
     NVFP4_TRY(cuda_status(launch_amax(x, dt, M, K, ldx, ws, 0, q->tensor_scale, dev_status, sms, s)));

@@ -11,13 +11,16 @@
 // Structure (persistent, one CTA per SM, 192 threads):
 //   warp 0     one lane issues TMA loads of A/W code tiles (128 B K-slices,
 //              128-byte swizzle) and bulk copies of the matching scale atoms
-//              into a 4-stage shared-memory ring;
+//              into a 3-stage shared-memory ring;
 //   warp 1     allocates 512 TMEM columns; one lane copies each stage's scale
-//              atoms into TMEM (tcgen05.cp 32x128b.warpx4) and issues 4 MMAs
-//              (K = 64 each) per stage; tcgen05.commit frees the stage and, at
-//              the end of a tile, signals the epilogue;
+//              atoms into TMEM (tcgen05.cp 32x128b.warpx4, two alternating
+//              buffers) interleaved with the 4 MMAs (K = 64 each) of the stage;
+//              tcgen05.commit frees the stage and, at the end of a tile,
+//              signals the epilogue;
 //   warps 2-5  read the 128 x 256 fp32 accumulator (tcgen05.ld 32x32b.x32, one
-//              TMEM lane quadrant per warp), scale by s_a s_w and store Y.
+//              TMEM lane quadrant per warp), scale by s_a s_w, transpose each
+//              32 x 32 chunk through shared memory and store Y with coalesced
+//              16-byte stores.
 // Tiles are 128 x 256 x 256 (M x N x K); tile order walks M fastest so that the
 // CTAs in flight share W tiles through L2.  Every mbarrier wait is bounded: on
 // timeout the kernel records NVFP4_ERR_TIMEOUT, every role leaves its loop, and
@@ -31,19 +34,20 @@ namespace {
 
 constexpr int BM = 128, BN = 256, BK = 256;
 constexpr int BK_BYTES = BK / 2;                 // one 128-byte swizzle row per k-tile
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * BK_BYTES;           // 16 KB
 constexpr int B_BYTES = BN * BK_BYTES;           // 32 KB
 constexpr int SFA_BYTES = 4 * 512;               // 4 k-atoms of one 128-row group
 constexpr int SFB_BYTES = 2 * 4 * 512;           // 2 row groups x 4 k-atoms
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
 constexpr int OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
+constexpr int EPI_BYTES = 4 * 32 * 33 * 4;      // per epilogue warp: a 32 x 32 fp32 tile (+1 pad)
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;    // + alignment slack
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;    // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;                  // 256 fp32 columns
-constexpr uint32_t SFA_COL = 256;                // 4 k-blocks x 4 columns
-constexpr uint32_t SFB_COL = 272;                // 4 k-blocks x 8 columns
+constexpr uint32_t SF_COL = 256;                 // two scale buffers of 48 columns, alternating by stage:
+constexpr uint32_t SF_BUF = 48;                  //   SFA 4 k-blocks x 4 columns, then SFB 4 k-blocks x 8
 constexpr int NUM_THREADS = 192;
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for 128B swizzle");
@@ -56,7 +60,7 @@ struct TcParams {
   const float* w_s;
   void* y;
   int64_t ldy;
-  int y_bf16;
+  int y_vec;       // Y base and row pitch allow 16-byte (fp32) / 8-byte (bf16) stores
   int M, N, K;
   int katoms;      // scale atoms along K per 128-row group = ceil(K / 64)
   int b_groups;    // 128-row groups of W = ceil(N / 128)
@@ -66,12 +70,14 @@ struct TcParams {
 
 // --------------------------------------------------------------- kernel
 
+template <bool BF16OUT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const TcParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  float* epi = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
   uint64_t* full = bars;               // [STAGES] TMA -> MMA
   uint64_t* empty = bars + STAGES;     // [STAGES] MMA -> TMA
   uint64_t* acc_full = bars + 2 * STAGES;
@@ -128,6 +134,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1 && lane == 0) {
     // -------------------------------------------------------- MMA issuer
     const uint32_t idesc = idesc_nvf4(BN);
+    uint32_t sf_flip = 0;
     int s = 0;
     uint32_t ph = 0;
     int local = 0;
@@ -142,15 +149,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int jmax = min(4, (p.K - kt * BK) / 64);
         const uint8_t* st_base = smem + s * STAGE_BYTES;
         const uint32_t a0 = saddr(st_base), b0 = saddr(st_base + OFF_B);
+        // scales of consecutive stages go to alternate TMEM buffers, so copying
+        // this stage's scales does not wait on the previous stage's MMAs
+        const uint32_t sfa = SF_COL + (sf_flip & 1u) * SF_BUF, sfb = sfa + 16u;
+        ++sf_flip;
         for (int j = 0; j < jmax; ++j) {
-          tc_cp_scales(tmem + SFA_COL + 4 * j, desc_sf_atom(saddr(st_base + OFF_SFA + j * 512)));
+          tc_cp_scales(tmem + sfa + 4 * j, desc_sf_atom(saddr(st_base + OFF_SFA + j * 512)));
           for (int g = 0; g < ngroups; ++g)
-            tc_cp_scales(tmem + SFB_COL + 8 * j + 4 * g,
-                         desc_sf_atom(saddr(st_base + OFF_SFB + g * 2048 + j * 512)));
-        }
-        for (int j = 0; j < jmax; ++j) {
+            tc_cp_scales(tmem + sfb + 8 * j + 4 * g, desc_sf_atom(saddr(st_base + OFF_SFB + g * 2048 + j * 512)));
           tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a0) + (uint64_t)(2 * j), desc_sw128(b0) + (uint64_t)(2 * j),
-                      idesc, tmem + SFA_COL + 4 * j, tmem + SFB_COL + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                      idesc, tmem + sfa + 4 * j, tmem + sfb + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
         }
         tc_commit(saddr(&empty[s]));  // stage reusable once these MMAs have read it
         if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -167,42 +175,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
       if (!mbar_wait(saddr(acc_full), (uint32_t)(local & 1), abort_flag, p.st)) break;
       tc_fence_after();
-      const int row = mb * BM + q * 32 + lane;
+      // Each warp owns TMEM lanes (= tile rows) 32q..32q+31.  A 32 x 32 chunk is
+      // read row-per-thread, transposed through shared memory, and written with
+      // 16-byte stores in which 8 lanes cover one 128-byte row segment.
+      float* buf = epi + q * 32 * 33;
+      const int sub_r = lane >> 3, sub_c = (lane & 7) * 4;
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + c * 32, r);
         tmem_ld_wait();
         const int col0 = nb * BN + c * 32;
-        if (row >= p.M || col0 >= p.N) continue;
-        if (p.y_bf16) {
-          __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (int64_t)row * p.ldy + col0;
-          const bool vec = col0 + 32 <= p.N && ((reinterpret_cast<uintptr_t>(yr) & 15u) == 0);
-          if (vec) {
+        if (col0 >= p.N) continue;  // uniform across the warp
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(r[i]) * alpha, __uint_as_float(r[i + 1]) * alpha);
-              v.y = pack_bf16x2(__uint_as_float(r[i + 2]) * alpha, __uint_as_float(r[i + 3]) * alpha);
-              v.z = pack_bf16x2(__uint_as_float(r[i + 4]) * alpha, __uint_as_float(r[i + 5]) * alpha);
-              v.w = pack_bf16x2(__uint_as_float(r[i + 6]) * alpha, __uint_as_float(r[i + 7]) * alpha);
-              *reinterpret_cast<uint4*>(yr + i) = v;
+        for (int i = 0; i < 32; ++i) buf[lane * 33 + i] = __uint_as_float(r[i]) * alpha;
+        __syncwarp();
+        if (p.y_vec && col0 + 32 <= p.N) {
+          // full 32-column chunk of an aligned Y: one 16-byte (fp32) or 8-byte
+          // (bf16) store per lane and row
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int lr = i * 4 + sub_r;
+            const int grow = mb * BM + q * 32 + lr;
+            if (grow < p.M) {
+              const float* src = buf + lr * 33 + sub_c;
+              const int64_t off = (int64_t)grow * p.ldy + col0 + sub_c;
+              if (BF16OUT)
+                *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.y) + off) =
+                    make_uint2(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]));
+              else
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + off) =
+                    make_float4(src[0], src[1], src[2], src[3]);
             }
-          } else {
-            for (int i = 0; i < 32 && col0 + i < p.N; ++i) yr[i] = __float2bfloat16_rn(__uint_as_float(r[i]) * alpha);
           }
         } else {
-          float* yr = reinterpret_cast<float*>(p.y) + (int64_t)row * p.ldy + col0;
-          const bool vec = col0 + 32 <= p.N && ((reinterpret_cast<uintptr_t>(yr) & 15u) == 0);
-          if (vec) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(yr + i) =
-                  make_float4(__uint_as_float(r[i]) * alpha, __uint_as_float(r[i + 1]) * alpha,
-                              __uint_as_float(r[i + 2]) * alpha, __uint_as_float(r[i + 3]) * alpha);
-          } else {
-            for (int i = 0; i < 32 && col0 + i < p.N; ++i) yr[i] = __uint_as_float(r[i]) * alpha;
+          // ragged last chunk or unaligned Y: element stores
+          for (int i = 0; i < 8; ++i) {
+            const int lr = i * 4 + sub_r;
+            const int grow = mb * BM + q * 32 + lr;
+            if (grow >= p.M) continue;
+            const float* src = buf + lr * 33 + sub_c;
+            const int64_t off = (int64_t)grow * p.ldy + col0 + sub_c;
+            for (int e = 0; e < 4 && col0 + sub_c + e < p.N; ++e) {
+              if (BF16OUT)
+                reinterpret_cast<__nv_bfloat16*>(p.y)[off + e] = __float2bfloat16_rn(src[e]);
+              else
+                reinterpret_cast<float*>(p.y)[off + e] = src[e];
+            }
           }
         }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
@@ -260,7 +281,11 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) 
     return cudaErrorInvalidValue;
   TcParams p{};
   p.sfa = g.a_scales; p.sfb = g.w_scales; p.a_s = g.a_s; p.w_s = g.w_s;
-  p.y = g.y; p.ldy = g.ldy; p.y_bf16 = g.y_bf16 ? 1 : 0;
+  p.y = g.y; p.ldy = g.ldy;
+  {
+    const size_t vec_bytes = g.y_bf16 ? 8 : 16, esize = g.y_bf16 ? 2 : 4;
+    p.y_vec = (reinterpret_cast<uintptr_t>(g.y) % vec_bytes == 0) && ((size_t)g.ldy * esize) % vec_bytes == 0;
+  }
   p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K;
   p.katoms = (int)((g.K + 63) / 64);
   p.b_groups = (int)((g.N + 127) / 128);
@@ -269,10 +294,11 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) 
   p.num_tiles = p.m_blocks * p.n_blocks;
   p.k_tiles = (int)((g.K + BK - 1) / BK);
   p.st = g.st;
-  cudaError_t e = cudaFuncSetAttribute(k_gemm_nvf4, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  auto kern = g.y_bf16 ? k_gemm_nvf4<true> : k_gemm_nvf4<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(p.num_tiles, num_sms));
-  k_gemm_nvf4<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
   return cudaGetLastError();
 }
 

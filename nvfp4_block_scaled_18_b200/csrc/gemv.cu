@@ -88,35 +88,37 @@ __global__ void __launch_bounds__(256, 1) k_gemv(GemmArgs g) {
   const int64_t n0 = (int64_t)blockIdx.x * 32;
   const int64_t n = n0 + lane;
   const bool row_ok = n < N;
-  const int64_t T = K / 64;
-  const int64_t t0 = (warp * T) / kWarps, t1 = ((warp + 1) * T) / kWarps;
+  const int T = (int)(K / 64);
+  const int t0 = (warp * T) / kWarps, t1 = ((warp + 1) * T) / kWarps;
   const int64_t cpitch = K / 2, spitch = K / 16;
 
+  // per-lane source pointers, fixed for the whole kernel (step t adds t*32 / t*4)
   const uint8_t* wrow_c = g.w_codes + (row_ok ? n : 0) * cpitch;
   const uint8_t* wrow_s = g.w_scales + (row_ok ? n : 0) * spitch;
   const int wbytes16 = row_ok ? 16 : 0, wbytes4 = row_ok ? 4 : 0;
   const int swz = (lane >> 2) & 1;  // swaps the lane's two 16-byte halves: conflict-free reads
+  // activation slices: lane i < 2*MT copies half h of row m's 32 code bytes, lane m < MT its 4 scale bytes
+  const int xm = lane >> 1, xh = lane & 1;
+  const bool x_lane = lane < 2 * MT, xrow_ok = x_lane && xm < Mreal;
+  const uint8_t* xc_src = g.a_codes + (xrow_ok ? xm : 0) * cpitch + xh * 16;
+  const uint8_t* rc_src = RES ? g.r_codes + (xrow_ok ? xm : 0) * cpitch + xh * 16 : nullptr;
+  const bool s_lane = lane < MT, srow_ok = s_lane && lane < Mreal;
+  const uint8_t* xs_src = g.a_scales + (srow_ok ? lane : 0) * spitch;
+  const uint8_t* rs_src = RES ? g.r_scales + (srow_ok ? lane : 0) * spitch : nullptr;
 
-  auto issue = [&](int64_t t, int slot) {
+  auto issue = [&](int t, int slot) {
     unsigned char* sb = wbase + slot * L::kSlot;
     const uint32_t wc = smem_u32(sb + L::kWc + lane * 32);
     cp_async16(wc + ((0 ^ swz) << 4), wrow_c + t * 32, wbytes16);
     cp_async16(wc + ((1 ^ swz) << 4), wrow_c + t * 32 + 16, wbytes16);
     cp_async4(smem_u32(sb + L::kWs + lane * 4), wrow_s + t * 4, wbytes4);
-    for (int i = lane; i < 2 * MT; i += 32) {
-      const int m = i >> 1, h = i & 1;
-      const bool ok = m < Mreal;
-      cp_async16(smem_u32(sb + L::kXc + m * 32 + h * 16),
-                 g.a_codes + (ok ? m : 0) * cpitch + t * 32 + h * 16, ok ? 16 : 0);
-      if (RES)
-        cp_async16(smem_u32(sb + L::kRc + m * 32 + h * 16),
-                   g.r_codes + (ok ? m : 0) * cpitch + t * 32 + h * 16, ok ? 16 : 0);
+    if (x_lane) {
+      cp_async16(smem_u32(sb + L::kXc + xm * 32 + xh * 16), xc_src + t * 32, xrow_ok ? 16 : 0);
+      if (RES) cp_async16(smem_u32(sb + L::kRc + xm * 32 + xh * 16), rc_src + t * 32, xrow_ok ? 16 : 0);
     }
-    for (int m = lane; m < MT; m += 32) {
-      const bool ok = m < Mreal;
-      cp_async4(smem_u32(sb + L::kXs + m * 4), g.a_scales + (ok ? m : 0) * spitch + t * 4, ok ? 4 : 0);
-      if (RES)
-        cp_async4(smem_u32(sb + L::kRs + m * 4), g.r_scales + (ok ? m : 0) * spitch + t * 4, ok ? 4 : 0);
+    if (s_lane) {
+      cp_async4(smem_u32(sb + L::kXs + lane * 4), xs_src + t * 4, srow_ok ? 4 : 0);
+      if (RES) cp_async4(smem_u32(sb + L::kRs + lane * 4), rs_src + t * 4, srow_ok ? 4 : 0);
     }
   };
 
@@ -170,8 +172,8 @@ __global__ void __launch_bounds__(256, 1) k_gemv(GemmArgs g) {
     if (t0 + i < t1) issue(t0 + i, i);
     cp_async_commit();
   }
-  for (int64_t t = t0; t < t1; ++t) {
-    const int slot = (int)((t - t0) % kStages);
+  int slot = 0;
+  for (int t = t0; t < t1; ++t) {
     cp_async_wait<kStages - 1>();
     __syncwarp();
     expand(slot);
@@ -210,6 +212,7 @@ __global__ void __launch_bounds__(256, 1) k_gemv(GemmArgs g) {
     __syncwarp();
     if (t + kStages < t1) issue(t + kStages, slot);
     cp_async_commit();
+    if (++slot == kStages) slot = 0;
   }
   cp_async_wait<0>();
 

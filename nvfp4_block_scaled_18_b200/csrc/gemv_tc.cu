@@ -10,17 +10,25 @@
 // the epilogue with their own tensor scales: Y = s_x s_w acc + s_r s_w acc_r.
 //
 // Grid: (ks, ceil(N/128)); the ks CTAs of one cluster split K between them and
-// each accumulates a 128 x NP fp32 partial in TMEM.  The partials are written
-// to shared memory and summed across the cluster through distributed shared
-// memory; CTA rank r of the cluster writes rows [r*128/ks, (r+1)*128/ks) of the
-// tile.  Roles inside a CTA (128 threads): warp 0 lane 0 issues TMA/bulk copies
-// into a shared-memory ring, warp 1 lane 0 copies scale atoms to TMEM and
-// issues the MMAs, then all four warps drain the accumulators.
+// each accumulates a 128 x NP fp32 partial in TMEM.  Row r of the tile is owned
+// by cluster rank floor(r*ks/128); every CTA pushes its partial rows straight
+// into the owner's shared memory (distributed shared-memory stores), and after
+// one cluster barrier each owner sums its rows and writes Y.  Roles inside a
+// CTA (128 threads): warp 0 lane 0 issues TMA/bulk copies into a shared-memory
+// ring, warp 1 lane 0 copies scale atoms to TMEM and issues the MMAs, then all
+// four warps drain the accumulators.
 //
-// Safety: every mbarrier wait is bounded; every CTA reaches both cluster
-// barriers on every path; the dynamic shared-memory request caps the CTAs per
-// SM so that their TMEM allocations always fit side by side (no CTA can block
-// in tcgen05.alloc behind a cluster peer).
+// Programmatic dependent launch: the kernel may start while the preceding
+// kernel on the stream (normally the activation quantizer) is still running.
+// Before griddepcontrol.wait it only sets up (barriers, TMEM) and asks L2 to
+// prefetch this CTA's W tiles and scale atoms; L2 is the point of coherence,
+// so a prefetch never yields stale data even if the preceding kernel writes W.
+// Every load that feeds the result is issued after the wait.
+//
+// Safety: every mbarrier wait is bounded; every CTA reaches every cluster
+// barrier on every path; the dynamic shared-memory request covers the whole
+// layout and caps the CTAs per SM so that their TMEM allocations always fit
+// side by side (no CTA can block in tcgen05.alloc behind a cluster peer).
 #include "kernels.h"
 #include "tcgen05.cuh"
 
@@ -50,16 +58,29 @@ struct Cfg {
   static constexpr int BAR = 256;
   // stages: as many as keep two CTAs per SM (four when TMEM allows only one CTA)
   static constexpr int BUDGET = TMEM_CTAS >= 2 ? 114 * 1024 : 224 * 1024;
-  static constexpr int STAGES = (4 * STAGE + BAR + 1024 <= BUDGET) ? 4 : ((3 * STAGE + BAR + 1024 <= BUDGET) ? 3 : 2);
+  // pushed partial rows: every source rank has a slot of ceil(128/ks) rows in
+  // its owner, ks * ceil(128/ks) <= 135 rows for ks <= 8
   static constexpr int PITCH = NP + 4;                            // floats per partial row (padded)
-  static constexpr int PART = 128 * PITCH * 4 * (RES ? 2 : 1);   // overlays the idle stage ring
-  static constexpr int SMEM_NEED = STAGES * STAGE + BAR + 1024;
+  static constexpr int PART_ROWS = 136;
+  static constexpr int PART = PART_ROWS * PITCH * 4 * (RES ? 2 : 1);
+  // a dedicated partial area (peers may push as soon as this CTA has started)
+  // when it still leaves three stages; otherwise it overlays the stage ring
+  static constexpr bool PART_OWN = PART <= 40 * 1024 && 3 * STAGE + PART + BAR + 1024 <= BUDGET;
+  static constexpr int PART_DED = PART_OWN ? PART : 0;
+  static constexpr int STAGES = (4 * STAGE + PART_DED + BAR + 1024 <= BUDGET)
+                                    ? 4
+                                    : ((3 * STAGE + PART_DED + BAR + 1024 <= BUDGET) ? 3 : 2);
+  // layout from the 1024-aligned base: ring | dedicated partials | barriers;
+  // +1024 covers the alignment of the dynamic shared-memory base
+  static constexpr int SMEM_NEED = STAGES * STAGE + PART_DED + BAR + 1024;
   // request that keeps at most TMEM_CTAS CTAs on an SM, so tcgen05.alloc never waits on a peer
   static constexpr int SMEM_MIN = 233472 / (TMEM_CTAS + 1) + 1024;
   static constexpr int SMEM = SMEM_NEED > SMEM_MIN ? SMEM_NEED : SMEM_MIN;
   static constexpr int CTAS_PER_SM = (233472 / (SMEM + 1024)) < TMEM_CTAS ? (233472 / (SMEM + 1024)) : TMEM_CTAS;
+  static_assert(1023 + STAGES * STAGE + PART_DED + BAR <= SMEM, "layout exceeds the shared-memory request");
+  static_assert((2 * STAGES + 1) * 8 + 8 <= BAR, "barrier block");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(PART <= STAGES * STAGE, "partials overlay the stage ring");
+  static_assert(PART_OWN || PART <= STAGES * STAGE, "partials overlay the stage ring");
   static_assert(233472 / (SMEM + 1024) <= TMEM_CTAS, "TMEM must fit every co-resident CTA");
   static_assert(CTAS_PER_SM >= 1, "residency");
 };
@@ -78,32 +99,6 @@ struct SwapParams {
   int* st;
 };
 
-template <int NP>
-__device__ __forceinline__ void drain_acc(uint32_t taddr, float* row_out) {
-  if constexpr (NP == 16) {
-    uint32_t r[16];
-    tmem_ld16(taddr, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 16; i += 4)
-      *reinterpret_cast<float4*>(row_out + i) =
-          make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
-                      __uint_as_float(r[i + 3]));
-  } else {
-#pragma unroll
-    for (int c = 0; c < NP; c += 32) {
-      uint32_t r[32];
-      tmem_ld32(taddr + c, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; i += 4)
-        *reinterpret_cast<float4*>(row_out + c + i) =
-            make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
-                        __uint_as_float(r[i + 3]));
-    }
-  }
-}
-
 template <int NP, bool RES, bool BF16OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemv_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -111,13 +106,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<NP, RES>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* part = reinterpret_cast<float*>(smem);    // reused once the mainloop is over
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE);
+  float* part = reinterpret_cast<float*>(C::PART_OWN ? smem + C::STAGES * C::STAGE : smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE + C::PART_DED);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* acc_full = bars + 2 * C::STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  griddep_launch_dependents();   // the next kernel may set itself up; it waits for this one's results
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank(), ks = cluster_nctarank();
@@ -140,10 +137,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  // with a dedicated partial area, peers may push into it once they know this
+  // CTA is running: announce it now, they wait for it before their first push
+  if (C::PART_OWN) cluster_arrive_relaxed();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // warm L2 with this CTA's W tiles and scale atoms while the preceding kernel finishes
+    for (int kt = kt0; kt < kt1; ++kt) {
+      prefetch_l2_tile_2d(&tmW, kt * 128, rt * 128);
+      prefetch_l2_bulk(p.sfw + ((size_t)rt * p.katoms_w + kt * 4) * 512,
+                       (uint32_t)min(4, (p.K - kt * 256) / 64) * 512u);
+    }
+  }
+  griddep_wait();   // X, R, the scales and the tensor scales come from the preceding kernel
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------- TMA producer
@@ -196,46 +206,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncwarp();
 
-  // ----------------------------------------- drain partials into shared memory
+  // ------------------- push this CTA's partial rows to the CTA that owns them
+  // Owner o = floor(r*ks/128) holds rows [ceil(o*128/ks), ceil((o+1)*128/ks))
+  // of the tile, at most ceil(128/ks) rows, and keeps one slot of that many
+  // rows per source rank.
   const bool ok = mbar_wait(saddr(acc_full), 0u, abort_flag, p.st);
   tc_fence_after();
+  __syncwarp();     // the cluster barriers below are warp-aligned
+  if (!C::PART_OWN) {
+    // the partials overlay the ring: a peer's ring is free once its MMAs are done
+    tc_fence_before();
+    cluster_arrive();
+  }
+  cluster_wait();   // dedicated area: pairs with the arrive at start-up
+  tc_fence_after();
+  const int rows_max = (int)((128u + ks - 1) / ks);
+  auto owner_row0 = [&](uint32_t o) { return (int)((o * 128u + ks - 1) / ks); };
   {
     const int row = warp * 32 + lane;                              // TMEM lane = W row of the tile
+    const uint32_t o = (uint32_t)row * ks / 128u;
+    const int slot = (int)rank * rows_max + (row - owner_row0(o));
+    const uint32_t dst = mapa_shared(saddr(part + slot * C::PITCH), o);
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    if (ok) {
-      drain_acc<NP>(lane_addr + C::ACC, part + row * C::PITCH);
-      if (RES) drain_acc<NP>(lane_addr + C::ACC_R, part + (128 + row) * C::PITCH);
-    } else {
-      for (int i = 0; i < NP; ++i) part[row * C::PITCH + i] = 0.0f;
+#pragma unroll
+    for (int acc_i = 0; acc_i < (RES ? 2 : 1); ++acc_i) {
+      const uint32_t dsti = dst + (uint32_t)(acc_i * C::PART_ROWS * C::PITCH * 4);
+      const uint32_t src = lane_addr + (acc_i ? C::ACC_R : C::ACC);
+#pragma unroll
+      for (int c = 0; c < NP; c += 16) {
+        uint32_t r[16];
+        tmem_ld16(src + c, r);
+        tmem_ld_wait();
+        if (!ok) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+          st_cluster_f32x4(dsti + (uint32_t)((c + i) * 4), __uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                           __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+      }
     }
   }
   tc_fence_before();
-  cluster_sync();
+  cluster_sync();   // every partial has landed in its owner's shared memory
 
-  // -------------------------------- reduce the K-split partials across the cluster
+  // ------------------------------------------------ owners sum their rows and store
   {
-    const int r0 = (int)((rank * 128u) / ks), r1 = (int)(((rank + 1) * 128u) / ks);
+    const int r0 = owner_row0(rank), r1 = owner_row0(rank + 1);
     const int nrows = r1 - r0;
     const float alpha = (*p.x_s) * (*p.w_s);
     const float alpha_r = RES ? (*p.r_s) * (*p.w_s) : 0.0f;
-    const uint32_t part_base = saddr(part);
     for (int idx = threadIdx.x; idx < nrows * p.M; idx += kThreads) {
       const int m = idx / nrows, i = idx - m * nrows;
       const int n = rt * 128 + r0 + i;
       if (n >= p.N) continue;
-      const uint32_t off = (uint32_t)(((r0 + i) * C::PITCH + m) * 4);
-      // issue every peer load before the first add so their latencies overlap
-      float v[8], vr[8];
-#pragma unroll
-      for (uint32_t pr = 0; pr < 8; ++pr) {
-        v[pr] = pr < ks ? ld_cluster_f32(mapa_shared(part_base + off, pr)) : 0.0f;
-        if (RES) vr[pr] = pr < ks ? ld_cluster_f32(mapa_shared(part_base + off + 128u * C::PITCH * 4u, pr)) : 0.0f;
-      }
       float sum = 0.0f, sum_r = 0.0f;
-#pragma unroll
-      for (int pr = 0; pr < 8; ++pr) {
-        sum += v[pr];
-        if (RES) sum_r += vr[pr];
+      for (uint32_t src = 0; src < ks; ++src) {
+        const int slot = (int)src * rows_max + i;
+        sum += part[slot * C::PITCH + m];
+        if (RES) sum_r += part[C::PART_ROWS * C::PITCH + slot * C::PITCH + m];
       }
       const float out = RES ? fmaf(sum, alpha, sum_r * alpha_r) : sum * alpha;
       if (BF16OUT)
@@ -244,7 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         reinterpret_cast<float*>(p.y)[(int64_t)m * p.ldy + n] = out;
     }
   }
-  cluster_sync();  // peers may still be reading this CTA's partials until here
 
   if (warp == 1) {
     __syncwarp();
@@ -284,13 +313,15 @@ cudaError_t launch_np(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the preceding kernel's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, tmR, p);
 }
 

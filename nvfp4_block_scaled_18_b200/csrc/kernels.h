@@ -32,6 +32,13 @@ cudaError_t launch_quant(int mode, const void* x, nvfp4_dtype dt, int64_t M, int
 cudaError_t launch_rms_stats(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                              const void* gamma, float eps, WsHeader* ws, float* rinv, float* s_out,
                              bool want_scale, int* st, int num_sms, cudaStream_t stream);
+// One-launch quantizer for inputs of at most quant_small_max_units(dt) 8-element
+// units (M * K / 8); returns cudaErrorNotSupported above that.  With residue,
+// r receives the residue; null s_in / sr_in mean "compute the tensor scale".
+int64_t quant_small_max_units(nvfp4_dtype dt);
+cudaError_t launch_quant_small(bool residue, const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                               const float* s_in, const float* sr_in, const QOut& q, const QOut& r, int* st,
+                               cudaStream_t stream);
 size_t reorder_smem_bytes(nvfp4_dtype dt, int64_t K, bool has_gamma);
 cudaError_t launch_reorder_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                  const void* gamma, const float* rinv, const int32_t* perm,

@@ -19,6 +19,7 @@
 // 16-element block and exchange their half-block maxima with one shuffle.
 #include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace nvfp4 {
 
@@ -152,6 +153,158 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
   }
   if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
   if (MODE == Q_MAIN_AMAXR) finish_tensor_scale(rkey, &ws->amax_bits[1], &ws->arrive[1], r.s, st);
+}
+
+// ------------------------------------------------- single-launch small inputs
+// Decode-sized activations (a few rows) are too small to hide two or three
+// dependent launches.  One cluster of kQC CTAs quantizes the whole tensor in
+// one launch: each thread keeps its 8-element units in registers, the CTAs
+// exchange their |x| maxima through distributed shared memory behind a cluster
+// barrier, and every CTA derives the same tensor scale.  The arithmetic is the
+// same quant_half_block as above, so codes and scales are identical to the
+// multi-launch path.
+
+constexpr int kQC = 8;              // CTAs per cluster (portable cluster size)
+constexpr int kQThreads = 512;      // threads per CTA
+constexpr int kQUnitsPerChunk = kQC * kQThreads;
+
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
+  __device__ __forceinline__ void get(float v[8]) const {
+    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    v[4] = __uint_as_float(u.z << 16); v[5] = __uint_as_float(u.z & 0xFFFF0000u);
+    v[6] = __uint_as_float(u.w << 16); v[7] = __uint_as_float(u.w & 0xFFFF0000u);
+  }
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.0f, 0.0f, 0.0f, 0.0f); }
+  __device__ __forceinline__ void get(float v[8]) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+// Cluster-wide maximum of `key` (every thread of the cluster calls it with the
+// same `slot`, a word this CTA publishes to its peers).  Result in every thread.
+__device__ __forceinline__ uint32_t cluster_max_u32(uint32_t key, uint32_t* red, uint32_t* slot) {
+  const uint32_t m = block_max_u32(key, red);
+  if (threadIdx.x == 0) *slot = m;
+  tc::cluster_sync();  // release/acquire: every CTA's slot is visible cluster-wide
+  const int lane = threadIdx.x & 31;
+  uint32_t a = 0u;
+  if (lane < kQC) a = __float_as_uint(tc::ld_cluster_f32(tc::mapa_shared(tc::saddr(slot), (uint32_t)lane)));
+  return warp_max_u32(a);
+}
+
+// Tensor scale from a |.| maximum key: fl32(amax / 2688), or 0 with
+// NVFP4_ERR_NONFINITE for an Inf/NaN maximum (reported once per cluster).
+__device__ __forceinline__ float scale_from_key(uint32_t a, bool reporter, int* st) {
+  if (a >= 0x7F800000u) {
+    if (reporter) report_status(st, NVFP4_ERR_NONFINITE);
+    return 0.0f;
+  }
+  return __fdiv_rn(__uint_as_float(a), 2688.0f);
+}
+
+// Unit u (8 elements) of this thread's i-th chunk.  Grid: exactly one cluster.
+template <typename T, int R, bool RES>
+__global__ void __launch_bounds__(kQThreads, 1)
+    k_quant_cluster(const T* __restrict__ x, int M, int K, int64_t ldx, const float* s_in,
+                    const float* sr_in, QOut q, QOut r, int* st) {
+  __shared__ uint32_t red[kQThreads / 32];
+  __shared__ uint32_t xch[2];       // published maxima: [0] |x|, [1] |residue|
+  // programmatic dependent launch: let the next kernel set itself up, and wait
+  // for the preceding one before reading x
+  tc::griddep_launch_dependents();
+  tc::griddep_wait();
+  const uint32_t rank = tc::cluster_ctarank();
+  const int upr = K >> 3;
+  const int U = M * upr;
+  const bool reporter = rank == 0 && threadIdx.x == 0;
+
+  Raw8<T> raw[R];
+  uint32_t key = 0u;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
+    if (u < U) {
+      const int row = u / upr, c8 = u - row * upr;
+      raw[i].load(x + (int64_t)row * ldx + (int64_t)c8 * 8);
+    } else {
+      raw[i].zero();
+    }
+    float v[8];
+    raw[i].get(v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
+  }
+  if (key >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
+
+  const bool exchange = s_in == nullptr || (RES && sr_in == nullptr);   // uniform
+  const float s = s_in != nullptr ? *s_in : scale_from_key(cluster_max_u32(key, red, &xch[0]), reporter, st);
+  float s_r = (RES && sr_in != nullptr) ? *sr_in : 0.0f;
+  if (reporter) {
+    if (q.s != s_in) *q.s = s;
+    if (RES && sr_in != nullptr && r.s != sr_in) *r.s = s_r;
+  }
+
+  uint32_t rkey = 0u;
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
+    const bool act = u < U;
+    const int row = act ? u / upr : 0, c8 = act ? u - row * upr : 0;
+    float v[8], deq[8];
+    raw[i].get(v);
+    uint32_t db;
+    const uint32_t codes = quant_half_block(v, s, db, RES ? deq : nullptr);
+    if (act) store_half_block(q, row, c8, codes, db);
+    if (RES) {
+      float rv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) rv[j] = __fsub_rn(v[j], deq[j]);
+      if (sr_in != nullptr) {
+        uint32_t dr;
+        const uint32_t rc = quant_half_block(rv, s_r, dr, nullptr);
+        if (act) store_half_block(r, row, c8, rc, dr);
+      } else if (act) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rkey = max(rkey, abs_key(rv[j]));
+      }
+    }
+  }
+
+  if (RES && sr_in == nullptr) {
+    s_r = scale_from_key(cluster_max_u32(rkey, red, &xch[1]), reporter, st);
+    if (reporter) *r.s = s_r;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
+      const bool act = u < U;
+      const int row = act ? u / upr : 0, c8 = act ? u - row * upr : 0;
+      float v[8], deq[8], rv[8];
+      raw[i].get(v);
+      uint32_t db, dr;
+      (void)quant_half_block(v, s, db, deq);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) rv[j] = __fsub_rn(v[j], deq[j]);
+      const uint32_t rc = quant_half_block(rv, s_r, dr, nullptr);
+      if (act) store_half_block(r, row, c8, rc, dr);
+    }
+  }
+  if (exchange) tc::cluster_sync();  // peers may read this CTA's xch words until here
 }
 
 // ----------------------------------------------------------- ARCQuant path
@@ -288,6 +441,60 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
 }
 
 // ------------------------------------------------------------ launchers
+
+// ------------------------------------------------- single-launch small inputs
+
+int64_t quant_small_max_units(nvfp4_dtype dt) {
+  return (int64_t)kQUnitsPerChunk * (dt == NVFP4_BF16 ? 16 : 8);
+}
+
+template <typename T, int R, bool RES>
+cudaError_t launch_quant_cluster_r(const void* x, int64_t M, int64_t K, int64_t ldx, const float* s_in,
+                                   const float* sr_in, const QOut& q, const QOut& r, int* st,
+                                   cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kQC, 1, 1);
+  cfg.blockDim = dim3(kQThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kQC;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the preceding kernel's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, k_quant_cluster<T, R, RES>, static_cast<const T*>(x), (int)M, (int)K, ldx,
+                            s_in, sr_in, q, r, st);
+}
+
+template <typename T, bool RES>
+cudaError_t launch_quant_cluster_t(const void* x, int64_t M, int64_t K, int64_t ldx, const float* s_in,
+                                   const float* sr_in, const QOut& q, const QOut& r, int* st,
+                                   cudaStream_t stream) {
+  const int64_t chunks = (M * (K >> 3) + kQUnitsPerChunk - 1) / kQUnitsPerChunk;
+  if (chunks <= 1) return launch_quant_cluster_r<T, 1, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
+  if (chunks <= 2) return launch_quant_cluster_r<T, 2, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
+  if (chunks <= 4) return launch_quant_cluster_r<T, 4, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
+  if (chunks <= 8) return launch_quant_cluster_r<T, 8, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
+  if constexpr (sizeof(T) == 2) {
+    if (chunks <= 16) return launch_quant_cluster_r<T, 16, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
+  }
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_quant_small(bool residue, const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                               const float* s_in, const float* sr_in, const QOut& q, const QOut& r, int* st,
+                               cudaStream_t stream) {
+  if (M * (K >> 3) > quant_small_max_units(dt)) return cudaErrorNotSupported;
+  if (dt == NVFP4_BF16)
+    return residue ? launch_quant_cluster_t<__nv_bfloat16, true>(x, M, K, ldx, s_in, sr_in, q, r, st, stream)
+                   : launch_quant_cluster_t<__nv_bfloat16, false>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
+  return residue ? launch_quant_cluster_t<float, true>(x, M, K, ldx, s_in, sr_in, q, r, st, stream)
+                 : launch_quant_cluster_t<float, false>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
+}
 
 static inline dim3 quant_grid(int64_t M, int64_t K, int num_sms) {
   const int64_t upr = K >> 3;

@@ -176,6 +176,17 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   return v;
 }
 
+// L2 prefetch of one TMA tile / of a contiguous range (16-byte aligned, size a
+// multiple of 16).  Hints only: nothing completes or waits on them.
+__device__ __forceinline__ void prefetch_l2_tile_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // The driver's tensor-map encoder, resolved at run time (no libcuda link).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 

@@ -140,7 +140,7 @@ def test_e4m3_exhaustive_through_quantizer(orc):
 
 # ------------------------------------------------------------------ residue
 
-@pytest.mark.parametrize("M,K", [(1, 5120), (4, 27648), (16, 5120), (64, 5120), (3, 80)])
+@pytest.mark.parametrize("M,K", [(1, 5120), (4, 27648), (16, 5120), (16, 27648), (64, 5120), (128, 5120), (3, 80)])
 def test_resserve_residue(orc, M, K):
     x = wl.resserve_x(M, K)
     xt = to_dev(x)
@@ -215,3 +215,45 @@ def test_rmsnorm_identity_perm_f32_and_ragged(orc):
                                       eps=1e-6, S=S, workspace=nv.Workspace(M, K))
     torch.cuda.synchronize()
     assert_same_q(xa, orc.rmsnorm_reorder_quantize(x, gamma, 1e-6, None, S))
+
+
+# ----------------------------------------- one-launch (small) vs multi-launch path
+
+# Inputs of at most 65536 (bf16) / 32768 (fp32) 8-element units run as one
+# cluster launch; larger ones as amax + quantize launches.  Both sides of the
+# boundary, plain and residue, computed and given tensor scales.
+@pytest.mark.parametrize("M,K,dt", [(16, 32768, torch.bfloat16), (17, 32768, torch.bfloat16),
+                                    (8, 32768, torch.float32), (9, 32768, torch.float32),
+                                    (5, 2048, torch.float32)])
+@pytest.mark.parametrize("given", [False, True])
+def test_quantize_paths_at_threshold(orc, M, K, dt, given):
+    x = wl.resserve_x(M, K)
+    xt = to_dev(x, dt)
+    s_in = np.float32(0.0035) if given else None
+    q = run_quantize(xt, nv.SF_TILED, scale_in=s_in)
+    assert_same_q(q, orc.quantize(x, s_in), f"plain M={M} K={K}")
+    q, r = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED), nv.NVFP4Tensor.empty(M, K, nv.SF_TILED)
+    ws = nv.Workspace(M, K)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kw = {}
+    if given:
+        kw = dict(scale_in=torch.tensor([s_in], device="cuda"),
+                  rscale_in=torch.tensor([np.float32(4e-4)], device="cuda"))
+    nv.nvfp4_quantize_residue(xt, q, r, workspace=ws, dev_status=st, **kw)
+    torch.cuda.synchronize()
+    assert st.item() == 0 and int(ws.buf.count_nonzero()) == 0
+    oq, orr = orc.quantize_residue(x, s_in, np.float32(4e-4)) if given else orc.quantize_residue(x)
+    assert_same_q(q, oq, "main")
+    assert_same_q(r, orr, "residue")
+
+
+def test_nonfinite_reported_multi_launch():
+    x = torch.ones((600, 4096), dtype=torch.float32, device="cuda")
+    x[599, 4095] = float("inf")
+    q = nv.NVFP4Tensor.empty(600, 4096)
+    ws = nv.Workspace(600, 4096)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_quantize(x, q, workspace=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 5
+    assert int(ws.buf.count_nonzero()) == 0
