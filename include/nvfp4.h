@@ -131,10 +131,17 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64
  * (ARCQuant post section 3.1-3.2: "unified GEMM call").
  * Kernel choice (K % 64 == 0 always):
  *   ROWMAJOR scales on both operands, M <= 16: CUDA-core decode GEMV;
- *   TILED scales on both operands, M <= 128: tensor-core few-row kernel (W is
- *     the 128-row MMA operand, K split across a thread-block cluster), K >= 256;
+ *   TILED W scales, M <= 16 (A in either layout): tensor-core decode kernel (W
+ *     is the 128-row MMA operand, K split across a thread-block cluster of up
+ *     to 16 CTAs), K >= 256;
+ *   TILED scales on both operands, 16 < M <= 128: tensor-core few-row kernel,
+ *     K >= 256;
  *   TILED scales, M > 128: tensor-core 128x256-tile GEMM, K >= 256.
  *   Other combinations return NVFP4_ERR_UNSUPPORTED.
+ * The tensor-core decode and few-row kernels may start before the preceding
+ * kernel on `stream` has finished (programmatic dependent launch); they read
+ * nothing that kernel produces until it has completed, so stream order is
+ * preserved.
  * y: device, aligned to sizeof(out_dt), row stride ldy >= N elements. */
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y,
                         nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
@@ -146,6 +153,36 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y,
 nvfp4_status nvfp4_gemm_residue(const nvfp4_tensor* a, const nvfp4_tensor* r,
                                 const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt, int64_t ldy,
                                 int* dev_status, void* stream);
+
+/* Decode linear with online activation quantization, in one kernel launch:
+ *   q <- nvfp4_quantize(X, scale_in)            (identical codes, scales, s)
+ *   y <- nvfp4_gemm(q, w)                        (same accumulation as above)
+ * The ks CTAs of each thread-block cluster together read all of X, agree on
+ * s = fl32(amax|X| / 2688) through distributed shared memory and encode their
+ * K-slice directly into the MMA operand; q is written as a by-product.  This
+ * is the decode step of the pages' pipeline (quantize activations, then the
+ * W4A4 GEMM) without the global-memory round trip of Q(X) in between.
+ * Requirements: M <= 16, K % 64 == 0, K >= 256, w with TILED scales, and
+ * M * K / 8 <= 65536 (bf16) / 32768 (fp32); otherwise NVFP4_ERR_UNSUPPORTED.
+ * q: M x K output in either scale layout.  No workspace is needed.  When the
+ * activation slice of a CTA does not fit its registers the call runs two
+ * launches (one-launch quantizer, then the decode kernel) with identical
+ * results.  Other arguments as nvfp4_quantize and nvfp4_gemm. */
+nvfp4_status nvfp4_quantize_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                 const float* scale_in, nvfp4_tensor* q, const nvfp4_tensor* w, void* y,
+                                 nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
+
+/* ResServe compensated decode linear with online quantization of X and of its
+ * residue, in one kernel launch:
+ *   (q, r) <- nvfp4_quantize_residue(X, scale_in, rscale_in)
+ *   y <- nvfp4_gemm_residue(q, r, w)
+ * The residue tensor scale needs a second cluster-wide maximum.  r may be
+ * NULL (then this is nvfp4_quantize_gemm).  Requirements and other arguments
+ * as nvfp4_quantize_gemm; r has the same shape and scale layout as q. */
+nvfp4_status nvfp4_quantize_residue_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                         const float* scale_in, const float* rscale_in, nvfp4_tensor* q,
+                                         nvfp4_tensor* r, const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt,
+                                         int64_t ldy, int* dev_status, void* stream);
 
 /* Largest M accepted by nvfp4_rmsnorm_reorder_quantize_noalloc. */
 #define NVFP4_NOALLOC_MAX_ROWS 65536

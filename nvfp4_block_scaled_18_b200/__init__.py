@@ -25,7 +25,8 @@ SF_ROWMAJOR, SF_TILED = 0, 1
 
 EXPORTED_SYMBOLS = ("nvfp4_scales_bytes", "nvfp4_workspace_size", "nvfp4_quantize",
                     "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize", "nvfp4_gemm",
-                    "nvfp4_gemm_residue", "nvfp4_rmsnorm_reorder_quantize_noalloc",
+                    "nvfp4_gemm_residue", "nvfp4_quantize_gemm", "nvfp4_quantize_residue_gemm",
+                    "nvfp4_rmsnorm_reorder_quantize_noalloc",
                     "nvfp4_status_string", "nvfp4_version")
 NVFP4_NOALLOC_MAX_ROWS = 65536
 
@@ -66,6 +67,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                                T, P, P]
         lib.nvfp4_gemm.argtypes = [T, T, P, ctypes.c_int, I64, P, P]
         lib.nvfp4_gemm_residue.argtypes = [T, T, T, P, ctypes.c_int, I64, P, P]
+        lib.nvfp4_quantize_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, P, T, T, P, ctypes.c_int, I64, P, P]
+        lib.nvfp4_quantize_residue_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, T, T, T, P,
+                                                    ctypes.c_int, I64, P, P]
         for fn in ("nvfp4_quantize", "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize",
                    "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_gemm", "nvfp4_gemm_residue"):
             getattr(lib, fn).restype = ctypes.c_int
@@ -250,3 +254,35 @@ def nvfp4_gemm_residue(a: NVFP4Tensor, r: NVFP4Tensor, w: NVFP4Tensor, y: torch.
     _check(lib.nvfp4_gemm_residue(ctypes.byref(ac), ctypes.byref(rc), ctypes.byref(wc), y.data_ptr(),
                                   _out_dtype(y), _ldx(y), _ptr(dev_status), _stream(stream)),
            "nvfp4_gemm_residue")
+
+
+def nvfp4_quantize_gemm(x: torch.Tensor, q: NVFP4Tensor, w: NVFP4Tensor, y: torch.Tensor,
+                        scale_in: Optional[torch.Tensor] = None,
+                        dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Decode linear with online activation quantization in one launch:
+    q <- Q(x), y <- s_x s_w Q(x) W^T (M <= 16, W with TILED scales)."""
+    lib = load_library()
+    M, K = x.shape
+    qc, wc = q.c(), w.c()
+    _check(lib.nvfp4_quantize_gemm(x.data_ptr(), _dtype_code(x), M, K, _ldx(x), _ptr(scale_in),
+                                   ctypes.byref(qc), ctypes.byref(wc), y.data_ptr(), _out_dtype(y), _ldx(y),
+                                   _ptr(dev_status), _stream(stream)),
+           "nvfp4_quantize_gemm")
+
+
+def nvfp4_quantize_residue_gemm(x: torch.Tensor, q: NVFP4Tensor, r: Optional[NVFP4Tensor], w: NVFP4Tensor,
+                                y: torch.Tensor, scale_in: Optional[torch.Tensor] = None,
+                                rscale_in: Optional[torch.Tensor] = None,
+                                dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """ResServe compensated decode linear in one launch: (q, r) <- Q(x), Q(x - deq Q(x));
+    y <- s_x s_w Q(x) W^T + s_r s_w Q(r) W^T."""
+    lib = load_library()
+    M, K = x.shape
+    qc, wc = q.c(), w.c()
+    rc = r.c() if r is not None else None
+    _check(lib.nvfp4_quantize_residue_gemm(x.data_ptr(), _dtype_code(x), M, K, _ldx(x), _ptr(scale_in),
+                                           _ptr(rscale_in), ctypes.byref(qc),
+                                           ctypes.byref(rc) if rc is not None else None, ctypes.byref(wc),
+                                           y.data_ptr(), _out_dtype(y), _ldx(y), _ptr(dev_status),
+                                           _stream(stream)),
+           "nvfp4_quantize_residue_gemm")

@@ -94,6 +94,15 @@ nvfp4_status run_gemm(const nvfp4_tensor* a, const nvfp4_tensor* r, const nvfp4_
   cudaError_t e;
   if (rowmajor && g.M <= 16) {
     e = launch_gemv(g, num_sms_current_device(), s);              // CUDA-core decode GEMV
+  } else if (w->sf_layout == NVFP4_SF_TILED && g.M <= 16) {
+    DecodeArgs d{};                                               // tensor-core decode kernel
+    d.x_codes = a->codes; d.x_scales = a->scales; d.x_s = a->tensor_scale;
+    if (r) { d.r_codes = r->codes; d.r_scales = r->scales; d.r_s = r->tensor_scale; }
+    d.x_tiled = a->sf_layout == NVFP4_SF_TILED;
+    d.w_codes = w->codes; d.w_scales = w->scales; d.w_s = w->tensor_scale;
+    d.y = y; d.ldy = ldy; d.y_bf16 = out_dt == NVFP4_BF16;
+    d.M = g.M; d.N = g.N; d.K = g.K; d.st = dev_status;
+    e = launch_decode_tc(d, num_sms_current_device(), s);
   } else if (tiled && g.M <= 128) {
     e = launch_gemv_tc(g, num_sms_current_device(), s);           // tensor cores, operands swapped
   } else if (tiled && r == nullptr) {
@@ -204,6 +213,46 @@ nvfp4_status nvfp4_gemm_residue(const nvfp4_tensor* a, const nvfp4_tensor* r, co
                                 void* stream) {
   if (r == nullptr) return NVFP4_ERR_INVALID_ARG;
   return run_gemm(a, r, w, y, out_dt, ldy, dev_status, stream);
+}
+
+nvfp4_status nvfp4_quantize_residue_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                         const float* scale_in, const float* rscale_in, nvfp4_tensor* q,
+                                         nvfp4_tensor* r, const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt,
+                                         int64_t ldy, int* dev_status, void* stream) {
+  NVFP4_TRY(check_input(x, dt, M, K, ldx));
+  NVFP4_TRY(check_tensor(q, M, K));
+  if (r != nullptr) {
+    NVFP4_TRY(check_tensor(r, M, K));
+    if (r->sf_layout != q->sf_layout) return NVFP4_ERR_UNSUPPORTED;
+  }
+  NVFP4_TRY(check_gemm_operands(q, r, w, y, out_dt, ldy));
+  if (M > 16 || w->sf_layout != NVFP4_SF_TILED || K < 256) return NVFP4_ERR_UNSUPPORTED;
+  if (M * (K / 8) > quant_small_max_units(dt)) return NVFP4_ERR_UNSUPPORTED;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = num_sms_current_device();
+  DecodeArgs d{};
+  d.x = x; d.x_bf16 = dt == NVFP4_BF16; d.ldx = ldx;
+  d.s_in = scale_in; d.sr_in = r ? rscale_in : nullptr;
+  d.q_out = qout(q);
+  if (r) d.r_out = qout(r);
+  d.w_codes = w->codes; d.w_scales = w->scales; d.w_s = w->tensor_scale;
+  d.y = y; d.ldy = ldy; d.y_bf16 = out_dt == NVFP4_BF16;
+  d.M = M; d.N = w->rows; d.K = K; d.st = dev_status;
+  cudaError_t e = launch_decode_tc(d, sms, s);
+  if (e != cudaErrorNotSupported) return cuda_status(e);
+  // the activation slice does not fit the fused kernel's registers: quantize
+  // in one launch, then run the same kernel on the NVFP4 operands
+  const QOut qo = qout(q), ro = r ? qout(r) : qout(q);
+  NVFP4_TRY(cuda_status(launch_quant_small(r != nullptr, x, dt, M, K, ldx, scale_in, d.sr_in, qo, ro,
+                                           dev_status, s)));
+  return run_gemm(q, r, w, y, out_dt, ldy, dev_status, stream);
+}
+
+nvfp4_status nvfp4_quantize_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                 const float* scale_in, nvfp4_tensor* q, const nvfp4_tensor* w, void* y,
+                                 nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream) {
+  return nvfp4_quantize_residue_gemm(x, dt, M, K, ldx, scale_in, nullptr, q, nullptr, w, y, out_dt, ldy,
+                                     dev_status, stream);
 }
 
 const char* nvfp4_status_string(nvfp4_status st) {

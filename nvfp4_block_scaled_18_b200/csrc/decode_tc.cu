@@ -1,0 +1,568 @@
+// Decode-sized NVFP4 linear (M <= 16 activation rows) on the tensor cores,
+// optionally fused with the online quantization of the activations, sm_100a.
+//
+// Y^T = W X^T with W (N x K, NVFP4, TILED scales) as the 128-row A operand of
+// tcgen05.mma.kind::mxf4nvf4.block_scale.block16 and the activation rows
+// (padded to N = 16) as the B operand.  With a residue R (ResServe abstract:
+// FP4 base plus FP4 residue, combined on-chip) the same W tile feeds a second
+// accumulator: Y = s_x s_w acc + s_r s_w acc_r.
+//
+// Fused mode (nvfp4_quantize_gemm): the kernel reads X in bf16/fp32 and
+// quantizes it itself.  The ks CTAs of a cluster split K; together they cover
+// the whole of X, so the tensor scale s = fl32(amax|X| / 2688) comes from one
+// exchange of per-CTA maxima through distributed shared memory, and each CTA
+// encodes its K-slice straight into shared memory in the MMA operand layout
+// (the encoding routine is the quantizer's, so codes and scales are
+// identical).  The cluster of the first 128-row tile also writes Q(X) (and
+// Q(R)) to global memory.  This removes the separate quantizer launch and the
+// hand-off between the two kernels from every decode call.
+// Plain mode (nvfp4_gemm): X codes arrive by TMA, X scales are gathered.
+//
+// Activation scales sit in shared memory as the four 512-byte scale atoms of
+// each k-tile (TILED layout of row group 0: line n holds row n's 4 block
+// scales of that K=64 chunk), one tcgen05.cp per MMA.  The scale operands of a
+// block-scaled MMA must start on a 4-column TMEM boundary, so one copy cannot
+// serve several MMAs.
+//
+// Grid: (ks, ceil(N/128)), cluster (ks, 1, 1), ks <= 16.  CTA rank r of a
+// cluster handles k-tiles [r*kt/ks, (r+1)*kt/ks).  Roles (256 threads): warp 0
+// lane 0 streams W tiles and scale atoms through a TMA ring; every warp takes
+// part in the activation quantization; warp 1 lane 0 then issues the scale
+// copies and MMAs; warps 0-3 drain the accumulators and push their partial rows
+// into the owning CTA's shared memory (row r of the tile belongs to rank
+// floor(r*ks/128)); one cluster barrier later each owner sums its rows and
+// writes Y.
+//
+// The kernel is a programmatic dependent of the preceding kernel: before
+// griddepcontrol.wait it only sets up and asks L2 to prefetch its W tiles
+// (L2 is coherent, so a prefetch never yields stale data); every load that
+// feeds the result is issued after the wait.
+//
+// Safety: every mbarrier wait is bounded; every CTA reaches every cluster
+// barrier on every path (the barrier sequence depends only on kernel
+// arguments, which are uniform over the cluster); the shared-memory request
+// covers the whole layout and the CTAs per SM are capped so that their TMEM
+// allocations always fit side by side.
+#include "kernels.h"
+#include "quant_common.cuh"
+#include "tcgen05.cuh"
+
+namespace nvfp4 {
+using namespace tc;
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int NP = 16;                       // activation rows, padded: the MMA N
+constexpr int W_TILE = 128 * 128;            // 128 W rows x 256 K-elements
+constexpr int SFW_BYTES = 4 * 512;           // one scale atom per K=64 chunk
+constexpr int WSTAGE = W_TILE + SFW_BYTES;   // 18 KB, keeps 1024-byte alignment
+constexpr int STAGES = 2;
+constexpr int X_TILE = NP * 128;             // activation codes of one k-tile (SW128)
+constexpr int SF_TILE = 4 * 512;             // activation scale atoms of one k-tile
+constexpr int BAR_BYTES = 256;
+constexpr int PITCH = NP + 4;                // floats per partial row
+constexpr int MAX_KS = 16;
+
+// Partial-row slots an owner holds: one slot of ceil(128/ks) rows per source
+// rank, maximised over every cluster size the launcher may pick.
+constexpr int max_part_rows() {
+  int m = 0;
+  for (int k = 1; k <= MAX_KS; ++k) m = (k * ((128 + k - 1) / k) > m) ? k * ((128 + k - 1) / k) : m;
+  return m;
+}
+constexpr int PART_ROWS = max_part_rows();   // 140 (ks = 14)
+// TMEM columns: acc [0,16), acc_r [16,32), W scales [32,48), X scales [48,64), R scales [64,80)
+constexpr uint32_t ACC = 0, ACC_R = 16, SFW_COL = 32, SFX_COL = 48, SFR_COL = 64, TMEM_COLS = 128;
+static_assert(SFW_COL % 4 == 0 && SFX_COL % 4 == 0 && SFR_COL % 4 == 0,
+              "block-scaled MMA scale operands start on 4-column TMEM boundaries");
+constexpr int TMEM_CTAS = 512 / TMEM_COLS;
+
+static_assert(WSTAGE % 1024 == 0 && X_TILE % 1024 == 0, "SW128 tiles need 1024-byte alignment");
+static_assert(PART_ROWS == 140, "slot count for ks <= 16");
+static_assert(2 * PART_ROWS * PITCH * 4 <= STAGES * WSTAGE, "partials overlay the W ring");
+static_assert((2 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier block");
+
+struct DecodeParams {
+  const void* x;        // fused: activations, M x K (ldx), bf16 or fp32
+  int64_t ldx;
+  const float* s_in;    // fused: given tensor scales or null (computed)
+  const float* sr_in;
+  QOut q, r;            // fused: Q(X), Q(R) written by the first row tile's cluster
+  const uint8_t* sfx;   // plain: X / R scales (ROWMAJOR or TILED) and tensor scales
+  const uint8_t* sfr;
+  int x_tiled;
+  const float* x_s;
+  const float* r_s;
+  const uint8_t* sfw;   // W scales, TILED
+  const float* w_s;
+  void* y;
+  int64_t ldy;
+  int M, N, K;
+  int katoms_w;         // scale atoms per 128-row group of W = K / 64
+  int k_tiles;          // ceil(K / 256)
+  int kt_max;           // k-tiles per CTA held in the activation area
+  int* st;
+};
+
+__host__ __device__ constexpr int smem_bytes(int kt_max, bool res) {
+  return 1024 + STAGES * WSTAGE + kt_max * (X_TILE + SF_TILE) * (res ? 2 : 1) + BAR_BYTES;
+}
+
+template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_decode_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                const __grid_constant__ CUtensorMap tmR, const DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int KT = p.kt_max;
+  uint8_t* xcodes = smem + STAGES * WSTAGE;                         // KT x 2 KB
+  uint8_t* rcodes = xcodes + KT * X_TILE;                           // KT x 2 KB (residue)
+  uint8_t* sfxp = rcodes + (RES ? KT * X_TILE : 0);                 // KT x 2 KB scale atoms
+  uint8_t* sfrp = sfxp + KT * SF_TILE;                              // KT x 2 KB (residue)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sfrp + (RES ? KT * SF_TILE : 0));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* x_full = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* part = reinterpret_cast<float*>(smem);                     // overlays the W ring afterwards
+  __shared__ uint32_t red[kWarps];
+  __shared__ uint32_t xch[2];                                       // published |x|, |r| maxima
+
+  griddep_launch_dependents();   // the next kernel may set itself up; it waits for this one's results
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank(), ks = cluster_nctarank();
+  const int rt = blockIdx.y;                                        // 128-row tile of W
+  const int kt0 = (int)((rank * (uint32_t)p.k_tiles) / ks);
+  const int kt1 = (int)(((rank + 1) * (uint32_t)p.k_tiles) / ks);
+  const int nkt = kt1 - kt0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(saddr(&full[s]), 1);
+      mbar_init(saddr(&empty[s]), 1);
+    }
+    mbar_init(saddr(acc_full), 1);
+    mbar_init(saddr(x_full), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto w_chunks = [&](int kt) { return min(4, (p.K - kt * 256) / 64); };   // K = 64 chunks in k-tile kt
+  auto load_w = [&](int kt, int s) {
+    const uint32_t sf = (uint32_t)w_chunks(kt) * 512u;
+    uint8_t* sb = smem + s * WSTAGE;
+    const uint32_t bar = saddr(&full[s]);
+    mbar_expect_tx(bar, (uint32_t)W_TILE + sf);
+    tma_load_2d(saddr(sb), &tmW, kt * 128, rt * 128, bar);
+    bulk_load(saddr(sb + W_TILE), p.sfw + ((size_t)rt * p.katoms_w + kt * 4) * 512, sf, bar);
+  };
+
+  if (warp == 0 && lane == 0) {
+    // warm L2 with this CTA's W tiles and scale atoms while the preceding kernel finishes
+    for (int kt = kt0; kt < kt1; ++kt) {
+      prefetch_l2_tile_2d(&tmW, kt * 128, rt * 128);
+      prefetch_l2_bulk(p.sfw + ((size_t)rt * p.katoms_w + kt * 4) * 512, (uint32_t)w_chunks(kt) * 512u);
+    }
+  }
+  griddep_wait();   // everything below may read the preceding kernel's results
+
+  const int pre = min(nkt, STAGES);
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < pre; ++i) load_w(kt0 + i, i);   // the ring starts empty
+    if (!FUSED) {
+      mbar_expect_tx(saddr(x_full), (uint32_t)(nkt * X_TILE * (RES ? 2 : 1)));
+      for (int t = 0; t < nkt; ++t) {
+        tma_load_2d(saddr(xcodes + t * X_TILE), &tmX, (kt0 + t) * 128, 0, saddr(x_full));
+        if (RES) tma_load_2d(saddr(rcodes + t * X_TILE), &tmR, (kt0 + t) * 128, 0, saddr(x_full));
+      }
+    }
+  }
+
+  float sx = 0.0f, sr = 0.0f;   // activation / residue tensor scales for the epilogue
+  if constexpr (!FUSED) {
+    sx = *p.x_s;
+    if (RES) sr = *p.r_s;
+    // ---- gather the activation scales into atoms: line n of atom j of k-tile t
+    // starts with the 4 block scales of row n in K chunk 4(kt0+t)+j
+    const int nblk = p.K >> 4;
+    for (int idx = threadIdx.x; idx < nkt * NP * 4 * (RES ? 2 : 1); idx += kThreads) {
+      const int which = idx / (nkt * NP * 4);
+      const int e = idx - which * (nkt * NP * 4);
+      const int t = e / (NP * 4), n = (e >> 2) & (NP - 1), j = e & 3;
+      const int chunk = 4 * (kt0 + t) + j;
+      const uint8_t* src = which ? p.sfr : p.sfx;
+      uint32_t word = 0u;
+      if (chunk * 4 < nblk) {
+        if (p.x_tiled)
+          word = *reinterpret_cast<const uint32_t*>(src + (size_t)chunk * 512 + n * 16);
+        else if (n < p.M)
+          word = *reinterpret_cast<const uint32_t*>(src + (size_t)n * nblk + chunk * 4);
+      }
+      *reinterpret_cast<uint32_t*>((which ? sfrp : sfxp) + t * SF_TILE + j * 512 + n * 16) = word;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  } else {
+    // ---- quantize this CTA's K-slice of X into the operand layout
+    const T* x = static_cast<const T*>(p.x);
+    const int c0 = kt0 * 256;
+    const int upr = (min(kt1 * 256, p.K) - c0) >> 3;   // 8-element units per row (a multiple of 8)
+    const int U = p.M * upr;
+    if (U > R * kThreads) report_status(p.st, NVFP4_ERR_UNSUPPORTED);   // the host split rules this out
+    const bool reporter = rank == 0 && threadIdx.x == 0;
+    const bool writer = blockIdx.y == 0;                // this cluster also writes Q(X), Q(R)
+    Raw8<T> raw[R];
+    uint32_t key = 0u;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int u = i * kThreads + (int)threadIdx.x;
+      if (u < U) {
+        const int row = u / upr, c8 = u - row * upr;
+        raw[i].load(x + (int64_t)row * p.ldx + c0 + c8 * 8);
+      } else {
+        raw[i].zero();
+      }
+      float v[8];
+      raw[i].get(v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
+    }
+    if (key >= 0x7F800000u) report_status(p.st, NVFP4_ERR_NONFINITE);
+    float s;
+    if (p.s_in != nullptr) {
+      s = *p.s_in;
+    } else {
+      s = scale_from_key(cluster_max_u32(key, red, &xch[0]), reporter, p.st);
+    }
+    float s_r = (RES && p.sr_in != nullptr) ? *p.sr_in : 0.0f;
+    if (writer && reporter) {
+      if (p.q.s != p.s_in) *p.q.s = s;
+      if (RES && p.sr_in != nullptr && p.r.s != p.sr_in) *p.r.s = s_r;
+    }
+
+    // place one encoded unit: codes into the SW128 tile, the block scale into the packed scales
+    auto place = [&](uint8_t* codes_area, uint8_t* sf_area, const QOut& qo, int u, uint32_t codes, uint32_t db) {
+      const int row = u / upr, c8 = u - row * upr;
+      const int t = c8 >> 5, kk = (c8 & 31) * 8;         // k-tile within the slice, column within it
+      const int chunk16 = kk >> 5;                         // 16-byte chunk of the 128-byte row
+      *reinterpret_cast<uint32_t*>(codes_area + t * X_TILE + row * 128 + ((chunk16 ^ (row & 7)) << 4) +
+                                   ((kk & 31) >> 1)) = codes;
+      const int bt = kk >> 4;                              // 16-block within the k-tile
+      if ((c8 & 1) == 0) sf_area[t * SF_TILE + (bt >> 2) * 512 + row * 16 + (bt & 3)] = (uint8_t)db;
+      if (writer) store_half_block(qo, row, (c0 >> 3) + c8, codes, db);
+    };
+
+    uint32_t rkey = 0u;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int u = i * kThreads + (int)threadIdx.x;
+      const bool act = u < U;
+      float v[8], deq[8];
+      raw[i].get(v);
+      uint32_t db;
+      const uint32_t codes = quant_half_block(v, s, db, RES ? deq : nullptr);
+      if (act) place(xcodes, sfxp, p.q, u, codes, db);
+      if (RES) {
+        float rv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rv[j] = __fsub_rn(v[j], deq[j]);
+        if (p.sr_in != nullptr) {
+          uint32_t dr;
+          const uint32_t rc = quant_half_block(rv, s_r, dr, nullptr);
+          if (act) place(rcodes, sfrp, p.r, u, rc, dr);
+        } else if (act) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) rkey = max(rkey, abs_key(rv[j]));
+        }
+      }
+    }
+    if (RES && p.sr_in == nullptr) {
+      s_r = scale_from_key(cluster_max_u32(rkey, red, &xch[1]), reporter, p.st);
+      if (writer && reporter) *p.r.s = s_r;
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int u = i * kThreads + (int)threadIdx.x;
+        float v[8], deq[8], rv[8];
+        raw[i].get(v);
+        uint32_t db, dr;
+        (void)quant_half_block(v, s, db, deq);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rv[j] = __fsub_rn(v[j], deq[j]);
+        const uint32_t rc = quant_half_block(rv, s_r, dr, nullptr);
+        if (u < U) place(rcodes, sfrp, p.r, u, rc, dr);
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic writes -> tensor core reads
+    sx = s;
+    sr = s_r;
+  }
+  __syncthreads();   // activation operand (fused) / packed scales (plain) complete
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------- W producer (rest of the ring)
+    int s = pre % STAGES;
+    uint32_t ph = (pre == STAGES) ? 1u : 0u;
+    for (int kt = kt0 + pre; kt < kt1; ++kt) {
+      if (!mbar_wait(saddr(&empty[s]), ph ^ 1u, abort_flag, p.st)) break;
+      load_w(kt, s);
+      if (++s == STAGES) { s = 0; ph ^= 1u; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // --------------------------------------------------------- MMA issuer
+    bool ok = true;
+    if (!FUSED) ok = mbar_wait(saddr(x_full), 0u, abort_flag, p.st);
+    const uint32_t idesc = idesc_nvf4(NP);
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kt = kt0; ok && kt < kt1; ++kt) {
+      if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) break;
+      tc_fence_after();
+      const int t = kt - kt0, jmax = w_chunks(kt);
+      const uint8_t* sb = smem + s * WSTAGE;
+      for (int j = 0; j < jmax; ++j) {
+        tc_cp_scales(tmem + SFW_COL + 4 * j, desc_sf_atom(saddr(sb + W_TILE + j * 512)));
+        tc_cp_scales(tmem + SFX_COL + 4 * j, desc_sf_atom(saddr(sfxp + t * SF_TILE + j * 512)));
+        if (RES) tc_cp_scales(tmem + SFR_COL + 4 * j, desc_sf_atom(saddr(sfrp + t * SF_TILE + j * 512)));
+      }
+      const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(xcodes + t * X_TILE));
+      const uint64_t dr = desc_sw128(saddr(rcodes + t * X_TILE));
+      for (int j = 0; j < jmax; ++j) {
+        const uint32_t acc = (kt > kt0 || j > 0) ? 1u : 0u;
+        tc_mma_nvf4(tmem + ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + SFW_COL + 4 * j,
+                    tmem + SFX_COL + 4 * j, acc);
+        if (RES)
+          tc_mma_nvf4(tmem + ACC_R, dw + (uint64_t)(2 * j), dr + (uint64_t)(2 * j), idesc, tmem + SFW_COL + 4 * j,
+                      tmem + SFR_COL + 4 * j, acc);
+      }
+      tc_commit(saddr(&empty[s]));
+      if (++s == STAGES) { s = 0; ph ^= 1u; }
+    }
+    tc_commit(saddr(acc_full));
+  }
+  __syncwarp();
+
+  // ------------------- push this CTA's partial rows to the CTA that owns them
+  const bool ok = mbar_wait(saddr(acc_full), 0u, abort_flag, p.st);
+  tc_fence_after();
+  __syncwarp();     // the cluster barriers below are warp-aligned
+  // the partials overlay the W ring: a peer's ring is free once its MMAs are done
+  tc_fence_before();
+  cluster_arrive();
+  cluster_wait();
+  tc_fence_after();
+  const int rows_max = (int)((128u + ks - 1) / ks);
+  auto owner_row0 = [&](uint32_t o) { return (int)((o * 128u + ks - 1) / ks); };
+  if (warp < 4) {
+    const int row = warp * 32 + lane;                              // TMEM lane = W row of the tile
+    const uint32_t o = (uint32_t)row * ks / 128u;
+    const int slot = (int)rank * rows_max + (row - owner_row0(o));
+    const uint32_t dst = mapa_shared(saddr(part + slot * PITCH), o);
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll
+    for (int acc_i = 0; acc_i < (RES ? 2 : 1); ++acc_i) {
+      uint32_t v[16];
+      tmem_ld16(lane_addr + (acc_i ? ACC_R : ACC), v);
+      tmem_ld_wait();
+      if (!ok) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0u;
+      }
+      const uint32_t dsti = dst + (uint32_t)(acc_i * PART_ROWS * PITCH * 4);
+#pragma unroll
+      for (int i = 0; i < 16; i += 4)
+        st_cluster_f32x4(dsti + (uint32_t)(i * 4), __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                         __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+    }
+  }
+  tc_fence_before();
+  cluster_sync();   // every partial has landed in its owner's shared memory
+
+  // ------------------------------------------------ owners sum their rows and store
+  {
+    const int r0 = owner_row0(rank), r1 = owner_row0(rank + 1);
+    const int nrows = r1 - r0;
+    const float ws = *p.w_s;
+    const float alpha = sx * ws, alpha_r = RES ? sr * ws : 0.0f;
+    for (int idx = threadIdx.x; idx < nrows * p.M; idx += kThreads) {
+      const int m = idx / nrows, i = idx - m * nrows;
+      const int n = rt * 128 + r0 + i;
+      if (n >= p.N) continue;
+      float sum = 0.0f, sum_r = 0.0f;
+      for (uint32_t src = 0; src < ks; ++src) {
+        const int slot = (int)src * rows_max + i;
+        sum += part[slot * PITCH + m];
+        if (RES) sum_r += part[PART_ROWS * PITCH + slot * PITCH + m];
+      }
+      const float out = RES ? fmaf(sum, alpha, sum_r * alpha_r) : sum * alpha;
+      if (BF16OUT)
+        reinterpret_cast<__nv_bfloat16*>(p.y)[(int64_t)m * p.ldy + n] = __float2bfloat16_rn(out);
+      else
+        reinterpret_cast<float*>(p.y)[(int64_t)m * p.ldy + n] = out;
+    }
+  }
+
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+
+// ------------------------------------------------------------------ host side
+
+constexpr int kMaxUnitsPerThread = 8;   // fused mode: activation units held in registers
+
+struct Choice {
+  int ks = 0, kt_max = 0, smem = 0;
+};
+
+// Cluster split of K.  Cost model per wave of resident CTAs: a CTA issues its
+// own scale copies and MMAs (~0.6 us per k-tile), an SM shares HBM bandwidth
+// among its CTAs (~0.4 us per k-tile each); extra waves repeat the cost.  The
+// larger split wins among equal costs.
+Choice choose_split(int row_tiles, int k_tiles, bool res, int num_sms, int regs_per_thread, int M, int K,
+                    int units_per_thread_cap) {
+  Choice best;
+  double best_cost = 1e30;
+  for (int ks = 1; ks <= std::min(MAX_KS, k_tiles); ++ks) {
+    const int kt_max = (k_tiles + ks - 1) / ks;
+    const int smem = smem_bytes(kt_max, res);
+    if (smem > 232448) continue;
+    if (units_per_thread_cap > 0) {   // fused: every activation unit of the slice fits in registers
+      const int slice = std::min(kt_max * 256, K);
+      if ((int64_t)M * (slice / 8) > (int64_t)units_per_thread_cap * kThreads) continue;
+    }
+    int per_sm = std::min(233472 / (smem + 1024), TMEM_CTAS);
+    per_sm = std::min(per_sm, 2048 / kThreads);
+    if (regs_per_thread > 0) per_sm = std::min(per_sm, 65536 / (regs_per_thread * kThreads));
+    if (per_sm < 1) continue;
+    const int64_t ctas = (int64_t)row_tiles * ks;
+    const int64_t slots = (int64_t)per_sm * num_sms;
+    const int64_t waves = (ctas + slots - 1) / slots;
+    const double per_sm_ctas = (double)((std::min(ctas, slots) + num_sms - 1) / num_sms);
+    const double cost = (double)waves * std::max(0.6 * kt_max, 0.4 * per_sm_ctas * kt_max) + 0.01 * ks;
+    if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && ks > best.ks)) {
+      best_cost = cost;
+      best = Choice{ks, kt_max, smem};
+    }
+  }
+  return best;
+}
+
+template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
+cudaError_t launch_cfg(const DecodeArgs& a, DecodeParams p, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                       const CUtensorMap& tmR, int num_sms, cudaStream_t stream) {
+  auto kern = k_decode_tc<T, FUSED, RES, BF16OUT, R>;
+  static int regs = -1;   // per instantiation
+  if (regs < 0) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
+    regs = fa.numRegs;
+  }
+  const int row_tiles = (int)((a.N + 127) / 128);
+  const Choice c = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs, (int)a.M, (int)a.K, FUSED ? R : 0);
+  if (c.ks == 0) return cudaErrorNotSupported;
+  p.kt_max = c.kt_max;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem);
+  if (e != cudaSuccess) return e;
+  if (c.ks > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)c.ks, (unsigned)row_tiles, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)c.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)c.ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the preceding kernel's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, tmR, p);
+}
+
+template <typename T, bool FUSED, bool RES, bool BF16OUT>
+cudaError_t launch_r(const DecodeArgs& a, const DecodeParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                     const CUtensorMap& tmR, int num_sms, cudaStream_t stream) {
+  if constexpr (!FUSED) {
+    return launch_cfg<T, FUSED, RES, BF16OUT, 0>(a, p, tmW, tmX, tmR, num_sms, stream);
+  } else {
+    // units per thread for the split the launcher will pick is not known yet:
+    // size the register array for the worst split this shape allows
+    const int row_tiles = (int)((a.N + 127) / 128);
+    const Choice c = choose_split(row_tiles, p.k_tiles, RES, num_sms, 0, (int)a.M, (int)a.K, kMaxUnitsPerThread);
+    if (c.ks == 0) return cudaErrorNotSupported;
+    const int64_t units = a.M * (std::min<int64_t>((int64_t)c.kt_max * 256, a.K) / 8);
+    const int upt = (int)((units + kThreads - 1) / kThreads);
+    if (upt <= 1) return launch_cfg<T, FUSED, RES, BF16OUT, 1>(a, p, tmW, tmX, tmR, num_sms, stream);
+    if (upt <= 2) return launch_cfg<T, FUSED, RES, BF16OUT, 2>(a, p, tmW, tmX, tmR, num_sms, stream);
+    if (upt <= 4) return launch_cfg<T, FUSED, RES, BF16OUT, 4>(a, p, tmW, tmX, tmR, num_sms, stream);
+    return launch_cfg<T, FUSED, RES, BF16OUT, 8>(a, p, tmW, tmX, tmR, num_sms, stream);
+  }
+}
+
+template <typename T, bool FUSED>
+cudaError_t launch_t(const DecodeArgs& a, const DecodeParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                     const CUtensorMap& tmR, int num_sms, cudaStream_t stream) {
+  const bool res = a.r_codes != nullptr || a.r_out.codes != nullptr;
+  if (res)
+    return a.y_bf16 ? launch_r<T, FUSED, true, true>(a, p, tmW, tmX, tmR, num_sms, stream)
+                    : launch_r<T, FUSED, true, false>(a, p, tmW, tmX, tmR, num_sms, stream);
+  return a.y_bf16 ? launch_r<T, FUSED, false, true>(a, p, tmW, tmX, tmR, num_sms, stream)
+                  : launch_r<T, FUSED, false, false>(a, p, tmW, tmX, tmR, num_sms, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stream) {
+  if (a.M < 1 || a.M > NP || a.K % 64 != 0 || a.K < 256 || a.N < 1) return cudaErrorNotSupported;
+  const bool fused = a.x != nullptr;
+  CUtensorMap tmW, tmX, tmR;
+  if (!encode_codes_map(&tmW, a.w_codes, a.N, a.K, 128)) return cudaErrorInvalidValue;
+  if (!fused) {
+    if (!encode_codes_map(&tmX, a.x_codes, a.M, a.K, NP)) return cudaErrorInvalidValue;
+    if (a.r_codes != nullptr) {
+      if (!encode_codes_map(&tmR, a.r_codes, a.M, a.K, NP)) return cudaErrorInvalidValue;
+    } else {
+      tmR = tmX;
+    }
+  } else {
+    tmX = tmW;   // unused in fused mode
+    tmR = tmW;
+  }
+  DecodeParams p{};
+  p.x = a.x; p.ldx = a.ldx; p.s_in = a.s_in; p.sr_in = a.sr_in;
+  p.q = a.q_out; p.r = a.r_out;
+  p.sfx = a.x_scales; p.sfr = a.r_scales; p.x_tiled = a.x_tiled ? 1 : 0; p.x_s = a.x_s; p.r_s = a.r_s;
+  p.sfw = a.w_scales; p.w_s = a.w_s;
+  p.y = a.y; p.ldy = a.ldy;
+  p.M = (int)a.M; p.N = (int)a.N; p.K = (int)a.K;
+  p.katoms_w = (int)(a.K / 64);
+  p.k_tiles = (int)((a.K + 255) / 256);
+  p.st = a.st;
+  if (fused)
+    return a.x_bf16 ? launch_t<__nv_bfloat16, true>(a, p, tmW, tmX, tmR, num_sms, stream)
+                    : launch_t<float, true>(a, p, tmW, tmX, tmR, num_sms, stream);
+  return launch_t<uint8_t, false>(a, p, tmW, tmX, tmR, num_sms, stream);
+}
+
+}  // namespace nvfp4

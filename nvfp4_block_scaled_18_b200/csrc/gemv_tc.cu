@@ -303,8 +303,9 @@ cudaError_t launch_np(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   p.k_tiles = (int)((g.K + 255) / 256);
   p.st = g.st;
   const int row_tiles = (int)((g.N + 127) / 128);
-  const int want = std::max(1, (C::CTAS_PER_SM * num_sms + row_tiles / 2) / row_tiles);
-  const int ks = std::max(1, std::min({8, p.k_tiles, want}));
+  // the largest K split whose CTAs are all resident at once (one wave)
+  const int fit = std::max(1, (C::CTAS_PER_SM * num_sms) / row_tiles);
+  const int ks = std::max(1, std::min({8, p.k_tiles, fit}));
   auto kern = k_gemv_tc<NP, RES, BF16OUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;

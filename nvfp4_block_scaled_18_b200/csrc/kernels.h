@@ -55,6 +55,26 @@ struct GemmArgs {
   int* st;
 };
 
+// Decode-sized linear (M <= 16) on the tensor cores.  Fused mode (x != null):
+// X is quantized inside the kernel and Q(X) (and Q(R)) written to q_out
+// (r_out); plain mode: X (and R) are NVFP4 tensors.  W must use TILED scales.
+struct DecodeArgs {
+  // fused mode
+  const void* x; bool x_bf16; int64_t ldx;
+  const float* s_in; const float* sr_in;
+  QOut q_out, r_out;                      // r_out.codes != null selects the residue
+  // plain mode
+  const uint8_t* x_codes; const uint8_t* x_scales; const float* x_s;
+  const uint8_t* r_codes; const uint8_t* r_scales; const float* r_s;
+  bool x_tiled;                           // X / R scale layout
+  // both
+  const uint8_t* w_codes; const uint8_t* w_scales; const float* w_s;
+  void* y; int64_t ldy; bool y_bf16;
+  int64_t M, N, K;
+  int* st;
+};
+cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_gemv(const GemmArgs& g, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);

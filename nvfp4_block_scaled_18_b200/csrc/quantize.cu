@@ -19,41 +19,10 @@
 // 16-element block and exchange their half-block maxima with one shuffle.
 #include "common.cuh"
 #include "kernels.h"
+#include "quant_common.cuh"
 #include "tcgen05.cuh"
 
 namespace nvfp4 {
-
-// Quantize the 8 values this thread owns (half of a 16-block; the partner lane
-// lane^1 owns the other half).  All 32 lanes must call it together.
-// Returns 8 packed E2M1 nibbles; d_byte receives the block's E4M3 scale; when
-// deq != nullptr it receives fl32(fl32(v(c) * d) * s) per element.
-__device__ __forceinline__ uint32_t quant_half_block(const float v[8], float s, uint32_t& d_byte,
-                                                     float* deq) {
-  float a = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
-  a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-  uint32_t db = 0;
-  if (s >= NVFP4_MIN_TENSOR_SCALE) db = f32_to_e4m3(__fdiv_rn(a, __fmul_rn(6.0f, s)));
-  const float d = e4m3_value(db);
-  const float inv = (d != 0.0f) ? __frcp_rn(__fmul_rn(d, s)) : 0.0f;
-  const uint32_t codes =
-      f32x8_to_e2m1(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv),
-                    __fmul_rn(v[3], inv), __fmul_rn(v[4], inv), __fmul_rn(v[5], inv),
-                    __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
-  if (deq != nullptr) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) deq[i] = __fmul_rn(__fmul_rn(e2m1_value(codes >> (4 * i)), d), s);
-  }
-  d_byte = db;
-  return codes;
-}
-
-__device__ __forceinline__ void store_half_block(const QOut& q, int64_t row, int64_t col8,
-                                                 uint32_t codes, uint32_t d_byte) {
-  *reinterpret_cast<uint32_t*>(q.codes + row * (q.cols >> 1) + col8 * 4) = codes;
-  if ((col8 & 1) == 0) q.scales[scale_offset(row, col8 >> 1, q.cols >> 4, q.tiled)] = (uint8_t)d_byte;
-}
 
 // Last-CTA-finishes reduction of a running |.| maximum into a tensor scale.
 // Every thread of every CTA calls it; `key` is the thread's local maximum.
@@ -167,56 +136,6 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
 constexpr int kQC = 8;              // CTAs per cluster (portable cluster size)
 constexpr int kQThreads = 512;      // threads per CTA
 constexpr int kQUnitsPerChunk = kQC * kQThreads;
-
-template <typename T>
-struct Raw8;
-template <>
-struct Raw8<__nv_bfloat16> {
-  uint4 u;
-  __device__ __forceinline__ void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
-  __device__ __forceinline__ void zero() { u = make_uint4(0u, 0u, 0u, 0u); }
-  __device__ __forceinline__ void get(float v[8]) const {
-    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xFFFF0000u);
-    v[4] = __uint_as_float(u.z << 16); v[5] = __uint_as_float(u.z & 0xFFFF0000u);
-    v[6] = __uint_as_float(u.w << 16); v[7] = __uint_as_float(u.w & 0xFFFF0000u);
-  }
-};
-template <>
-struct Raw8<float> {
-  float4 a, b;
-  __device__ __forceinline__ void load(const float* p) {
-    a = __ldg(reinterpret_cast<const float4*>(p));
-    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  }
-  __device__ __forceinline__ void zero() { a = b = make_float4(0.0f, 0.0f, 0.0f, 0.0f); }
-  __device__ __forceinline__ void get(float v[8]) const {
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  }
-};
-
-// Cluster-wide maximum of `key` (every thread of the cluster calls it with the
-// same `slot`, a word this CTA publishes to its peers).  Result in every thread.
-__device__ __forceinline__ uint32_t cluster_max_u32(uint32_t key, uint32_t* red, uint32_t* slot) {
-  const uint32_t m = block_max_u32(key, red);
-  if (threadIdx.x == 0) *slot = m;
-  tc::cluster_sync();  // release/acquire: every CTA's slot is visible cluster-wide
-  const int lane = threadIdx.x & 31;
-  uint32_t a = 0u;
-  if (lane < kQC) a = __float_as_uint(tc::ld_cluster_f32(tc::mapa_shared(tc::saddr(slot), (uint32_t)lane)));
-  return warp_max_u32(a);
-}
-
-// Tensor scale from a |.| maximum key: fl32(amax / 2688), or 0 with
-// NVFP4_ERR_NONFINITE for an Inf/NaN maximum (reported once per cluster).
-__device__ __forceinline__ float scale_from_key(uint32_t a, bool reporter, int* st) {
-  if (a >= 0x7F800000u) {
-    if (reporter) report_status(st, NVFP4_ERR_NONFINITE);
-    return 0.0f;
-  }
-  return __fdiv_rn(__uint_as_float(a), 2688.0f);
-}
 
 // Unit u (8 elements) of this thread's i-th chunk.  Grid: exactly one cluster.
 template <typename T, int R, bool RES>

@@ -72,3 +72,34 @@ def test_validation_before_launch(lib):
     a_tiled = _tensor(4, 64, good, good, good, layout=1)
     assert lib.nvfp4_gemm(ctypes.byref(a_tiled), ctypes.byref(w), good, 0, 32, None, None) == 3
     assert lib.nvfp4_gemm_residue(ctypes.byref(a), None, ctypes.byref(w), good, 0, 32, None, None) == 1
+
+
+def test_fused_decode_validation_before_launch(lib):
+    good = 1 << 20
+    f = lib.nvfp4_quantize_residue_gemm
+    g = lib.nvfp4_quantize_gemm
+
+    def call(M=4, K=512, N=256, dt=1, wl=1, ql=1, x=good, y=good, r=True, ldx=None):
+        q = _tensor(M, K, good, good, good, layout=ql)
+        rr = _tensor(M, K, good, good, good, layout=ql)
+        w = _tensor(N, K, good, good, good, layout=wl)
+        return f(x, dt, M, K, K if ldx is None else ldx, None, None, ctypes.byref(q),
+                 ctypes.byref(rr) if r else None, ctypes.byref(w), y, 0, N, None, None)
+
+    assert call(x=None) == 1                      # null x
+    assert call(y=None) == 1                      # null y
+    assert call(x=good + 4) == 2                  # misaligned x
+    assert call(M=17) == 3                        # decode sizes only
+    assert call(wl=0) == 3                        # W must have TILED scales
+    assert call(K=192) == 3                       # K >= 256
+    assert call(K=320 + 16) == 3                  # K % 64
+    assert call(M=16, K=65536) == 3               # beyond the one-launch quantizer
+    assert call(M=16, K=32768, dt=0) == 3         # fp32: half the units
+    q = _tensor(4, 512, good, good, good, layout=1)
+    r_other = _tensor(4, 512, good, good, good, layout=0)
+    w = _tensor(256, 512, good, good, good, layout=1)
+    assert f(good, 1, 4, 512, 512, None, None, ctypes.byref(q), ctypes.byref(r_other), ctypes.byref(w), good,
+             0, 256, None, None) == 3             # r layout differs from q
+    w_bad = _tensor(256, 256, good, good, good, layout=1)
+    assert g(good, 1, 4, 512, 512, None, ctypes.byref(q), ctypes.byref(w_bad), good, 0, 256, None, None) == 1
+    assert g(good, 1, 4, 512, 512, None, None, ctypes.byref(w), good, 0, 256, None, None) == 1
