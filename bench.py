@@ -7,14 +7,17 @@ Prints ONE JSON line (rank 0).  Default workload ("decode"): the decode GEMV
 configuration -- M in {1,2,4,8,16}, (N,K) in {(4096,4096), (14336,4096),
 (4096,14336)}, bf16 activations N(0,1) with 1% of channels x50 quantized online
 (per-tensor amax, block scales, codes) and multiplied by pre-quantized NVFP4
-weights N(0,0.02).  One step = all 15 (M, shape) linear calls, each
-nvfp4_quantize + nvfp4_gemm.  Weights rotate through 4 copies per shape
-(302 MB) so each call streams its weights from HBM, not L2.
+weights N(0,0.02).  One step = all 15 (M, shape) linear calls, each one
+nvfp4_quantize_gemm (activation quantization and GEMM in one launch; Q(X) is
+written as well).  Every shape has enough weight copies (>= 260 MB) that each
+call streams its weights from HBM, not L2.
 
 value = aggregate algorithmic GB/s of a step (per call N*K*9/16 + M*K*(2+9/16)
 + 4*M*N bytes), device-timed with CUDA events around K graph-replayed steps.
-Multi-GPU: replicas only (the decode path has no data-path exchange); value is
-the bytes all ranks processed over the slowest rank's time.
+Per-call times in "detail" come from graphs of back-to-back calls of one shape
+(the steady state of a chain of layers).  Multi-GPU: replicas only (the decode
+path has no data-path exchange); value is the bytes all ranks processed over
+the slowest rank's time.
 """
 from __future__ import annotations
 
@@ -150,6 +153,11 @@ def sum_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------ decode workload
 
+# DRAM traffic / algorithmic bytes of k_decode_tc from its ncu capture (None once the kernel
+# changes after the capture)
+DECODE_TRAFFIC_RATIO = 33.091328e6 / (4096 * 14336 * 9 / 16 + 1 * 14336 * (2 + 9 / 16) + 4 * 1 * 4096)
+
+
 def decode_bytes(M, N, K):
     """Algorithmic bytes of one online-quantized linear call: W codes+scales, X bf16
     read, X NVFP4 written/read once, Y fp32 written."""
@@ -161,11 +169,11 @@ def gemv_bytes(M, N, K):
 
 
 class DecodeWorkload:
-    """Decode step: 15 (M, shape) online-quantized linear calls.  Operands use
-    TILED block scales, so nvfp4_gemm runs the tensor-core few-row path; a
-    ROWMAJOR twin of every operand (same codes) serves to time the CUDA-core
-    GEMV on the same data."""
-    COPIES = 4
+    """Decode step: 15 (M, shape) linear calls, each nvfp4_quantize_gemm on TILED
+    weights (tensor-core decode kernel, activation quantization fused).  Every
+    shape keeps enough weight copies to exceed L2.  A ROWMAJOR twin of every
+    weight (same codes) serves to time the CUDA-core GEMV on the same data."""
+    L2_SPAN = 260e6
 
     def __init__(self, dev):
         import nvfp4_block_scaled_18_b200 as nv
@@ -174,7 +182,7 @@ class DecodeWorkload:
         self.shapes = list(wl.DECODE_SHAPES)
         self.Ms = list(wl.DECODE_M)
         self.calls = [(M, N, K) for M in self.Ms for (N, K) in self.shapes]
-        self.W, self.Wrm = {}, {}
+        self.W, self.Wrm, self.copies = {}, {}, {}
         for (N, K) in self.shapes:
             w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
             q0 = nv.NVFP4Tensor.empty(N, K, nv.SF_TILED, device=dev)
@@ -182,12 +190,13 @@ class DecodeWorkload:
             r0 = nv.NVFP4Tensor.empty(N, K, nv.SF_ROWMAJOR, device=dev)
             nv.nvfp4_quantize(w, r0, workspace=nv.Workspace(N, K, dev))
             del w
+            n = max(4, int(np.ceil(self.L2_SPAN / (N * K * 9 / 16))))
             tiled, rowm = [q0], [r0]
-            for _ in range(self.COPIES - 1):
+            for _ in range(n - 1):
                 c = q0.codes.clone()
                 tiled.append(nv.NVFP4Tensor(c, q0.scales.clone(), q0.tensor_scale.clone(), N, K, nv.SF_TILED))
                 rowm.append(nv.NVFP4Tensor(c, r0.scales.clone(), r0.tensor_scale.clone(), N, K, nv.SF_ROWMAJOR))
-            self.W[(N, K)], self.Wrm[(N, K)] = tiled, rowm
+            self.W[(N, K)], self.Wrm[(N, K)], self.copies[(N, K)] = tiled, rowm, n
         self.X, self.Xhost, self.QX, self.QXrm, self.WS, self.Y, self.Yhost = {}, {}, {}, {}, {}, {}, {}
         for M in self.Ms:
             for K in sorted({k for _, k in self.shapes}):
@@ -201,19 +210,37 @@ class DecodeWorkload:
                 self.Y[(M, N, K)] = torch.empty((M, N), dtype=torch.float32, device=dev)
                 self.Yhost[(M, N, K)] = torch.empty((M, N), dtype=torch.float32).pin_memory()
         self.step_bytes = sum(decode_bytes(*c) for c in self.calls)
-        self.launches_per_step = 3 * len(self.calls)  # amax + quantize + GEMV per call
+        # 1 launch per call when quantization is fused, 2 where quantize-then-GEMM is chosen
+        self.plan = {c: nv.nvfp4_quantize_gemm_plan(*c) for c in self.calls}
+        assert all(v in (1, 2) for v in self.plan.values()), self.plan
+        self.launches_per_step = sum(self.plan.values())
+        self.phases = max(self.copies.values())
         torch.cuda.synchronize()
 
-    def copy_index(self, step, i):
-        return ((step * len(self.calls) + i) // len(self.shapes)) % self.COPIES
+    def weight(self, N, K, i, rowmajor=False):
+        ws = (self.Wrm if rowmajor else self.W)[(N, K)]
+        return ws[i % len(ws)]
+
+    def call(self, M, N, K, i, mode="fused"):
+        """One linear call with weight copy i: 'fused' (one launch), 'separate'
+        (nvfp4_quantize + nvfp4_gemm) or 'cuda_core' (ROWMAJOR operands)."""
+        nv = self.nv
+        x, y = self.X[(M, K)], self.Y[(M, N, K)]
+        if mode == "fused":
+            nv.nvfp4_quantize_gemm(x, self.QX[(M, K)], self.weight(N, K, i), y)
+        elif mode == "separate":
+            nv.nvfp4_quantize(x, self.QX[(M, K)], workspace=self.WS[(M, K)])
+            nv.nvfp4_gemm(self.QX[(M, K)], self.weight(N, K, i), y)
+        else:
+            nv.nvfp4_quantize(x, self.QXrm[(M, K)], workspace=self.WS[(M, K)])
+            nv.nvfp4_gemm(self.QXrm[(M, K)], self.weight(N, K, i, rowmajor=True), y)
 
     def run_step(self, step, e2e=False):
-        nv = self.nv
-        for i, (M, N, K) in enumerate(self.calls):
+        for (M, N, K) in self.calls:
             if e2e:
                 self.X[(M, K)].copy_(self.Xhost[(M, K)], non_blocking=True)
-            nv.nvfp4_quantize(self.X[(M, K)], self.QX[(M, K)], workspace=self.WS[(M, K)])
-            nv.nvfp4_gemm(self.QX[(M, K)], self.W[(N, K)][self.copy_index(step, i)], self.Y[(M, N, K)])
+            # every call of a step streams its own weight copy
+            self.call(M, N, K, step * len(self.Ms) + self.Ms.index(M))
             if e2e:
                 self.Yhost[(M, N, K)].copy_(self.Y[(M, N, K)], non_blocking=True)
 
@@ -242,6 +269,16 @@ def capture_graphs(wk, phases, e2e=False):
     return graphs
 
 
+class EagerStep:
+    """Stands in for a captured step graph: replay() launches the step directly."""
+
+    def __init__(self, wk, phase, e2e=False):
+        self.wk, self.phase, self.e2e = wk, phase, e2e
+
+    def replay(self):
+        self.wk.run_step(self.phase, self.e2e)
+
+
 def time_graphs(graphs, steps, warmup, world, sampler=None):
     n = len(graphs)
     for i in range(warmup):
@@ -264,24 +301,90 @@ def time_graphs(graphs, steps, warmup, world, sampler=None):
     return start.elapsed_time(end)
 
 
-def time_gemv_launches(wk, rowmajor=False, reps=24):
-    """Per-launch device time (ms) of the decode GEMM for every (M, shape):
-    the tensor-core few-row kernel (TILED operands) or, with rowmajor=True, the
-    CUDA-core GEMV on the same codes.  Weights rotate through the copies."""
-    nv = wk.nv
+def time_back_to_back(fn, n, reps=5):
+    """Per-call device time (ms) of fn(0..n-1) captured back to back in one graph:
+    median over reps replays of (replay time / n)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(n):
+            fn(i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b) / n)
+    del g
+    return statistics.median(times)
+
+
+def time_decode_calls(wk, mode):
+    """Per-call time (ms) of every decode (M, shape) in one mode, back to back
+    over all weight copies of the shape (never L2-resident)."""
     out = {}
     for (M, N, K) in wk.calls:
-        qx = (wk.QXrm if rowmajor else wk.QX)[(M, K)]
-        ws = (wk.Wrm if rowmajor else wk.W)[(N, K)]
-        y = wk.Y[(M, N, K)]
-        nv.nvfp4_quantize(wk.X[(M, K)], qx, workspace=wk.WS[(M, K)])
-        i = [0]
-
-        def call():
-            nv.nvfp4_gemm(qx, ws[i[0] % wk.COPIES], y)
-            i[0] += 1
-        out[(M, N, K)] = time_launches(call, reps=reps)
+        n = wk.copies[(N, K)]
+        out[(M, N, K)] = time_back_to_back(lambda i: wk.call(M, N, K, i, mode), n)
     return out
+
+
+class ResServeDecode:
+    """ResServe decode (M in 1,4,16; (N,K) in (5120,5120),(27648,5120),(5120,27648);
+    Student-t(3) x 0.5 activations): fused plain vs fused residue-compensated
+    linear, to report the latency overhead of the residue at M <= 16."""
+    L2_SPAN = 260e6
+
+    def __init__(self, dev):
+        import nvfp4_block_scaled_18_b200 as nv
+        from nvfp4_block_scaled_18_b200 import workloads as wl
+        self.nv = nv
+        self.Ms = [m for m in wl.RESSERVE_M if m <= 16]
+        self.shapes = list(wl.RESSERVE_SHAPES)
+        self.W, self.buf = {}, {}
+        for (N, K) in self.shapes:
+            w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
+            q0 = nv.NVFP4Tensor.empty(N, K, nv.SF_TILED, device=dev)
+            nv.nvfp4_quantize(w, q0, workspace=nv.Workspace(N, K, dev))
+            del w
+            n = max(2, int(np.ceil(self.L2_SPAN / (N * K * 9 / 16))))
+            self.W[(N, K)] = [q0] + [nv.NVFP4Tensor(q0.codes.clone(), q0.scales.clone(), q0.tensor_scale.clone(),
+                                                    N, K, nv.SF_TILED) for _ in range(n - 1)]
+            for M in self.Ms:
+                self.buf[(M, N, K)] = dict(
+                    x=wl.to_bf16(wl.resserve_x(M, K)).to(dev),
+                    q=nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev),
+                    r=nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev),
+                    y=torch.empty((M, N), dtype=torch.float32, device=dev))
+        torch.cuda.synchronize()
+
+    def measure(self):
+        out = {}
+        for (N, K) in self.shapes:
+            ws = self.W[(N, K)]
+            for M in self.Ms:
+                b = self.buf[(M, N, K)]
+                t0 = time_back_to_back(lambda i: self.nv.nvfp4_quantize_gemm(b["x"], b["q"], ws[i % len(ws)], b["y"]),
+                                       len(ws))
+                t1 = time_back_to_back(lambda i: self.nv.nvfp4_quantize_residue_gemm(b["x"], b["q"], b["r"],
+                                                                                     ws[i % len(ws)], b["y"]),
+                                       len(ws))
+                out[f"M{M}_N{N}_K{K}"] = {"plain_us": round(t0 * 1e3, 3), "residue_us": round(t1 * 1e3, 3),
+                                          "overhead_pct": round((t1 - t0) / t0 * 100.0, 1)}
+        worst = max(v["overhead_pct"] for v in out.values())
+        mean = float(np.mean([v["overhead_pct"] for v in out.values()]))
+        return {"per_call": out, "overhead_pct_max": worst, "overhead_pct_mean": round(mean, 1),
+                "target": "<= 10% extra latency at M <= 16"}
 
 
 # ------------------------------------------------------------ prefill workload
@@ -379,32 +482,14 @@ def prefill_e2e(wk, steps):
     return start.elapsed_time(end)
 
 
-def time_launches(fn, reps=8, rounds=3):
-    """Median device time (ms) of fn() launches: CUDA events around each launch,
-    all queued behind a sleep kernel so host gaps never enter the intervals."""
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-    fn()
-    times = []
-    for _ in range(rounds):
-        torch.cuda.synchronize()
-        torch.cuda._sleep(20_000_000)
-        for r in range(reps):
-            ev[r][0].record()
-            fn()
-            ev[r][1].record()
-        torch.cuda.synchronize()
-        times += [a.elapsed_time(b) for a, b in ev]
-    return statistics.median(times)
-
-
 def measure_prefill_from(wk, peaks):
     """Per-launch GEMM and quantizer times on the prefill workload."""
     out, flops_total, gemm_ms_total = {}, 0.0, 0.0
     for (name, M, N, Keff, S) in wk.calls:
         K = Keff - S
         wk.quantize(N, K, S)
-        g_ms = time_launches(lambda: wk.gemm(N, K, S))
-        q_ms = time_launches(lambda: wk.quantize(N, K, S))
+        g_ms = time_back_to_back(lambda i: wk.gemm(N, K, S), 4)
+        q_ms = time_back_to_back(lambda i: wk.quantize(N, K, S), 4)
         flops = 2.0 * M * N * Keff
         q_bytes = 2 * M * K + M * Keff * 9 // 16
         flops_total += flops
@@ -516,6 +601,51 @@ def reference_arm(args):
     return 0
 
 
+# ------------------------------------------------------------------ profiling cases
+
+def profile_case(case: str) -> int:
+    """A handful of launches of one kernel, inputs just above L2, for ncu:
+    decode   -- nvfp4_quantize_gemm, M=1, (N,K)=(4096,14336), 5 weight copies (147 MB)
+    prefill  -- nvfp4_gemm, M=8192, (N,K)=(14336,4096) (A 19 MB, W 33 MB, Y 470 MB)
+    quantize -- nvfp4_quantize of the 8192x4096 bf16 prefill activations (67 MB)."""
+    import nvfp4_block_scaled_18_b200 as nv
+    from nvfp4_block_scaled_18_b200 import workloads as wl
+    dev = torch.device("cuda", torch.cuda.current_device())
+    nv.load_library()
+    if case == "decode":
+        M, N, K = 1, 4096, 14336
+        w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
+        ws = []
+        for _ in range(5):
+            q = nv.NVFP4Tensor.empty(N, K, nv.SF_TILED, device=dev)
+            nv.nvfp4_quantize(w, q, workspace=nv.Workspace(N, K, dev))
+            ws.append(q)
+        x = wl.to_bf16(wl.decode_x(M, K)).to(dev)
+        qx = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev)
+        y = torch.empty((M, N), device=dev)
+        for i in range(10):
+            nv.nvfp4_quantize_gemm(x, qx, ws[i % 5], y)
+    elif case == "prefill":
+        M, N, K = 8192, 14336, 4096
+        qa = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev)
+        qw = nv.NVFP4Tensor.empty(N, K, nv.SF_TILED, device=dev)
+        nv.nvfp4_quantize(wl.to_bf16(wl.prefill_x(M, K)).to(dev), qa, workspace=nv.Workspace(M, K, dev))
+        nv.nvfp4_quantize(torch.from_numpy(wl.weights_normal(N, K)).to(dev), qw, workspace=nv.Workspace(N, K, dev))
+        y = torch.empty((M, N), device=dev)
+        for _ in range(3):
+            nv.nvfp4_gemm(qa, qw, y)
+    else:
+        M, K = 8192, 4096
+        x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
+        q = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev)
+        ws = nv.Workspace(M, K, dev)
+        for _ in range(3):
+            nv.nvfp4_quantize(x, q, workspace=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": case, "ok": True}), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -527,10 +657,17 @@ def main():
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="decode line without the prefill sub-measurement")
+    ap.add_argument("--eager", action="store_true",
+                    help="decode: launch every step directly on the stream (no CUDA graphs) and skip the "
+                         "per-call detail; for profilers that cannot follow graph replays")
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize"],
+                    help="run a few launches of one kernel on a small case (for ncu captures) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         return reference_arm(args)
+    if args.profile_case:
+        return profile_case(args.profile_case)
 
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -540,7 +677,7 @@ def main():
 
     if args.workload == "decode":
         wk = DecodeWorkload(dev)
-        phases = DecodeWorkload.COPIES
+        phases = wk.phases
         unit, work_per_step = "GB/s", float(wk.step_bytes)
         scale = 1e9
         steps = args.steps
@@ -550,7 +687,8 @@ def main():
         unit, work_per_step = "TFLOP/s", float(sum(2.0 * M * N * Keff for (_, M, N, Keff, _) in wk.calls))
         scale = 1e12
         steps = max(1, min(args.steps, 40))
-    graphs = capture_graphs(wk, phases)
+    eager = args.eager and args.workload == "decode"
+    graphs = [EagerStep(wk, p) for p in range(phases)] if eager else capture_graphs(wk, phases)
     sampler = ClockSampler(torch.cuda.current_device())
     ms = time_graphs(graphs, steps, args.warmup, world, sampler)
     clocks = sampler.stop()
@@ -561,7 +699,7 @@ def main():
     # end to end: pinned host X -> device, quantize + GEMM, Y -> pinned host, every step
     e2e_steps = max(4 * phases, min(steps, 400)) if args.workload == "decode" else max(2, min(steps, 5))
     if args.workload == "decode":
-        e2e_graphs = capture_graphs(wk, phases, e2e=True)
+        e2e_graphs = [EagerStep(wk, p, True) for p in range(phases)] if eager else capture_graphs(wk, phases, e2e=True)
         ms_e2e = max_over_ranks(time_graphs(e2e_graphs, e2e_steps, args.warmup, world), world)
         h2d, d2h = wk.h2d_bytes(), wk.d2h_bytes()
     else:
@@ -572,28 +710,51 @@ def main():
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5)}
-    if args.workload == "decode":
-        per = time_gemv_launches(wk)
-        per_cc = time_gemv_launches(wk, rowmajor=True)
-        g_bytes = sum(gemv_bytes(*c) for c in wk.calls)
-        achieved = g_bytes / (sum(per.values()) * 1e-3) / 1e9
-        achieved_cc = g_bytes / (sum(per_cc.values()) * 1e-3) / 1e9
+    if eager:
+        detail = {"mode": "eager launches, no per-call detail"}
+        roofline = {"bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": None,
+                    "traffic": None, "kernel": "k_decode_tc", "peak_source": peaks["source"]}
+        config = {"workload": "decode GEMV (eager launches)", "calls_per_step": len(wk.calls),
+                  "parallelism": f"replicas x{world}"}
+        launches = wk.launches_per_step * steps
+    elif args.workload == "decode":
+        per = time_decode_calls(wk, "fused")
+        per_sep = time_decode_calls(wk, "separate")
+        per_cc = time_decode_calls(wk, "cuda_core")
+        tot = lambda d: sum(d.values())
+        achieved = wk.step_bytes / (tot(per) * 1e-3) / 1e9
         line["us_per_call"] = round(ms_per_step * 1e3 / len(wk.calls), 3)
+        gbps = lambda c, t: round(decode_bytes(*c) / (t * 1e-3) / 1e9, 1)
         detail = {f"M{M}_N{N}_K{K}": {
-            "tc_us": round(per[(M, N, K)] * 1e3, 3),
-            "tc_GBps": round(gemv_bytes(M, N, K) / (per[(M, N, K)] * 1e-3) / 1e9, 1),
-            "cuda_core_us": round(per_cc[(M, N, K)] * 1e3, 3),
-            "cuda_core_GBps": round(gemv_bytes(M, N, K) / (per_cc[(M, N, K)] * 1e-3) / 1e9, 1)}
+            "fused_us": round(per[(M, N, K)] * 1e3, 3), "fused_GBps": gbps((M, N, K), per[(M, N, K)]),
+            "separate_us": round(per_sep[(M, N, K)] * 1e3, 3),
+            "cuda_core_us": round(per_cc[(M, N, K)] * 1e3, 3), "cuda_core_GBps": gbps((M, N, K), per_cc[(M, N, K)])}
             for (M, N, K) in wk.calls}
-        detail["cuda_core_gemv_aggregate"] = {"achieved_GBps": round(achieved_cc, 1),
-                                              "frac": round(achieved_cc / peaks["hbm_gbs"], 4)}
+        for name, d in (("fused", per), ("separate", per_sep), ("cuda_core", per_cc)):
+            a = wk.step_bytes / (tot(d) * 1e-3) / 1e9
+            detail[f"{name}_aggregate"] = {"us_per_call": round(tot(d) * 1e3 / len(wk.calls), 3),
+                                           "GBps": round(a, 1), "frac_hbm": round(a / peaks["hbm_gbs"], 4)}
+        detail["per_call_timing"] = "graphs of back-to-back calls of one shape over all its weight copies"
+        del graphs
+        rs = ResServeDecode(dev)
+        detail["resserve_residue_overhead"] = rs.measure()
+        del rs
+        # DRAM bytes per launch from the ncu capture of k_decode_tc (M=1, (4096,14336)):
+        # 33.091 MB measured against 33.077 MB algorithmic; scaled to the average call of a step
+        traffic = wk.step_bytes / len(wk.calls) * DECODE_TRAFFIC_RATIO if DECODE_TRAFFIC_RATIO else None
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
-                    "kernel": "k_gemv_tc (tensor-core few-row GEMM, all 15 decode launches)",
+                    "frac": round(achieved / peaks["hbm_gbs"], 4),
+                    "traffic": None if traffic is None else round(traffic),
+                    "traffic_basis": "bytes per average call of a step: algorithmic x (measured/algorithmic) "
+                                     "of the profiled launch (profiles/k_decode_tc_m1_4096x14336.md)",
+                    "kernel": "k_decode_tc (fused quantize + GEMM; plain GEMM after the quantizer on the calls "
+                              "where that is estimated faster), all 15 decode calls back to back",
+                    "launches_per_step": wk.launches_per_step,
                     "peak_source": peaks["source"]}
         config = {"workload": "decode GEMV (M in 1,2,4,8,16; (N,K) in (4096,4096),(14336,4096),(4096,14336)); "
-                              "online bf16->NVFP4 activation quantization + NVFP4 GEMM, fp32 out",
-                  "calls_per_step": len(wk.calls), "l2": "weights rotate through 4 copies per shape (302 MB > L2)",
+                              "online bf16->NVFP4 activation quantization + NVFP4 GEMM in one launch, fp32 out",
+                  "calls_per_step": len(wk.calls),
+                  "l2": "every call streams its own weight copy; >= 260 MB of copies per shape (> L2)",
                   "parallelism": f"replicas x{world}"}
         launches = wk.launches_per_step * steps
     else:
@@ -608,8 +769,8 @@ def main():
                  "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d,
                          "d2h_bytes_per_step": d2h},
                  "gpu_launches": launches, "clocks": clocks, "detail": detail})
-    if args.workload == "decode" and not args.no_prefill:
-        del graphs, e2e_graphs
+    if args.workload == "decode" and not args.no_prefill and not eager:
+        del e2e_graphs
         pw = PrefillWorkload(dev)
         pdetail, proof = measure_prefill_from(pw, peaks)
         line["prefill"] = {"roofline": proof, "detail": pdetail}

@@ -172,6 +172,14 @@ nvfp4_status nvfp4_quantize_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64
                                  const float* scale_in, nvfp4_tensor* q, const nvfp4_tensor* w, void* y,
                                  nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
 
+/* Number of kernel launches nvfp4_quantize_gemm (residue = 0) or
+ * nvfp4_quantize_residue_gemm (residue != 0) makes for these sizes on the
+ * current device: 1 (quantization fused into the GEMM), 2 (quantize, then the
+ * GEMM on the NVFP4 operands, chosen when estimated faster), 0 (unsupported).
+ * It launches nothing and reads no device memory; it may initialise the CUDA
+ * runtime on the current device (kernel attribute queries). */
+int nvfp4_quantize_gemm_plan(int64_t M, int64_t N, int64_t K, nvfp4_dtype dt, int residue, nvfp4_dtype out_dt);
+
 /* ResServe compensated decode linear with online quantization of X and of its
  * residue, in one kernel launch:
  *   (q, r) <- nvfp4_quantize_residue(X, scale_in, rscale_in)

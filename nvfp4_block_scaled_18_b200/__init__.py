@@ -26,6 +26,7 @@ SF_ROWMAJOR, SF_TILED = 0, 1
 EXPORTED_SYMBOLS = ("nvfp4_scales_bytes", "nvfp4_workspace_size", "nvfp4_quantize",
                     "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize", "nvfp4_gemm",
                     "nvfp4_gemm_residue", "nvfp4_quantize_gemm", "nvfp4_quantize_residue_gemm",
+                    "nvfp4_quantize_gemm_plan",
                     "nvfp4_rmsnorm_reorder_quantize_noalloc",
                     "nvfp4_status_string", "nvfp4_version")
 NVFP4_NOALLOC_MAX_ROWS = 65536
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.nvfp4_gemm.argtypes = [T, T, P, ctypes.c_int, I64, P, P]
         lib.nvfp4_gemm_residue.argtypes = [T, T, T, P, ctypes.c_int, I64, P, P]
         lib.nvfp4_quantize_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, P, T, T, P, ctypes.c_int, I64, P, P]
+        lib.nvfp4_quantize_gemm_plan.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.nvfp4_quantize_gemm_plan.restype = ctypes.c_int
         lib.nvfp4_quantize_residue_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, T, T, T, P,
                                                     ctypes.c_int, I64, P, P]
         for fn in ("nvfp4_quantize", "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize",
@@ -286,3 +289,12 @@ def nvfp4_quantize_residue_gemm(x: torch.Tensor, q: NVFP4Tensor, r: Optional[NVF
                                            y.data_ptr(), _out_dtype(y), _ldx(y), _ptr(dev_status),
                                            _stream(stream)),
            "nvfp4_quantize_residue_gemm")
+
+
+def nvfp4_quantize_gemm_plan(M: int, N: int, K: int, x_dtype=torch.bfloat16, residue: bool = False,
+                             out_dtype=torch.float32) -> int:
+    """Kernel launches one nvfp4_quantize[_residue]_gemm call makes for these sizes
+    (1 fused, 2 quantize-then-GEMM, 0 unsupported).  Host-only."""
+    lib = load_library()
+    code = lambda d: NVFP4_BF16 if d == torch.bfloat16 else NVFP4_F32
+    return lib.nvfp4_quantize_gemm_plan(M, N, K, code(x_dtype), 1 if residue else 0, code(out_dtype))

@@ -248,6 +248,27 @@ nvfp4_status nvfp4_quantize_residue_gemm(const void* x, nvfp4_dtype dt, int64_t 
   return run_gemm(q, r, w, y, out_dt, ldy, dev_status, stream);
 }
 
+int nvfp4_quantize_gemm_plan(int64_t M, int64_t N, int64_t K, nvfp4_dtype dt, int residue, nvfp4_dtype out_dt) {
+  if (M < 1 || M > 16 || N < 1 || K < 256 || K % 64 != 0 || !dt_ok(dt) || !dt_ok(out_dt)) return 0;
+  if (M * (K / 8) > quant_small_max_units(dt)) return 0;
+  static const uint8_t dummy[16] = {0};
+  DecodeArgs d{};
+  d.x = dummy; d.x_bf16 = dt == NVFP4_BF16; d.ldx = K;
+  d.q_out = QOut{const_cast<uint8_t*>(dummy), const_cast<uint8_t*>(dummy), nullptr, K, true};
+  if (residue) d.r_out = d.q_out;
+  d.w_codes = dummy; d.w_scales = dummy;
+  d.y_bf16 = out_dt == NVFP4_BF16;
+  d.M = M; d.N = N; d.K = K; d.dry_run = true;
+  const cudaError_t e = launch_decode_tc(d, num_sms_current_device(), nullptr);
+  if (e == cudaSuccess) return 1;
+  if (e != cudaErrorNotSupported) return 0;
+  d.x = nullptr;                       // quantize, then the decode kernel on NVFP4 operands
+  d.x_codes = dummy; d.x_scales = dummy; d.x_tiled = true;
+  if (residue) { d.r_codes = dummy; d.r_scales = dummy; }
+  d.r_out = QOut{};
+  return launch_decode_tc(d, num_sms_current_device(), nullptr) == cudaSuccess ? 2 : 0;
+}
+
 nvfp4_status nvfp4_quantize_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                  const float* scale_in, nvfp4_tensor* q, const nvfp4_tensor* w, void* y,
                                  nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream) {

@@ -3,9 +3,11 @@
 //
 // Y^T = W X^T with W (N x K, NVFP4, TILED scales) as the 128-row A operand of
 // tcgen05.mma.kind::mxf4nvf4.block_scale.block16 and the activation rows
-// (padded to N = 16) as the B operand.  With a residue R (ResServe abstract:
-// FP4 base plus FP4 residue, combined on-chip) the same W tile feeds a second
-// accumulator: Y = s_x s_w acc + s_r s_w acc_r.
+// (padded to 16) as the B operand.  With a residue R (ResServe abstract: FP4
+// base plus FP4 residue, combined on-chip) X and R are stacked into one
+// 32-row B operand (rows 0-15 X, 16-31 R): each MMA then produces both
+// products side by side in one accumulator, for the same instruction count as
+// the plain case, and Y = s_x s_w acc[:, 0:16] + s_r s_w acc[:, 16:32].
 //
 // Fused mode (nvfp4_quantize_gemm): the kernel reads X in bf16/fp32 and
 // quantizes it itself.  The ks CTAs of a cluster split K; together they cover
@@ -24,14 +26,18 @@
 // block-scaled MMA must start on a 4-column TMEM boundary, so one copy cannot
 // serve several MMAs.
 //
-// Grid: (ks, ceil(N/128)), cluster (ks, 1, 1), ks <= 16.  CTA rank r of a
-// cluster handles k-tiles [r*kt/ks, (r+1)*kt/ks).  Roles (256 threads): warp 0
-// lane 0 streams W tiles and scale atoms through a TMA ring; every warp takes
-// part in the activation quantization; warp 1 lane 0 then issues the scale
+// Grid: (ks, ceil(N/128)), cluster (ks, 1, 1), ks <= 8.  CTA rank r of a
+// cluster handles k-tiles [r*kt/ks, (r+1)*kt/ks).  Roles (256 threads): every
+// warp takes part in the activation quantization; warp 0 lane 0 streams W
+// tiles and scale atoms through a TMA ring; warp 1 lane 0 issues the scale
 // copies and MMAs; warps 0-3 drain the accumulators and push their partial rows
-// into the owning CTA's shared memory (row r of the tile belongs to rank
-// floor(r*ks/128)); one cluster barrier later each owner sums its rows and
-// writes Y.
+// into a dedicated area of the owning CTA's shared memory (row r of the tile
+// belongs to rank floor(r*ks/128)); one cluster barrier later each owner sums
+// its rows and writes Y.  Per-CTA maxima travel the same way: each CTA writes
+// its maximum into every peer, so one barrier later every CTA reads all of them
+// locally.  Every CTA announces at start-up that it is running (a relaxed
+// cluster arrive) and waits for its peers' announcements before its first
+// store into another CTA's shared memory.
 //
 // The kernel is a programmatic dependent of the preceding kernel: before
 // griddepcontrol.wait it only sets up and asks L2 to prefetch its W tiles
@@ -43,6 +49,8 @@
 // arguments, which are uniform over the cluster); the shared-memory request
 // covers the whole layout and the CTAs per SM are capped so that their TMEM
 // allocations always fit side by side.
+#include <cstring>
+
 #include "kernels.h"
 #include "quant_common.cuh"
 #include "tcgen05.cuh"
@@ -53,16 +61,17 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int NP = 16;                       // activation rows, padded: the MMA N
+constexpr int NP = 16;                       // activation rows, padded
 constexpr int W_TILE = 128 * 128;            // 128 W rows x 256 K-elements
 constexpr int SFW_BYTES = 4 * 512;           // one scale atom per K=64 chunk
 constexpr int WSTAGE = W_TILE + SFW_BYTES;   // 18 KB, keeps 1024-byte alignment
 constexpr int STAGES = 2;
-constexpr int X_TILE = NP * 128;             // activation codes of one k-tile (SW128)
-constexpr int SF_TILE = 4 * 512;             // activation scale atoms of one k-tile
+constexpr int X_TILE = NP * 128;             // codes of one operand (X or R) in one k-tile (SW128)
+constexpr int SF_TILE = 4 * 512;             // scale atoms of one k-tile (lines 0-15 X, 16-31 R)
+__host__ __device__ constexpr int b_tile(bool res) { return X_TILE * (res ? 2 : 1); }   // MMA B tile
 constexpr int BAR_BYTES = 256;
-constexpr int PITCH = NP + 4;                // floats per partial row
-constexpr int MAX_KS = 16;
+constexpr int PITCH = NP;                    // floats per partial row (16-byte aligned rows)
+constexpr int MAX_KS = 8;   // portable cluster size: larger clusters wait for free slots inside one GPC
 
 // Partial-row slots an owner holds: one slot of ceil(128/ks) rows per source
 // rank, maximised over every cluster size the launcher may pick.
@@ -71,16 +80,16 @@ constexpr int max_part_rows() {
   for (int k = 1; k <= MAX_KS; ++k) m = (k * ((128 + k - 1) / k) > m) ? k * ((128 + k - 1) / k) : m;
   return m;
 }
-constexpr int PART_ROWS = max_part_rows();   // 140 (ks = 14)
-// TMEM columns: acc [0,16), acc_r [16,32), W scales [32,48), X scales [48,64), R scales [64,80)
-constexpr uint32_t ACC = 0, ACC_R = 16, SFW_COL = 32, SFX_COL = 48, SFR_COL = 64, TMEM_COLS = 128;
-static_assert(SFW_COL % 4 == 0 && SFX_COL % 4 == 0 && SFR_COL % 4 == 0,
-              "block-scaled MMA scale operands start on 4-column TMEM boundaries");
+constexpr int PART_ROWS = max_part_rows();   // 133 (ks = 7)
+// TMEM columns: acc [0,32) (X products in 0-15, R products in 16-31), W scales
+// [32,48), X/R scales [48,64)
+constexpr uint32_t ACC = 0, ACC_R = 16, SFW_COL = 32, SFX_COL = 48, TMEM_COLS = 64;
+static_assert(SFW_COL % 4 == 0 && SFX_COL % 4 == 0, "block-scaled MMA scale operands start on 4-column TMEM boundaries");
 constexpr int TMEM_CTAS = 512 / TMEM_COLS;
 
 static_assert(WSTAGE % 1024 == 0 && X_TILE % 1024 == 0, "SW128 tiles need 1024-byte alignment");
-static_assert(PART_ROWS == 140, "slot count for ks <= 16");
-static_assert(2 * PART_ROWS * PITCH * 4 <= STAGES * WSTAGE, "partials overlay the W ring");
+static_assert(PART_ROWS == 133, "slot count for ks <= 8");
+__host__ __device__ constexpr int part_bytes(bool res) { return PART_ROWS * PITCH * 4 * (res ? 2 : 1); }
 static_assert((2 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier block");
 
 struct DecodeParams {
@@ -105,8 +114,12 @@ struct DecodeParams {
   int* st;
 };
 
+// u / d for u < 2^16, d < 2^16 with m = ceil(2^32 / d): the error u*(m - 2^32/d)/2^32
+// stays below 1/d, so the quotient is exact.
+__device__ __forceinline__ int div_magic(int u, uint32_t m) { return (int)__umulhi((uint32_t)u, m); }
+
 __host__ __device__ constexpr int smem_bytes(int kt_max, bool res) {
-  return 1024 + STAGES * WSTAGE + kt_max * (X_TILE + SF_TILE) * (res ? 2 : 1) + BAR_BYTES;
+  return 1024 + STAGES * WSTAGE + kt_max * (b_tile(res) + SF_TILE) + part_bytes(res) + BAR_BYTES;
 }
 
 template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
@@ -117,19 +130,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int KT = p.kt_max;
   uint8_t* xcodes = smem + STAGES * WSTAGE;                         // KT x 2 KB
-  uint8_t* rcodes = xcodes + KT * X_TILE;                           // KT x 2 KB (residue)
-  uint8_t* sfxp = rcodes + (RES ? KT * X_TILE : 0);                 // KT x 2 KB scale atoms
-  uint8_t* sfrp = sfxp + KT * SF_TILE;                              // KT x 2 KB (residue)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sfrp + (RES ? KT * SF_TILE : 0));
+  constexpr int BT = b_tile(RES);                                   // B tile bytes per k-tile
+  uint8_t* rcodes = xcodes + X_TILE;                                // R rows 16-31 of each B tile
+  uint8_t* sfxp = xcodes + KT * BT;                                 // KT x 2 KB scale atoms
+  uint8_t* sfrp = sfxp + NP * 16;                                   // R scales: atom lines 16-31
+  float* part = reinterpret_cast<float*>(sfxp + KT * SF_TILE);      // pushed partial rows
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(part) + part_bytes(RES));
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
   uint64_t* x_full = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* part = reinterpret_cast<float*>(smem);                     // overlays the W ring afterwards
   __shared__ uint32_t red[kWarps];
-  __shared__ uint32_t xch[2];                                       // published |x|, |r| maxima
+  __shared__ uint32_t xall[2][MAX_KS];                              // every CTA's |x|, |r| maximum
 
   griddep_launch_dependents();   // the next kernel may set itself up; it waits for this one's results
 
@@ -160,6 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  cluster_arrive_relaxed();   // this CTA is running: peers may store into its shared memory
+  bool peers_running = false; // this thread has waited for the peers' start-up arrivals
 
   auto w_chunks = [&](int kt) { return min(4, (p.K - kt * 256) / 64); };   // K = 64 chunks in k-tile kt
   auto load_w = [&](int kt, int s) {
@@ -180,17 +196,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   griddep_wait();   // everything below may read the preceding kernel's results
 
-  const int pre = min(nkt, STAGES);
-  if (warp == 0 && lane == 0) {
-    for (int i = 0; i < pre; ++i) load_w(kt0 + i, i);   // the ring starts empty
-    if (!FUSED) {
-      mbar_expect_tx(saddr(x_full), (uint32_t)(nkt * X_TILE * (RES ? 2 : 1)));
-      for (int t = 0; t < nkt; ++t) {
-        tma_load_2d(saddr(xcodes + t * X_TILE), &tmX, (kt0 + t) * 128, 0, saddr(x_full));
-        if (RES) tma_load_2d(saddr(rcodes + t * X_TILE), &tmR, (kt0 + t) * 128, 0, saddr(x_full));
+  // fused: issue the activation loads first, so they are not queued behind the W stream
+  [[maybe_unused]] Raw8<T> raw[FUSED ? R : 1];
+  [[maybe_unused]] const int c0 = kt0 * 256;
+  [[maybe_unused]] const int upr = (min(kt1 * 256, p.K) - c0) >> 3;   // 8-element units per row (multiple of 8)
+  // 2^32 / upr, rounded up (slices of one launch have one of two widths)
+  [[maybe_unused]] const uint32_t upr_m = (uint32_t)((0x100000000ull + (uint64_t)upr - 1) / (uint64_t)upr);
+  [[maybe_unused]] const int U = p.M * upr;
+  if constexpr (FUSED) {
+    const T* x = static_cast<const T*>(p.x);
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int u = i * kThreads + (int)threadIdx.x;
+      if (u < U) {
+        const int row = div_magic(u, upr_m), c8 = u - row * upr;
+        raw[i].load(x + (int64_t)row * p.ldx + c0 + c8 * 8);
+      } else {
+        raw[i].zero();
       }
     }
   }
+  const int pre = min(nkt, STAGES);
+  if (warp == 0 && lane == 0) {
+    if (!FUSED) {
+      mbar_expect_tx(saddr(x_full), (uint32_t)(nkt * BT));
+      for (int t = 0; t < nkt; ++t) {
+        tma_load_2d(saddr(xcodes + t * BT), &tmX, (kt0 + t) * 128, 0, saddr(x_full));
+        if (RES) tma_load_2d(saddr(rcodes + t * BT), &tmR, (kt0 + t) * 128, 0, saddr(x_full));
+      }
+    }
+    for (int i = 0; i < pre; ++i) load_w(kt0 + i, i);   // the ring starts empty
+  }
+
+  // Cluster-wide maximum: publish this CTA's maximum into every peer, then
+  // read all of them locally after one barrier.  Every thread calls it.
+  auto cluster_max = [&](uint32_t key, int which) {
+    const uint32_t m = block_max_u32(key, red);
+    if (!peers_running) {
+      cluster_wait();
+      peers_running = true;
+    }
+    if (threadIdx.x < ks) st_cluster_u32(mapa_shared(saddr(&xall[which][rank]), threadIdx.x), m);
+    cluster_sync();
+    return warp_max_u32(lane < (int)ks ? xall[which][lane] : 0u);
+  };
 
   float sx = 0.0f, sr = 0.0f;   // activation / residue tensor scales for the epilogue
   if constexpr (!FUSED) {
@@ -212,29 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         else if (n < p.M)
           word = *reinterpret_cast<const uint32_t*>(src + (size_t)n * nblk + chunk * 4);
       }
-      *reinterpret_cast<uint32_t*>((which ? sfrp : sfxp) + t * SF_TILE + j * 512 + n * 16) = word;
+      *reinterpret_cast<uint32_t*>((which ? sfrp : sfxp) + t * SF_TILE + j * 512 + n * 16) = word;   // R: lines 16-31
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   } else {
     // ---- quantize this CTA's K-slice of X into the operand layout
-    const T* x = static_cast<const T*>(p.x);
-    const int c0 = kt0 * 256;
-    const int upr = (min(kt1 * 256, p.K) - c0) >> 3;   // 8-element units per row (a multiple of 8)
-    const int U = p.M * upr;
     if (U > R * kThreads) report_status(p.st, NVFP4_ERR_UNSUPPORTED);   // the host split rules this out
     const bool reporter = rank == 0 && threadIdx.x == 0;
     const bool writer = blockIdx.y == 0;                // this cluster also writes Q(X), Q(R)
-    Raw8<T> raw[R];
     uint32_t key = 0u;
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-      const int u = i * kThreads + (int)threadIdx.x;
-      if (u < U) {
-        const int row = u / upr, c8 = u - row * upr;
-        raw[i].load(x + (int64_t)row * p.ldx + c0 + c8 * 8);
-      } else {
-        raw[i].zero();
-      }
       float v[8];
       raw[i].get(v);
 #pragma unroll
@@ -245,7 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (p.s_in != nullptr) {
       s = *p.s_in;
     } else {
-      s = scale_from_key(cluster_max_u32(key, red, &xch[0]), reporter, p.st);
+      s = scale_from_key(cluster_max(key, 0), reporter, p.st);
     }
     float s_r = (RES && p.sr_in != nullptr) ? *p.sr_in : 0.0f;
     if (writer && reporter) {
@@ -253,12 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (RES && p.sr_in != nullptr && p.r.s != p.sr_in) *p.r.s = s_r;
     }
 
-    // place one encoded unit: codes into the SW128 tile, the block scale into the packed scales
+    // place one encoded unit: codes into the SW128 tile, the block scale into its atom
     auto place = [&](uint8_t* codes_area, uint8_t* sf_area, const QOut& qo, int u, uint32_t codes, uint32_t db) {
-      const int row = u / upr, c8 = u - row * upr;
+      const int row = div_magic(u, upr_m), c8 = u - row * upr;
       const int t = c8 >> 5, kk = (c8 & 31) * 8;         // k-tile within the slice, column within it
       const int chunk16 = kk >> 5;                         // 16-byte chunk of the 128-byte row
-      *reinterpret_cast<uint32_t*>(codes_area + t * X_TILE + row * 128 + ((chunk16 ^ (row & 7)) << 4) +
+      *reinterpret_cast<uint32_t*>(codes_area + t * BT + row * 128 + ((chunk16 ^ (row & 7)) << 4) +
                                    ((kk & 31) >> 1)) = codes;
       const int bt = kk >> 4;                              // 16-block within the k-tile
       if ((c8 & 1) == 0) sf_area[t * SF_TILE + (bt >> 2) * 512 + row * 16 + (bt & 3)] = (uint8_t)db;
@@ -290,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (RES && p.sr_in == nullptr) {
-      s_r = scale_from_key(cluster_max_u32(rkey, red, &xch[1]), reporter, p.st);
+      s_r = scale_from_key(cluster_max(rkey, 1), reporter, p.st);
       if (writer && reporter) *p.r.s = s_r;
 #pragma unroll
       for (int i = 0; i < R; ++i) {
@@ -324,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------- MMA issuer
     bool ok = true;
     if (!FUSED) ok = mbar_wait(saddr(x_full), 0u, abort_flag, p.st);
-    const uint32_t idesc = idesc_nvf4(NP);
+    const uint32_t idesc = idesc_nvf4(RES ? 2 * NP : NP);
     int s = 0;
     uint32_t ph = 0;
     for (int kt = kt0; ok && kt < kt1; ++kt) {
@@ -335,17 +372,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < jmax; ++j) {
         tc_cp_scales(tmem + SFW_COL + 4 * j, desc_sf_atom(saddr(sb + W_TILE + j * 512)));
         tc_cp_scales(tmem + SFX_COL + 4 * j, desc_sf_atom(saddr(sfxp + t * SF_TILE + j * 512)));
-        if (RES) tc_cp_scales(tmem + SFR_COL + 4 * j, desc_sf_atom(saddr(sfrp + t * SF_TILE + j * 512)));
       }
-      const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(xcodes + t * X_TILE));
-      const uint64_t dr = desc_sw128(saddr(rcodes + t * X_TILE));
+      const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(xcodes + t * BT));
       for (int j = 0; j < jmax; ++j) {
         const uint32_t acc = (kt > kt0 || j > 0) ? 1u : 0u;
         tc_mma_nvf4(tmem + ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + SFW_COL + 4 * j,
                     tmem + SFX_COL + 4 * j, acc);
-        if (RES)
-          tc_mma_nvf4(tmem + ACC_R, dw + (uint64_t)(2 * j), dr + (uint64_t)(2 * j), idesc, tmem + SFW_COL + 4 * j,
-                      tmem + SFR_COL + 4 * j, acc);
       }
       tc_commit(saddr(&empty[s]));
       if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -358,11 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool ok = mbar_wait(saddr(acc_full), 0u, abort_flag, p.st);
   tc_fence_after();
   __syncwarp();     // the cluster barriers below are warp-aligned
-  // the partials overlay the W ring: a peer's ring is free once its MMAs are done
-  tc_fence_before();
-  cluster_arrive();
-  cluster_wait();
-  tc_fence_after();
+  if (!peers_running) cluster_wait();   // uniform: no maximum was exchanged
   const int rows_max = (int)((128u + ks - 1) / ks);
   auto owner_row0 = [&](uint32_t o) { return (int)((o * 128u + ks - 1) / ks); };
   if (warp < 4) {
@@ -424,58 +452,64 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ host side
 
-constexpr int kMaxUnitsPerThread = 8;   // fused mode: activation units held in registers
+constexpr double kFixedUs = 5.0;     // launch-to-exit latency of one wave of CTAs (measured, few k-tiles)
+constexpr double kTileUs = 0.8;      // issue time of one k-tile (8 scale copies, 4 MMAs, 1 commit) per CTA
+constexpr double kQuantUs = 4.0;     // one-launch quantizer plus the hand-off to the next kernel
+constexpr double kExchangeUs = 1.3;  // fused: one cluster-wide maximum (stores into peers + barrier)
+constexpr double kUnitUs = 0.15;     // fused: encoding one 8-element unit per thread, per co-resident CTA
 
 struct Choice {
   int ks = 0, kt_max = 0, smem = 0;
+  double cost = 1e30;
 };
 
-// Cluster split of K.  Cost model per wave of resident CTAs: a CTA issues its
-// own scale copies and MMAs (~0.6 us per k-tile), an SM shares HBM bandwidth
-// among its CTAs (~0.4 us per k-tile each); extra waves repeat the cost.  The
-// larger split wins among equal costs.
-Choice choose_split(int row_tiles, int k_tiles, bool res, int num_sms, int regs_per_thread, int M, int K,
-                    int units_per_thread_cap) {
+// Cluster split of K for a kernel instance with `regs` registers per thread:
+// waves of resident CTAs cost a fixed latency plus the per-CTA issue time of
+// their k-tiles and, fused (units_cap > 0), the cluster-wide maxima and the
+// encoding of the CTA's activation slice (every unit of which must fit in
+// units_cap registers arrays per thread).  The smaller split wins ties.
+Choice choose_split(int row_tiles, int k_tiles, bool res, int num_sms, int regs, int M, int K, int units_cap) {
   Choice best;
-  double best_cost = 1e30;
   for (int ks = 1; ks <= std::min(MAX_KS, k_tiles); ++ks) {
     const int kt_max = (k_tiles + ks - 1) / ks;
     const int smem = smem_bytes(kt_max, res);
     if (smem > 232448) continue;
-    if (units_per_thread_cap > 0) {   // fused: every activation unit of the slice fits in registers
-      const int slice = std::min(kt_max * 256, K);
-      if ((int64_t)M * (slice / 8) > (int64_t)units_per_thread_cap * kThreads) continue;
-    }
-    int per_sm = std::min(233472 / (smem + 1024), TMEM_CTAS);
-    per_sm = std::min(per_sm, 2048 / kThreads);
-    if (regs_per_thread > 0) per_sm = std::min(per_sm, 65536 / (regs_per_thread * kThreads));
+    const int slice = std::min(kt_max * 256, K);
+    const int64_t units = (int64_t)M * (slice / 8);
+    if (units_cap > 0 && units > (int64_t)units_cap * kThreads) continue;
+    int per_sm = std::min({233472 / (smem + 1024), TMEM_CTAS, 2048 / kThreads});
+    if (regs > 0) per_sm = std::min(per_sm, 65536 / (((regs + 7) / 8) * 8 * kThreads));
     if (per_sm < 1) continue;
-    const int64_t ctas = (int64_t)row_tiles * ks;
-    const int64_t slots = (int64_t)per_sm * num_sms;
+    const int64_t ctas = (int64_t)row_tiles * ks, slots = (int64_t)per_sm * num_sms;
     const int64_t waves = (ctas + slots - 1) / slots;
-    const double per_sm_ctas = (double)((std::min(ctas, slots) + num_sms - 1) / num_sms);
-    const double cost = (double)waves * std::max(0.6 * kt_max, 0.4 * per_sm_ctas * kt_max) + 0.01 * ks;
-    if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && ks > best.ks)) {
-      best_cost = cost;
-      best = Choice{ks, kt_max, smem};
+    double wave = kFixedUs + kTileUs * kt_max;
+    if (units_cap > 0) {
+      const double upt = (double)((units + kThreads - 1) / kThreads) * (res ? 2.0 : 1.0);
+      const double co_resident = (double)std::min<int64_t>(per_sm, (std::min(ctas, slots) + num_sms - 1) / num_sms);
+      wave += kExchangeUs * (res ? 2.0 : 1.0) + kUnitUs * co_resident * upt;
     }
+    const double cost = (double)waves * wave;
+    if (cost < best.cost - 1e-9) best = Choice{ks, kt_max, smem, cost};
   }
   return best;
 }
 
 template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
-cudaError_t launch_cfg(const DecodeArgs& a, DecodeParams p, const CUtensorMap& tmW, const CUtensorMap& tmX,
-                       const CUtensorMap& tmR, int num_sms, cudaStream_t stream) {
-  auto kern = k_decode_tc<T, FUSED, RES, BF16OUT, R>;
-  static int regs = -1;   // per instantiation
+int regs_of() {
+  static int regs = -1;
   if (regs < 0) {
     cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return cudaErrorInvalidDeviceFunction;
-    regs = fa.numRegs;
+    regs = cudaFuncGetAttributes(&fa, k_decode_tc<T, FUSED, RES, BF16OUT, R>) == cudaSuccess ? fa.numRegs : 255;
   }
+  return regs;
+}
+
+template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
+cudaError_t launch_cfg(const DecodeArgs& a, DecodeParams p, const Choice& c, const CUtensorMap& tmW,
+                       const CUtensorMap& tmX, const CUtensorMap& tmR, cudaStream_t stream) {
+  if (a.dry_run) return cudaSuccess;
+  auto kern = k_decode_tc<T, FUSED, RES, BF16OUT, R>;
   const int row_tiles = (int)((a.N + 127) / 128);
-  const Choice c = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs, (int)a.M, (int)a.K, FUSED ? R : 0);
-  if (c.ks == 0) return cudaErrorNotSupported;
   p.kt_max = c.kt_max;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem);
   if (e != cudaSuccess) return e;
@@ -503,20 +537,33 @@ cudaError_t launch_cfg(const DecodeArgs& a, DecodeParams p, const CUtensorMap& t
 template <typename T, bool FUSED, bool RES, bool BF16OUT>
 cudaError_t launch_r(const DecodeArgs& a, const DecodeParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
                      const CUtensorMap& tmR, int num_sms, cudaStream_t stream) {
+  const int row_tiles = (int)((a.N + 127) / 128);
+  const int M = (int)a.M, K = (int)a.K;
+  // the same kernel on NVFP4 operands: the split for the plain instance
+  const Choice plain = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<float, false, RES, BF16OUT, 0>(),
+                                    M, K, 0);
   if constexpr (!FUSED) {
-    return launch_cfg<T, FUSED, RES, BF16OUT, 0>(a, p, tmW, tmX, tmR, num_sms, stream);
+    if (plain.ks == 0) return cudaErrorNotSupported;
+    return launch_cfg<float, false, RES, BF16OUT, 0>(a, p, plain, tmW, tmX, tmR, stream);
   } else {
-    // units per thread for the split the launcher will pick is not known yet:
-    // size the register array for the worst split this shape allows
-    const int row_tiles = (int)((a.N + 127) / 128);
-    const Choice c = choose_split(row_tiles, p.k_tiles, RES, num_sms, 0, (int)a.M, (int)a.K, kMaxUnitsPerThread);
-    if (c.ks == 0) return cudaErrorNotSupported;
-    const int64_t units = a.M * (std::min<int64_t>((int64_t)c.kt_max * 256, a.K) / 8);
-    const int upt = (int)((units + kThreads - 1) / kThreads);
-    if (upt <= 1) return launch_cfg<T, FUSED, RES, BF16OUT, 1>(a, p, tmW, tmX, tmR, num_sms, stream);
-    if (upt <= 2) return launch_cfg<T, FUSED, RES, BF16OUT, 2>(a, p, tmW, tmX, tmR, num_sms, stream);
-    if (upt <= 4) return launch_cfg<T, FUSED, RES, BF16OUT, 4>(a, p, tmW, tmX, tmR, num_sms, stream);
-    return launch_cfg<T, FUSED, RES, BF16OUT, 8>(a, p, tmW, tmX, tmR, num_sms, stream);
+    // fused: the register-array size with the cheapest split; not worth it
+    // (cudaErrorNotSupported) when quantizing separately is estimated faster
+    const Choice c1 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 1>(), M, K, 1);
+    const Choice c2 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 2>(), M, K, 2);
+    const Choice c4 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 4>(), M, K, 4);
+    const Choice c8 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 8>(), M, K, 8);
+    const Choice* best = &c1;
+    int r = 1;
+    if (c2.cost < best->cost - 1e-9) { best = &c2; r = 2; }
+    if (c4.cost < best->cost - 1e-9) { best = &c4; r = 4; }
+    if (c8.cost < best->cost - 1e-9) { best = &c8; r = 8; }
+    if (best->ks == 0 || best->cost > plain.cost + kQuantUs) return cudaErrorNotSupported;
+    switch (r) {
+      case 1: return launch_cfg<T, true, RES, BF16OUT, 1>(a, p, *best, tmW, tmX, tmR, stream);
+      case 2: return launch_cfg<T, true, RES, BF16OUT, 2>(a, p, *best, tmW, tmX, tmR, stream);
+      case 4: return launch_cfg<T, true, RES, BF16OUT, 4>(a, p, *best, tmW, tmX, tmR, stream);
+      default: return launch_cfg<T, true, RES, BF16OUT, 8>(a, p, *best, tmW, tmX, tmR, stream);
+    }
   }
 }
 
@@ -537,8 +584,15 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
   if (a.M < 1 || a.M > NP || a.K % 64 != 0 || a.K < 256 || a.N < 1) return cudaErrorNotSupported;
   const bool fused = a.x != nullptr;
   CUtensorMap tmW, tmX, tmR;
-  if (!encode_codes_map(&tmW, a.w_codes, a.N, a.K, 128)) return cudaErrorInvalidValue;
-  if (!fused) {
+  if (a.dry_run) {
+    std::memset(&tmW, 0, sizeof(tmW));
+    tmX = tmR = tmW;
+  } else if (!encode_codes_map(&tmW, a.w_codes, a.N, a.K, 128)) {
+    return cudaErrorInvalidValue;
+  }
+  if (a.dry_run) {
+    // configuration only
+  } else if (!fused) {
     if (!encode_codes_map(&tmX, a.x_codes, a.M, a.K, NP)) return cudaErrorInvalidValue;
     if (a.r_codes != nullptr) {
       if (!encode_codes_map(&tmR, a.r_codes, a.M, a.K, NP)) return cudaErrorInvalidValue;
@@ -562,7 +616,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
   if (fused)
     return a.x_bf16 ? launch_t<__nv_bfloat16, true>(a, p, tmW, tmX, tmR, num_sms, stream)
                     : launch_t<float, true>(a, p, tmW, tmX, tmR, num_sms, stream);
-  return launch_t<uint8_t, false>(a, p, tmW, tmX, tmR, num_sms, stream);
+  return launch_t<float, false>(a, p, tmW, tmX, tmR, num_sms, stream);   // element type unused
 }
 
 }  // namespace nvfp4

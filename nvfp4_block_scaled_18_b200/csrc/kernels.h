@@ -72,7 +72,10 @@ struct DecodeArgs {
   void* y; int64_t ldy; bool y_bf16;
   int64_t M, N, K;
   int* st;
+  bool dry_run;                           // choose the configuration only; launch nothing
 };
+// cudaErrorNotSupported: fused mode is estimated slower than quantize-then-GEMM
+// (or does not fit); nothing was launched.
 cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_gemv(const GemmArgs& g, int num_sms, cudaStream_t stream);

@@ -16,7 +16,7 @@
  *  - "ResServe: Accurate and Efficient FP4 LLM Inference with Residue
  *    Compensation" abstract: FP4 activation base plus an FP4-quantized residue.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *  - one FP32 per-tensor scale s = fl32(amax / (6*448));
  *  - block scale d = E4M3_RNE(fl32(amax_block / fl32(6*s))), saturating at 448;
  *  - element code c = E2M1_RNE(fl32(x * fl32(1 / fl32(d*s)))), ties to the even

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import nvfp4_block_scaled_18_b200 as nv
 
@@ -103,3 +104,12 @@ def test_fused_decode_validation_before_launch(lib):
     w_bad = _tensor(256, 256, good, good, good, layout=1)
     assert g(good, 1, 4, 512, 512, None, ctypes.byref(q), ctypes.byref(w_bad), good, 0, 256, None, None) == 1
     assert g(good, 1, 4, 512, 512, None, None, ctypes.byref(w), good, 0, 256, None, None) == 1
+
+
+def test_quantize_gemm_plan_rejects_without_device(lib):
+    # unsupported sizes answer 0 before any CUDA call
+    assert nv.nvfp4_quantize_gemm_plan(17, 4096, 4096) == 0
+    assert nv.nvfp4_quantize_gemm_plan(4, 4096, 192) == 0
+    assert nv.nvfp4_quantize_gemm_plan(4, 4096, 320 + 16) == 0
+    assert nv.nvfp4_quantize_gemm_plan(16, 128, 65536) == 0
+    assert nv.nvfp4_quantize_gemm_plan(16, 128, 32768, x_dtype=torch.float32) == 0

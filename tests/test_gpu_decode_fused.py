@@ -181,3 +181,15 @@ def test_decode_kernel_on_nvfp4_operands(orc, x_layout, M, N, K):
         torch.cuda.synchronize()
         assert st.item() == 0
         assert rel_fro(y.cpu().numpy()[:, rows], ref) <= REL_FRO_TOL
+
+
+def test_quantize_gemm_plan():
+    """The launch plan names one fused launch for the small decode calls and
+    at most two launches for every decode shape."""
+    assert nv.nvfp4_quantize_gemm_plan(1, 4096, 4096) == 1
+    for M in wl.DECODE_M:
+        for (N, K) in wl.DECODE_SHAPES:
+            assert nv.nvfp4_quantize_gemm_plan(M, N, K) in (1, 2)
+        for (N, K) in wl.RESSERVE_SHAPES:
+            assert nv.nvfp4_quantize_gemm_plan(M, N, K, residue=True) in (1, 2)
+    assert nv.nvfp4_quantize_gemm_plan(17, 4096, 4096) == 0
