@@ -112,18 +112,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------ distributed
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """One process per GPU (torchrun env).  NCCL where CUDA is present, gloo
+    otherwise (host-only runs and tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    use_cuda = torch.cuda.is_available()
+    if backend is None:
+        backend = "nccl" if use_cuda else "gloo"
+    if use_cuda:
+        torch.cuda.set_device(local if world > 1 else 0)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -133,22 +137,32 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def _all_reduce_scalar(x: float, world: int, op) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    import torch.distributed as dist
+    return _all_reduce_scalar(x, world, dist.ReduceOp.MAX if world > 1 else None)
 
 
 def sum_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _all_reduce_scalar(x, world, dist.ReduceOp.SUM if world > 1 else None)
+
+
+def replica_throughput(work: float, ms: float, world: int, scale: float):
+    """Whole-job throughput of independent replicas: the work all ranks did over
+    the slowest rank's time.  Returns (value in units/s / scale, max ms)."""
+    ms_max = max_over_ranks(ms, world)
+    total = sum_over_ranks(work, world)
+    return total / (ms_max * 1e-3) / scale, ms_max
 
 
 # ------------------------------------------------------------ decode workload
@@ -692,21 +706,19 @@ def main():
     sampler = ClockSampler(torch.cuda.current_device())
     ms = time_graphs(graphs, steps, args.warmup, world, sampler)
     clocks = sampler.stop()
-    ms_max = max_over_ranks(ms, world)
-    value = sum_over_ranks(work_per_step * steps, world) / (ms_max * 1e-3) / scale
+    value, ms_max = replica_throughput(work_per_step * steps, ms, world, scale)
     ms_per_step = ms_max / steps
 
     # end to end: pinned host X -> device, quantize + GEMM, Y -> pinned host, every step
     e2e_steps = max(4 * phases, min(steps, 400)) if args.workload == "decode" else max(2, min(steps, 5))
     if args.workload == "decode":
         e2e_graphs = [EagerStep(wk, p, True) for p in range(phases)] if eager else capture_graphs(wk, phases, e2e=True)
-        ms_e2e = max_over_ranks(time_graphs(e2e_graphs, e2e_steps, args.warmup, world), world)
+        ms_e2e = time_graphs(e2e_graphs, e2e_steps, args.warmup, world)
         h2d, d2h = wk.h2d_bytes(), wk.d2h_bytes()
     else:
         ms_e2e, h2d, d2h = prefill_e2e(wk, e2e_steps), wk.h2d_bytes(), wk.d2h_bytes()
-        ms_e2e = max_over_ranks(ms_e2e, world)
         e2e_graphs = []
-    e2e_value = sum_over_ranks(work_per_step * e2e_steps, world) / (ms_e2e * 1e-3) / scale
+    e2e_value, _ = replica_throughput(work_per_step * e2e_steps, ms_e2e, world, scale)
 
     line = {"metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
             "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5)}

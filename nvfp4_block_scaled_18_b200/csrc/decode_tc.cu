@@ -29,8 +29,9 @@
 // Grid: (ks, ceil(N/128)), cluster (ks, 1, 1), ks <= 8.  CTA rank r of a
 // cluster handles k-tiles [r*kt/ks, (r+1)*kt/ks).  Roles (256 threads): every
 // warp takes part in the activation quantization; warp 0 lane 0 streams W
-// tiles and scale atoms through a TMA ring; warp 1 lane 0 issues the scale
-// copies and MMAs; warps 0-3 drain the accumulators and push their partial rows
+// tiles and scale atoms through a TMA ring; warp 2 lane 0 copies each stage's
+// scale atoms into TMEM (one buffer per stage) while warp 1 lane 0 issues the
+// MMAs of the previous stage; warps 0-3 drain the accumulators and push their partial rows
 // into a dedicated area of the owning CTA's shared memory (row r of the tile
 // belongs to rank floor(r*ks/128)); one cluster barrier later each owner sums
 // its rows and writes Y.  Per-CTA maxima travel the same way: each CTA writes
@@ -81,16 +82,18 @@ constexpr int max_part_rows() {
   return m;
 }
 constexpr int PART_ROWS = max_part_rows();   // 133 (ks = 7)
-// TMEM columns: acc [0,32) (X products in 0-15, R products in 16-31), W scales
-// [32,48), X/R scales [48,64)
-constexpr uint32_t ACC = 0, ACC_R = 16, SFW_COL = 32, SFX_COL = 48, TMEM_COLS = 64;
-static_assert(SFW_COL % 4 == 0 && SFX_COL % 4 == 0, "block-scaled MMA scale operands start on 4-column TMEM boundaries");
+// TMEM columns: acc [0,32) (X products in 0-15, R products in 16-31), then one
+// scale buffer per ring stage: W scales [+0,+16), X/R scales [+16,+32)
+constexpr uint32_t ACC = 0, ACC_R = 16, SF_COL = 32, SF_BUF = 32, SFX_OFF = 16, TMEM_COLS = 128;
+static_assert(SF_COL % 4 == 0 && SF_BUF % 4 == 0 && SFX_OFF % 4 == 0,
+              "block-scaled MMA scale operands start on 4-column TMEM boundaries");
+static_assert(SF_COL + STAGES * SF_BUF <= TMEM_COLS, "TMEM columns");
 constexpr int TMEM_CTAS = 512 / TMEM_COLS;
 
 static_assert(WSTAGE % 1024 == 0 && X_TILE % 1024 == 0, "SW128 tiles need 1024-byte alignment");
 static_assert(PART_ROWS == 133, "slot count for ks <= 8");
 __host__ __device__ constexpr int part_bytes(bool res) { return PART_ROWS * PITCH * 4 * (res ? 2 : 1); }
-static_assert((2 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier block");
+static_assert((3 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier block");
 
 struct DecodeParams {
   const void* x;        // fused: activations, M x K (ldx), bf16 or fp32
@@ -140,7 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
   uint64_t* x_full = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_full + 1);
+  uint64_t* sf_full = x_full + 1;                                   // [STAGES] scales copied to TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   __shared__ uint32_t red[kWarps];
   __shared__ uint32_t xall[2][MAX_KS];                              // every CTA's |x|, |r| maximum
@@ -158,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(saddr(&full[s]), 1);
       mbar_init(saddr(&empty[s]), 1);
+      mbar_init(saddr(&sf_full[s]), 1);
     }
     mbar_init(saddr(acc_full), 1);
     mbar_init(saddr(x_full), 1);
@@ -357,6 +362,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_w(kt, s);
       if (++s == STAGES) { s = 0; ph ^= 1u; }
     }
+  } else if (warp == 2 && lane == 0) {
+    // ------------------------------------------------ scale copies (own issuer)
+    // Stage s's scales go to TMEM buffer s.  A stage is refilled only after the
+    // MMAs that read it (and its scale buffer) have completed, so waiting for
+    // the stage's data is enough before overwriting the buffer.
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kt = kt0; kt < kt1; ++kt) {
+      if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) break;
+      tc_fence_after();
+      const int t = kt - kt0, jmax = w_chunks(kt);
+      const uint8_t* sb = smem + s * WSTAGE;
+      const uint32_t sfw = SF_COL + (uint32_t)s * SF_BUF, sfx = sfw + SFX_OFF;
+      for (int j = 0; j < jmax; ++j) {
+        tc_cp_scales(tmem + sfw + 4 * j, desc_sf_atom(saddr(sb + W_TILE + j * 512)));
+        tc_cp_scales(tmem + sfx + 4 * j, desc_sf_atom(saddr(sfxp + t * SF_TILE + j * 512)));
+      }
+      tc_commit(saddr(&sf_full[s]));
+      if (++s == STAGES) { s = 0; ph ^= 1u; }
+    }
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------- MMA issuer
     bool ok = true;
@@ -366,18 +391,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     for (int kt = kt0; ok && kt < kt1; ++kt) {
       if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) break;
+      if (!mbar_wait(saddr(&sf_full[s]), ph, abort_flag, p.st)) break;
       tc_fence_after();
       const int t = kt - kt0, jmax = w_chunks(kt);
       const uint8_t* sb = smem + s * WSTAGE;
-      for (int j = 0; j < jmax; ++j) {
-        tc_cp_scales(tmem + SFW_COL + 4 * j, desc_sf_atom(saddr(sb + W_TILE + j * 512)));
-        tc_cp_scales(tmem + SFX_COL + 4 * j, desc_sf_atom(saddr(sfxp + t * SF_TILE + j * 512)));
-      }
+      const uint32_t sfw = SF_COL + (uint32_t)s * SF_BUF, sfx = sfw + SFX_OFF;
       const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(xcodes + t * BT));
       for (int j = 0; j < jmax; ++j) {
         const uint32_t acc = (kt > kt0 || j > 0) ? 1u : 0u;
-        tc_mma_nvf4(tmem + ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + SFW_COL + 4 * j,
-                    tmem + SFX_COL + 4 * j, acc);
+        tc_mma_nvf4(tmem + ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + sfw + 4 * j,
+                    tmem + sfx + 4 * j, acc);
       }
       tc_commit(saddr(&empty[s]));
       if (++s == STAGES) { s = 0; ph ^= 1u; }

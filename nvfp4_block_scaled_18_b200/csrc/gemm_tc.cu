@@ -8,19 +8,22 @@
 // compensation (ARCQuant blog post, section 3.1-3.2: one GEMM over the
 // augmented K) runs through this kernel unchanged.
 //
-// Structure (persistent, one CTA per SM, 192 threads):
+// Structure (persistent, one CTA per SM, 352 threads):
 //   warp 0     one lane issues TMA loads of A/W code tiles (128 B K-slices,
 //              128-byte swizzle) and bulk copies of the matching scale atoms
 //              into a 3-stage shared-memory ring;
-//   warp 1     allocates 512 TMEM columns; one lane copies each stage's scale
-//              atoms into TMEM (tcgen05.cp 32x128b.warpx4, two alternating
-//              buffers) interleaved with the 4 MMAs (K = 64 each) of the stage;
-//              tcgen05.commit frees the stage and, at the end of a tile,
-//              signals the epilogue;
-//   warps 2-5  read the 128 x 256 fp32 accumulator (tcgen05.ld 32x32b.x32, one
-//              TMEM lane quadrant per warp), scale by s_a s_w, transpose each
-//              32 x 32 chunk through shared memory and store Y with coalesced
-//              16-byte stores.
+//   warp 2     one lane copies each stage's scale atoms into TMEM
+//              (tcgen05.cp 32x128b.warpx4) into one of two alternating
+//              buffers, and signals the MMA issuer through tcgen05.commit;
+//   warp 1     allocates 512 TMEM columns; one lane issues the 4 MMAs (K = 64
+//              each) of a stage once its scales are in TMEM; tcgen05.commit
+//              frees the stage (and, two stages later, its scale buffer) and,
+//              at the end of a tile, signals the epilogue;
+//   warps 3-10 read the 128 x 256 fp32 accumulator (tcgen05.ld 32x32b.x32; two
+//              warps per TMEM lane quadrant, 128 columns each), scale by
+//              s_a s_w, transpose each 32 x 32 chunk through shared memory and
+//              store Y with coalesced 16-byte stores.
+// Copies and MMAs come from two issuing threads so that they overlap.
 // Tiles are 128 x 256 x 256 (M x N x K); tile order walks M fastest so that the
 // CTAs in flight share W tiles through L2.  Every mbarrier wait is bounded: on
 // timeout the kernel records NVFP4_ERR_TIMEOUT, every role leaves its loop, and
@@ -41,17 +44,18 @@ constexpr int SFA_BYTES = 4 * 512;               // 4 k-atoms of one 128-row gro
 constexpr int SFB_BYTES = 2 * 4 * 512;           // 2 row groups x 4 k-atoms
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
 constexpr int OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
-constexpr int EPI_BYTES = 4 * 32 * 33 * 4;      // per epilogue warp: a 32 x 32 fp32 tile (+1 pad)
+constexpr int EPI_BYTES = 8 * 32 * 33 * 4;      // per epilogue warp: a 32 x 32 fp32 tile (+1 pad)
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;    // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;                  // 256 fp32 columns
 constexpr uint32_t SF_COL = 256;                 // two scale buffers of 48 columns, alternating by stage:
 constexpr uint32_t SF_BUF = 48;                  //   SFA 4 k-blocks x 4 columns, then SFB 4 k-blocks x 8
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 352;
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for 128B swizzle");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert((2 * STAGES + 2) * 8 + 8 <= 128 && 128 + 2 * 8 <= BAR_BYTES, "barrier block: ring, accumulator, scale buffers");
 
 struct TcParams {
   const uint8_t* sfa;
@@ -84,6 +88,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* sf_full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + EPI_BYTES + 128);   // [2] scales in TMEM
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -92,7 +97,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(saddr(&empty[s]), 1);
     }
     mbar_init(saddr(acc_full), 1);
-    mbar_init(saddr(acc_empty), 4);
+    mbar_init(saddr(&sf_full[0]), 1);
+    mbar_init(saddr(&sf_full[1]), 1);
+    mbar_init(saddr(acc_empty), 8);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -149,24 +156,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int jmax = min(4, (p.K - kt * BK) / 64);
         const uint8_t* st_base = smem + s * STAGE_BYTES;
         const uint32_t a0 = saddr(st_base), b0 = saddr(st_base + OFF_B);
-        // scales of consecutive stages go to alternate TMEM buffers, so copying
-        // this stage's scales does not wait on the previous stage's MMAs
-        const uint32_t sfa = SF_COL + (sf_flip & 1u) * SF_BUF, sfb = sfa + 16u;
+        const uint32_t buf = sf_flip & 1u;
+        const uint32_t sfa = SF_COL + buf * SF_BUF, sfb = sfa + 16u;
+        if (!mbar_wait(saddr(&sf_full[buf]), (sf_flip >> 1) & 1u, abort_flag, p.st)) goto mma_done;
+        tc_fence_after();
         ++sf_flip;
-        for (int j = 0; j < jmax; ++j) {
-          tc_cp_scales(tmem + sfa + 4 * j, desc_sf_atom(saddr(st_base + OFF_SFA + j * 512)));
-          for (int g = 0; g < ngroups; ++g)
-            tc_cp_scales(tmem + sfb + 8 * j + 4 * g, desc_sf_atom(saddr(st_base + OFF_SFB + g * 2048 + j * 512)));
+        for (int j = 0; j < jmax; ++j)
           tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a0) + (uint64_t)(2 * j), desc_sw128(b0) + (uint64_t)(2 * j),
                       idesc, tmem + sfa + 4 * j, tmem + sfb + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
-        }
         tc_commit(saddr(&empty[s]));  // stage reusable once these MMAs have read it
         if (++s == STAGES) { s = 0; ph ^= 1u; }
       }
       tc_commit(saddr(acc_full));     // accumulator complete
     }
   mma_done:;
-  } else if (warp >= 2) {
+  } else if (warp == 2 && lane == 0) {
+    // ----------------------------------------------------- scale copies (separate issuer)
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t gs = 0;   // global stage counter
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      const int nb = tile / p.m_blocks;
+      const int ngroups = min(2, p.b_groups - nb * 2);
+      for (int kt = 0; kt < p.k_tiles; ++kt, ++gs) {
+        if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) goto sf_done;
+        if (gs >= 2) {
+          const uint32_t g2 = gs - 2;
+          if (!mbar_wait(saddr(&empty[g2 % STAGES]), (g2 / STAGES) & 1u, abort_flag, p.st)) goto sf_done;
+        }
+        tc_fence_after();
+        const int jmax = min(4, (p.K - kt * BK) / 64);
+        const uint8_t* st_base = smem + s * STAGE_BYTES;
+        const uint32_t sfa = SF_COL + (gs & 1u) * SF_BUF, sfb = sfa + 16u;
+        for (int j = 0; j < jmax; ++j) {
+          tc_cp_scales(tmem + sfa + 4 * j, desc_sf_atom(saddr(st_base + OFF_SFA + j * 512)));
+          for (int g = 0; g < ngroups; ++g)
+            tc_cp_scales(tmem + sfb + 8 * j + 4 * g, desc_sf_atom(saddr(st_base + OFF_SFB + g * 2048 + j * 512)));
+        }
+        tc_commit(saddr(&sf_full[gs & 1u]));
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      }
+    }
+  sf_done:;
+  } else if (warp >= 3) {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     int local = 0;
@@ -178,9 +210,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // Each warp owns TMEM lanes (= tile rows) 32q..32q+31.  A 32 x 32 chunk is
       // read row-per-thread, transposed through shared memory, and written with
       // 16-byte stores in which 8 lanes cover one 128-byte row segment.
-      float* buf = epi + q * 32 * 33;
+      const int ew = warp - 3, half = ew / 4;
+      float* buf = epi + ew * 32 * 33;
       const int sub_r = lane >> 3, sub_c = (lane & 7) * 4;
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + c * 32, r);
         tmem_ld_wait();

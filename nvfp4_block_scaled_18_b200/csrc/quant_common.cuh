@@ -39,6 +39,51 @@ __device__ __forceinline__ uint32_t quant_half_block(const float v[8], float s, 
   return codes;
 }
 
+// Quantize one whole 16-element block held by one thread: the arithmetic of
+// quant_half_block (same block maximum, scale, reciprocal and per-element
+// rounding), without the pair exchange and with the per-block work done once.
+// Returns the 16 packed E2M1 nibbles, element i in bits 4i..4i+3.
+__device__ __forceinline__ uint64_t quant_block16(const float v[16], float s, uint32_t& d_byte, float* deq) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+  uint32_t db = 0;
+  if (s >= NVFP4_MIN_TENSOR_SCALE) db = f32_to_e4m3(__fdiv_rn(a, __fmul_rn(6.0f, s)));
+  const float d = e4m3_value(db);
+  const float inv = (d != 0.0f) ? __frcp_rn(__fmul_rn(d, s)) : 0.0f;
+  const uint32_t lo =
+      f32x8_to_e2m1(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv), __fmul_rn(v[3], inv),
+                    __fmul_rn(v[4], inv), __fmul_rn(v[5], inv), __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+  const uint32_t hi =
+      f32x8_to_e2m1(__fmul_rn(v[8], inv), __fmul_rn(v[9], inv), __fmul_rn(v[10], inv), __fmul_rn(v[11], inv),
+                    __fmul_rn(v[12], inv), __fmul_rn(v[13], inv), __fmul_rn(v[14], inv), __fmul_rn(v[15], inv));
+  if (deq != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      deq[i] = __fmul_rn(__fmul_rn(e2m1_value(lo >> (4 * i)), d), s);
+      deq[8 + i] = __fmul_rn(__fmul_rn(e2m1_value(hi >> (4 * i)), d), s);
+    }
+  }
+  d_byte = db;
+  return (uint64_t)lo | ((uint64_t)hi << 32);
+}
+
+// Load 16 consecutive elements (32-byte aligned for bf16, 64-byte for fp32) as fp32.
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float v[16]) {
+  load8(p, v);
+  load8(p + 8, v + 8);
+}
+__device__ __forceinline__ void load16(const float* p, float v[16]) {
+  load8(p, v);
+  load8(p + 8, v + 8);
+}
+
+// Store the codes (8 bytes) and scale of block b of `row` (block-per-thread kernels).
+__device__ __forceinline__ void store_block16(const QOut& q, int64_t row, int b, uint64_t codes, uint32_t d_byte) {
+  *reinterpret_cast<uint64_t*>(q.codes + row * (q.cols >> 1) + (int64_t)b * 8) = codes;
+  q.scales[scale_offset(row, b, q.cols >> 4, q.tiled)] = (uint8_t)d_byte;
+}
+
 __device__ __forceinline__ void store_half_block(const QOut& q, int64_t row, int64_t col8,
                                                  uint32_t codes, uint32_t d_byte) {
   *reinterpret_cast<uint32_t*>(q.codes + row * (q.cols >> 1) + col8 * 4) = codes;

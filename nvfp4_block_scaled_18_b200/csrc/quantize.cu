@@ -14,9 +14,9 @@
 //
 // Every rounding step uses an explicit _rn intrinsic so that no multiply-add
 // is contracted: the codes and scales are bit-identical to the definition in
-// include/nvfp4.h.  Thread mapping: one thread owns 8 consecutive elements
-// (one 16-byte bf16 vector); the two threads of an even/odd lane pair own one
-// 16-element block and exchange their half-block maxima with one shuffle.
+// include/nvfp4.h.  Thread mapping: one thread owns one 16-element block (two
+// 16-byte bf16 vectors), so the per-block scale, division and reciprocal are
+// computed once per block.
 #include "common.cuh"
 #include "kernels.h"
 #include "quant_common.cuh"
@@ -72,50 +72,43 @@ __global__ void __launch_bounds__(256) k_amax(const T* __restrict__ x, int64_t M
   finish_tensor_scale(key, &ws->amax_bits[slot], &ws->arrive[slot], s_out, st);
 }
 
+// One thread per 16-element block (two 16-byte bf16 loads); a CTA covers up to
+// 256 consecutive blocks of a row, rows grid-strided over blockIdx.y.
 template <typename T, int MODE>
 __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t M, int64_t K,
                                                int64_t ldx, const float* s_ptr,
                                                const float* sr_ptr, QOut q, QOut r, WsHeader* ws,
                                                int* st) {
-  const int64_t upr = K >> 3;
+  const int nb = (int)(K >> 4);
   const float s = *s_ptr;
   const float s_r = (MODE == Q_RES_ONLY || MODE == Q_BOTH) ? *sr_ptr : 0.0f;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     if (MODE != Q_RES_ONLY && q.s != s_ptr) *q.s = s;
     if (MODE == Q_BOTH && r.s != sr_ptr) *r.s = s_r;
   }
+  const int b = (int)(blockIdx.x * blockDim.x + threadIdx.x);
   uint32_t bad = 0, rkey = 0;
-  for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
-    for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < upr;
-         base += (int64_t)gridDim.x * blockDim.x) {
-      const int64_t c8 = base + threadIdx.x;
-      const bool act = c8 < upr;
-      float v[8];
-      if (act) {
-        load8(x + row * ldx + c8 * 8, v);
-      } else {
+  if (b < nb) {
+    for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
+      float v[16];
+      load16(x + row * ldx + (int64_t)b * 16, v);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) bad = max(bad, abs_key(v[i]));
+      for (int i = 0; i < 16; ++i) bad = max(bad, abs_key(v[i]));
       uint32_t db;
-      float deq[8];
-      const uint32_t codes = quant_half_block(v, s, db, MODE == Q_PLAIN ? nullptr : deq);
-      if (act && MODE != Q_RES_ONLY) store_half_block(q, row, c8, codes, db);
+      float deq[16];
+      const uint64_t codes = quant_block16(v, s, db, MODE == Q_PLAIN ? nullptr : deq);
+      if (MODE != Q_RES_ONLY) store_block16(q, row, b, codes, db);
       if (MODE != Q_PLAIN) {
-        float rv[8];
+        float rv[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) rv[i] = __fsub_rn(v[i], deq[i]);
+        for (int i = 0; i < 16; ++i) rv[i] = __fsub_rn(v[i], deq[i]);
         if (MODE == Q_MAIN_AMAXR) {
-          if (act) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) rkey = max(rkey, abs_key(rv[i]));
-          }
+          for (int i = 0; i < 16; ++i) rkey = max(rkey, abs_key(rv[i]));
         } else {
           uint32_t dr;
-          const uint32_t rc = quant_half_block(rv, s_r, dr, nullptr);
-          if (act) store_half_block(r, row, c8, rc, dr);
+          const uint64_t rc = quant_block16(rv, s_r, dr, nullptr);
+          store_block16(r, row, b, rc, dr);
         }
       }
     }
@@ -127,17 +120,17 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
 // ------------------------------------------------- single-launch small inputs
 // Decode-sized activations (a few rows) are too small to hide two or three
 // dependent launches.  One cluster of kQC CTAs quantizes the whole tensor in
-// one launch: each thread keeps its 8-element units in registers, the CTAs
+// one launch: each thread keeps its 16-element blocks in registers, the CTAs
 // exchange their |x| maxima through distributed shared memory behind a cluster
 // barrier, and every CTA derives the same tensor scale.  The arithmetic is the
-// same quant_half_block as above, so codes and scales are identical to the
-// multi-launch path.
+// same per-block routine (quant_block16) as k_quant, so codes and scales are
+// identical to the multi-launch path.
 
 constexpr int kQC = 8;              // CTAs per cluster (portable cluster size)
 constexpr int kQThreads = 512;      // threads per CTA
-constexpr int kQUnitsPerChunk = kQC * kQThreads;
+constexpr int kQUnitsPerChunk = kQC * kQThreads;   // 16-element blocks per chunk of the cluster
 
-// Unit u (8 elements) of this thread's i-th chunk.  Grid: exactly one cluster.
+// Block u (16 elements) of this thread's i-th chunk.  Grid: exactly one cluster.
 template <typename T, int R, bool RES>
 __global__ void __launch_bounds__(kQThreads, 1)
     k_quant_cluster(const T* __restrict__ x, int M, int K, int64_t ldx, const float* s_in,
@@ -149,25 +142,32 @@ __global__ void __launch_bounds__(kQThreads, 1)
   tc::griddep_launch_dependents();
   tc::griddep_wait();
   const uint32_t rank = tc::cluster_ctarank();
-  const int upr = K >> 3;
-  const int U = M * upr;
+  const int nb = K >> 4;
+  const int U = M * nb;
   const bool reporter = rank == 0 && threadIdx.x == 0;
 
-  Raw8<T> raw[R];
+  Raw8<T> raw[R][2];
   uint32_t key = 0u;
 #pragma unroll
   for (int i = 0; i < R; ++i) {
     const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
     if (u < U) {
-      const int row = u / upr, c8 = u - row * upr;
-      raw[i].load(x + (int64_t)row * ldx + (int64_t)c8 * 8);
+      const int row = u / nb, b = u - row * nb;
+      const T* src = x + (int64_t)row * ldx + (int64_t)b * 16;
+      raw[i][0].load(src);
+      raw[i][1].load(src + 8);
     } else {
-      raw[i].zero();
+      raw[i][0].zero();
+      raw[i][1].zero();
     }
-    float v[8];
-    raw[i].get(v);
+  }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
+  for (int i = 0; i < R; ++i) {
+    float v[16];
+    raw[i][0].get(v);
+    raw[i][1].get(v + 8);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) key = max(key, abs_key(v[j]));
   }
   if (key >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
 
@@ -184,23 +184,24 @@ __global__ void __launch_bounds__(kQThreads, 1)
   for (int i = 0; i < R; ++i) {
     const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
     const bool act = u < U;
-    const int row = act ? u / upr : 0, c8 = act ? u - row * upr : 0;
-    float v[8], deq[8];
-    raw[i].get(v);
+    const int row = act ? u / nb : 0, b = act ? u - row * nb : 0;
+    float v[16], deq[16];
+    raw[i][0].get(v);
+    raw[i][1].get(v + 8);
     uint32_t db;
-    const uint32_t codes = quant_half_block(v, s, db, RES ? deq : nullptr);
-    if (act) store_half_block(q, row, c8, codes, db);
+    const uint64_t codes = quant_block16(v, s, db, RES ? deq : nullptr);
+    if (act) store_block16(q, row, b, codes, db);
     if (RES) {
-      float rv[8];
+      float rv[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) rv[j] = __fsub_rn(v[j], deq[j]);
+      for (int j = 0; j < 16; ++j) rv[j] = __fsub_rn(v[j], deq[j]);
       if (sr_in != nullptr) {
         uint32_t dr;
-        const uint32_t rc = quant_half_block(rv, s_r, dr, nullptr);
-        if (act) store_half_block(r, row, c8, rc, dr);
+        const uint64_t rc = quant_block16(rv, s_r, dr, nullptr);
+        if (act) store_block16(r, row, b, rc, dr);
       } else if (act) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) rkey = max(rkey, abs_key(rv[j]));
+        for (int j = 0; j < 16; ++j) rkey = max(rkey, abs_key(rv[j]));
       }
     }
   }
@@ -211,16 +212,17 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
-      const bool act = u < U;
-      const int row = act ? u / upr : 0, c8 = act ? u - row * upr : 0;
-      float v[8], deq[8], rv[8];
-      raw[i].get(v);
+      if (u >= U) continue;
+      const int row = u / nb, b = u - row * nb;
+      float v[16], deq[16], rv[16];
+      raw[i][0].get(v);
+      raw[i][1].get(v + 8);
       uint32_t db, dr;
-      (void)quant_half_block(v, s, db, deq);
+      (void)quant_block16(v, s, db, deq);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) rv[j] = __fsub_rn(v[j], deq[j]);
-      const uint32_t rc = quant_half_block(rv, s_r, dr, nullptr);
-      if (act) store_half_block(r, row, c8, rc, dr);
+      for (int j = 0; j < 16; ++j) rv[j] = __fsub_rn(v[j], deq[j]);
+      const uint64_t rc = quant_block16(rv, s_r, dr, nullptr);
+      store_block16(r, row, b, rc, dr);
     }
   }
   if (exchange) tc::cluster_sync();  // peers may read this CTA's xch words until here
@@ -317,8 +319,8 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
     sperm[k] = p;
     if (gamma) sgamma[k] = load1(gamma + k);
   }
-  const int64_t upr = K >> 3;
-  const int64_t rupr = S >> 3;
+  const int nb = (int)(K >> 4);     // blocks of the reordered row
+  const int nbr = (int)(S >> 4);    // residue blocks (the first S reordered columns)
   uint32_t bad = 0;
   for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
     __syncthreads();  // previous row fully consumed (and sperm/sgamma ready)
@@ -327,32 +329,33 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
       reinterpret_cast<uint4*>(srow)[c] = __ldg(reinterpret_cast<const uint4*>(xr) + c);
     __syncthreads();
     const float ri = gamma ? rinv[row] : 1.0f;
-    for (int64_t base = 0; base < upr; base += blockDim.x) {
-      const int64_t c8 = base + threadIdx.x;
-      const bool act = c8 < upr;
-      float v[8];
+    // one thread per 16-element block of the reordered row
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+      float v[16];
+      int32_t pv[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float y = 0.0f;
-        if (act) {
-          const int32_t p = sperm[c8 * 8 + i];
-          y = load1(srow + p);
-          bad = max(bad, abs_key(y));
-          if (gamma) y = __fmul_rn(__fmul_rn(y, ri), sgamma[p]);
-        }
+      for (int j = 0; j < 4; ++j)   // 16-byte reads of the cached permutation (no bank conflicts)
+        *reinterpret_cast<int4*>(pv + 4 * j) = reinterpret_cast<const int4*>(sperm)[b * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int32_t p = pv[i];
+        float y = load1(srow + p);
+        bad = max(bad, abs_key(y));
+        if (gamma) y = __fmul_rn(__fmul_rn(y, ri), sgamma[p]);
         v[i] = y;
       }
       uint32_t db;
-      float deq[8];
-      const uint32_t codes = quant_half_block(v, s, db, deq);
-      if (act) store_half_block(q, row, c8, codes, db);
-      if (base < rupr) {  // uniform across the CTA: every lane takes part in the shuffle
-        float rv[8];
+      float deq[16];
+      const bool res = b < nbr;
+      const uint64_t codes = quant_block16(v, s, db, res ? deq : nullptr);
+      store_block16(q, row, b, codes, db);
+      if (res) {
+        float rv[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) rv[i] = __fsub_rn(v[i], deq[i]);
+        for (int i = 0; i < 16; ++i) rv[i] = __fsub_rn(v[i], deq[i]);
         uint32_t dr;
-        const uint32_t rc = quant_half_block(rv, s, dr, nullptr);
-        if (c8 < rupr) store_half_block(q, row, upr + c8, rc, dr);
+        const uint64_t rc = quant_block16(rv, s, dr, nullptr);
+        store_block16(q, row, nb + b, rc, dr);
       }
     }
   }
@@ -363,8 +366,9 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
 
 // ------------------------------------------------- single-launch small inputs
 
+// capacity in 8-element units: each thread holds up to 8 (bf16) / 4 (fp32) 16-element blocks
 int64_t quant_small_max_units(nvfp4_dtype dt) {
-  return (int64_t)kQUnitsPerChunk * (dt == NVFP4_BF16 ? 16 : 8);
+  return 2 * (int64_t)kQUnitsPerChunk * (dt == NVFP4_BF16 ? 8 : 4);
 }
 
 template <typename T, int R, bool RES>
@@ -393,13 +397,13 @@ template <typename T, bool RES>
 cudaError_t launch_quant_cluster_t(const void* x, int64_t M, int64_t K, int64_t ldx, const float* s_in,
                                    const float* sr_in, const QOut& q, const QOut& r, int* st,
                                    cudaStream_t stream) {
-  const int64_t chunks = (M * (K >> 3) + kQUnitsPerChunk - 1) / kQUnitsPerChunk;
+  // chunks of kQUnitsPerChunk 16-element blocks
+  const int64_t chunks = (M * (K >> 4) + kQUnitsPerChunk - 1) / kQUnitsPerChunk;
   if (chunks <= 1) return launch_quant_cluster_r<T, 1, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
   if (chunks <= 2) return launch_quant_cluster_r<T, 2, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
   if (chunks <= 4) return launch_quant_cluster_r<T, 4, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
-  if (chunks <= 8) return launch_quant_cluster_r<T, 8, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
   if constexpr (sizeof(T) == 2) {
-    if (chunks <= 16) return launch_quant_cluster_r<T, 16, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
+    if (chunks <= 8) return launch_quant_cluster_r<T, 8, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
   }
   return cudaErrorNotSupported;
 }
@@ -439,11 +443,19 @@ cudaError_t launch_amax(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int
              : launch_amax_t<float>(x, M, K, ldx, ws, slot, s_out, st, num_sms, stream);
 }
 
+// k_quant grid: one thread per 16-element block, (x) blocks of a row, (y) rows.
+static inline dim3 quant_block_grid(int64_t M, int64_t K, int num_sms) {
+  const int64_t gx = std::min<int64_t>(((K >> 4) + 255) / 256, 65535);
+  const int64_t target = (int64_t)num_sms * 8;
+  const int64_t gy = std::max<int64_t>(1, std::min<int64_t>({M, 65535, (target + gx - 1) / gx}));
+  return dim3((unsigned)gx, (unsigned)gy);
+}
+
 template <typename T>
 cudaError_t launch_quant_t(int mode, const void* x, int64_t M, int64_t K, int64_t ldx,
                            const float* s_ptr, const float* sr_ptr, const QOut& q, const QOut& r,
                            WsHeader* ws, int* st, int num_sms, cudaStream_t stream) {
-  const dim3 g = quant_grid(M, K, num_sms);
+  const dim3 g = quant_block_grid(M, K, num_sms);
   const T* xp = static_cast<const T*>(x);
   switch (mode) {
     case Q_PLAIN: k_quant<T, Q_PLAIN><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
@@ -494,7 +506,9 @@ cudaError_t launch_reorder_quant_t(const void* x, int64_t M, int64_t K, int64_t 
   cudaError_t e = cudaFuncSetAttribute(k_reorder_quant<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  const int per_sm = smem <= 72 * 1024 ? 3 : (smem <= 110 * 1024 ? 2 : 1);
+  // rows are processed one at a time per CTA (load, barrier, encode): keep
+  // several CTAs per SM so that rows overlap
+  const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (200 * 1024) / smem));
   const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * per_sm));
   k_reorder_quant<T><<<g, 256, smem, stream>>>(static_cast<const T*>(x), M, K, ldx,
                                                static_cast<const T*>(gamma), rinv, perm, S, s_ptr,
