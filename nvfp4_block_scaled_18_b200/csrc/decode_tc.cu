@@ -33,21 +33,25 @@
 // scale atoms into TMEM (one buffer per stage) while warp 1 lane 0 issues the
 // MMAs of the previous stage; warps 0-3 drain the accumulators and push their partial rows
 // into a dedicated area of the owning CTA's shared memory (row r of the tile
-// belongs to rank floor(r*ks/128)); one cluster barrier later each owner sums
-// its rows and writes Y.  Per-CTA maxima travel the same way: each CTA writes
-// its maximum into every peer, so one barrier later every CTA reads all of them
-// locally.  Every CTA announces at start-up that it is running (a relaxed
-// cluster arrive) and waits for its peers' announcements before its first
-// store into another CTA's shared memory.
+// belongs to rank floor(r*ks/128)); each owner sums its rows and writes Y.
+// Per-CTA maxima travel the same way: each CTA sends its maximum to every
+// peer.  All traffic between CTAs is point to point: st.async stores whose
+// bytes complete on an mbarrier of the receiving CTA, armed at start-up with
+// the exact byte count it will receive, so a receiver waits only for its own
+// data and no cluster-wide barrier sits on the critical path.  Every CTA
+// announces at start-up that it is running (a relaxed cluster arrive) and
+// waits for its peers' announcements before its first store into another CTA's
+// shared memory; it exits only after every byte addressed to it has arrived.
 //
 // The kernel is a programmatic dependent of the preceding kernel: before
 // griddepcontrol.wait it only sets up and asks L2 to prefetch its W tiles
 // (L2 is coherent, so a prefetch never yields stale data); every load that
 // feeds the result is issued after the wait.
 //
-// Safety: every mbarrier wait is bounded; every CTA reaches every cluster
-// barrier on every path (the barrier sequence depends only on kernel
-// arguments, which are uniform over the cluster); the shared-memory request
+// Safety: every mbarrier wait is bounded; every CTA reaches the start-up
+// cluster barrier and sends every store its peers count on, on every path
+// (both depend only on kernel arguments, which are uniform over the cluster,
+// and a CTA whose pipeline gave up sends zeros); the shared-memory request
 // covers the whole layout and the CTAs per SM are capped so that their TMEM
 // allocations always fit side by side.
 #include <cstring>
@@ -93,7 +97,7 @@ constexpr int TMEM_CTAS = 512 / TMEM_COLS;
 static_assert(WSTAGE % 1024 == 0 && X_TILE % 1024 == 0, "SW128 tiles need 1024-byte alignment");
 static_assert(PART_ROWS == 133, "slot count for ks <= 8");
 __host__ __device__ constexpr int part_bytes(bool res) { return PART_ROWS * PITCH * 4 * (res ? 2 : 1); }
-static_assert((3 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier block");
+static_assert((3 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier block");
 
 struct DecodeParams {
   const void* x;        // fused: activations, M x K (ldx), bf16 or fp32
@@ -144,7 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = bars + 2 * STAGES;
   uint64_t* x_full = acc_full + 1;
   uint64_t* sf_full = x_full + 1;                                   // [STAGES] scales copied to TMEM
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + STAGES);
+  uint64_t* xbar = sf_full + STAGES;                                // [2] peers' |x|, |r| maxima arrived
+  uint64_t* pbar = xbar + 2;                                        // peers' partial rows arrived
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   __shared__ uint32_t red[kWarps];
   __shared__ uint32_t xall[2][MAX_KS];                              // every CTA's |x|, |r| maximum
@@ -157,6 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt0 = (int)((rank * (uint32_t)p.k_tiles) / ks);
   const int kt1 = (int)(((rank + 1) * (uint32_t)p.k_tiles) / ks);
   const int nkt = kt1 - kt0;
+  // rows [owner_row0(o), owner_row0(o + 1)) of the tile are summed by rank o
+  auto owner_row0 = [&](uint32_t o) { return (int)((o * 128u + ks - 1) / ks); };
+  const bool x_exchange = FUSED && p.s_in == nullptr;
+  const bool r_exchange = FUSED && RES && p.sr_in == nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -166,6 +176,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(saddr(acc_full), 1);
     mbar_init(saddr(x_full), 1);
+    for (int i = 0; i < 2; ++i) mbar_init(saddr(&xbar[i]), 1);
+    mbar_init(saddr(pbar), 1);
+    // Arm the receive barriers with every byte the peers will send: one word
+    // per exchanged maximum, and 16 (X) or 32 (X and R) floats per owned row.
+    if (x_exchange) mbar_expect_tx(saddr(&xbar[0]), (ks - 1u) * 4u);
+    if (r_exchange) mbar_expect_tx(saddr(&xbar[1]), (ks - 1u) * 4u);
+    const uint32_t owned = (uint32_t)(owner_row0(rank + 1) - owner_row0(rank));
+    mbar_expect_tx(saddr(pbar), (ks - 1u) * owned * (uint32_t)(NP * 4 * (RES ? 2 : 1)));
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -233,17 +251,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < pre; ++i) load_w(kt0 + i, i);   // the ring starts empty
   }
 
-  // Cluster-wide maximum: publish this CTA's maximum into every peer, then
-  // read all of them locally after one barrier.  Every thread calls it.
+  // Cluster-wide maximum: send this CTA's maximum to every peer (st.async,
+  // counted on the peer's barrier xbar[which]), then wait until all peers'
+  // maxima have arrived here.  Every thread calls it.
   auto cluster_max = [&](uint32_t key, int which) {
     const uint32_t m = block_max_u32(key, red);
     if (!peers_running) {
       cluster_wait();
       peers_running = true;
     }
-    if (threadIdx.x < ks) st_cluster_u32(mapa_shared(saddr(&xall[which][rank]), threadIdx.x), m);
-    cluster_sync();
-    return warp_max_u32(lane < (int)ks ? xall[which][lane] : 0u);
+    if (threadIdx.x < ks && threadIdx.x != rank)
+      st_async_u32(mapa_shared(saddr(&xall[which][rank]), threadIdx.x), m,
+                   mapa_shared(saddr(&xbar[which]), threadIdx.x));
+    (void)mbar_wait<true>(saddr(&xbar[which]), 0u, abort_flag, p.st);
+    return max(m, warp_max_u32(lane < (int)ks && lane != (int)rank ? xall[which][lane] : 0u));
   };
 
   float sx = 0.0f, sr = 0.0f;   // activation / residue tensor scales for the epilogue
@@ -412,15 +433,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------- push this CTA's partial rows to the CTA that owns them
   const bool ok = mbar_wait(saddr(acc_full), 0u, abort_flag, p.st);
   tc_fence_after();
-  __syncwarp();     // the cluster barriers below are warp-aligned
+  __syncwarp();     // the cluster barrier below is warp-aligned
   if (!peers_running) cluster_wait();   // uniform: no maximum was exchanged
   const int rows_max = (int)((128u + ks - 1) / ks);
-  auto owner_row0 = [&](uint32_t o) { return (int)((o * 128u + ks - 1) / ks); };
   if (warp < 4) {
+    // Own rows are stored locally; the others travel by st.async and are
+    // counted on the owner's barrier pbar.
     const int row = warp * 32 + lane;                              // TMEM lane = W row of the tile
     const uint32_t o = (uint32_t)row * ks / 128u;
     const int slot = (int)rank * rows_max + (row - owner_row0(o));
+    const bool local = o == rank;
     const uint32_t dst = mapa_shared(saddr(part + slot * PITCH), o);
+    const uint32_t dst_bar = mapa_shared(saddr(pbar), o);
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
 #pragma unroll
     for (int acc_i = 0; acc_i < (RES ? 2 : 1); ++acc_i) {
@@ -431,15 +455,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = 0u;
       }
-      const uint32_t dsti = dst + (uint32_t)(acc_i * PART_ROWS * PITCH * 4);
+      const int off = acc_i * PART_ROWS * PITCH;
+      if (local) {
 #pragma unroll
-      for (int i = 0; i < 16; i += 4)
-        st_cluster_f32x4(dsti + (uint32_t)(i * 4), __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                         __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<uint4*>(part + slot * PITCH + off + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+          st_async_f32x4(dst + (uint32_t)((off + i) * 4), __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                         __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]), dst_bar);
+      }
     }
   }
   tc_fence_before();
-  cluster_sync();   // every partial has landed in its owner's shared memory
+  __syncthreads();  // own partial rows stored; TMEM reads done before the dealloc
+  // Every peer's partial rows have landed here.  Each CTA also waits for all
+  // bytes addressed to it before it exits, so no store targets an exited CTA.
+  (void)mbar_wait<true>(saddr(pbar), 0u, abort_flag, p.st);
 
   // ------------------------------------------------ owners sum their rows and store
   {
@@ -478,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr double kFixedUs = 5.0;     // launch-to-exit latency of one wave of CTAs (measured, few k-tiles)
 constexpr double kTileUs = 0.8;      // issue time of one k-tile (8 scale copies, 4 MMAs, 1 commit) per CTA
 constexpr double kQuantUs = 4.0;     // one-launch quantizer plus the hand-off to the next kernel
-constexpr double kExchangeUs = 1.3;  // fused: one cluster-wide maximum (stores into peers + barrier)
+constexpr double kExchangeUs = 1.3;  // fused: one cluster-wide maximum (stores into peers + wait)
 constexpr double kUnitUs = 0.15;     // fused: encoding one 8-element unit per thread, per co-resident CTA
 
 struct Choice {
