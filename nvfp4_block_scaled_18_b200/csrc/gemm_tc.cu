@@ -11,7 +11,7 @@
 // Structure (persistent, one CTA per SM, 352 threads):
 //   warp 0     one lane issues TMA loads of A/W code tiles (128 B K-slices,
 //              128-byte swizzle) and bulk copies of the matching scale atoms
-//              into a 3-stage shared-memory ring;
+//              into a 4-stage shared-memory ring;
 //   warp 2     one lane copies each stage's scale atoms into TMEM
 //              (tcgen05.cp 32x128b.warpx4) into one of two alternating
 //              buffers, and signals the MMA issuer through tcgen05.commit;
@@ -19,10 +19,12 @@
 //              each) of a stage once its scales are in TMEM; tcgen05.commit
 //              frees the stage (and, two stages later, its scale buffer) and,
 //              at the end of a tile, signals the epilogue;
-//   warps 3-10 read the 128 x 256 fp32 accumulator (tcgen05.ld 32x32b.x32; two
-//              warps per TMEM lane quadrant, 128 columns each), scale by
-//              s_a s_w, transpose each 32 x 32 chunk through shared memory and
-//              store Y with coalesced 16-byte stores.
+//   warps 3-10 read the 128 x 256 fp32 accumulator into registers
+//              (tcgen05.ld 32x32b.x32; two warps per TMEM lane quadrant, 128
+//              columns each) and release it at once, so that the next tile's
+//              MMAs start while they scale by s_a s_w, transpose 32 x 8 chunks
+//              through shared memory and store Y with 16-byte stores, two
+//              lanes per 32-byte row segment.
 // Copies and MMAs come from two issuing threads so that they overlap.
 // Tiles are 128 x 256 x 256 (M x N x K); tile order walks M fastest so that the
 // CTAs in flight share W tiles through L2.  Every mbarrier wait is bounded: on
@@ -37,14 +39,15 @@ namespace {
 
 constexpr int BM = 128, BN = 256, BK = 256;
 constexpr int BK_BYTES = BK / 2;                 // one 128-byte swizzle row per k-tile
-constexpr int STAGES = 3;
+constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK_BYTES;           // 16 KB
 constexpr int B_BYTES = BN * BK_BYTES;           // 32 KB
 constexpr int SFA_BYTES = 4 * 512;               // 4 k-atoms of one 128-row group
 constexpr int SFB_BYTES = 2 * 4 * 512;           // 2 row groups x 4 k-atoms
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
 constexpr int OFF_B = A_BYTES, OFF_SFA = A_BYTES + B_BYTES, OFF_SFB = OFF_SFA + SFA_BYTES;
-constexpr int EPI_BYTES = 8 * 32 * 33 * 4;      // per epilogue warp: a 32 x 32 fp32 tile (+1 pad)
+constexpr int EPI_WARPS = 8, EPI_PITCH = 9;      // per epilogue warp: a 32 x 8 fp32 chunk (+1 pad)
+constexpr int EPI_BYTES = EPI_WARPS * 32 * EPI_PITCH * 4;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;    // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(saddr(acc_full), 1);
     mbar_init(saddr(&sf_full[0]), 1);
     mbar_init(saddr(&sf_full[1]), 1);
-    mbar_init(saddr(acc_empty), 8);
+    mbar_init(saddr(acc_empty), EPI_WARPS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -207,60 +210,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
       if (!mbar_wait(saddr(acc_full), (uint32_t)(local & 1), abort_flag, p.st)) break;
       tc_fence_after();
-      // Each warp owns TMEM lanes (= tile rows) 32q..32q+31.  A 32 x 32 chunk is
-      // read row-per-thread, transposed through shared memory, and written with
-      // 16-byte stores in which 8 lanes cover one 128-byte row segment.
+      // Each warp owns TMEM lanes (= tile rows) 32q..32q+31 and columns
+      // [128 half, 128 half + 128): read them all, then free the accumulator.
       const int ew = warp - 3, half = ew / 4;
-      float* buf = epi + ew * 32 * 33;
-      const int sub_r = lane >> 3, sub_c = (lane & 7) * 4;
-      for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + c * 32, r);
-        tmem_ld_wait();
-        const int col0 = nb * BN + c * 32;
-        if (col0 >= p.N) continue;  // uniform across the warp
+      uint32_t r[BN / 64][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) buf[lane * 33 + i] = __uint_as_float(r[i]) * alpha;
-        __syncwarp();
-        if (p.y_vec && col0 + 32 <= p.N) {
-          // full 32-column chunk of an aligned Y: one 16-byte (fp32) or 8-byte
-          // (bf16) store per lane and row
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int lr = i * 4 + sub_r;
-            const int grow = mb * BM + q * 32 + lr;
-            if (grow < p.M) {
-              const float* src = buf + lr * 33 + sub_c;
-              const int64_t off = (int64_t)grow * p.ldy + col0 + sub_c;
-              if (BF16OUT)
-                *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.y) + off) =
-                    make_uint2(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]));
-              else
-                *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + off) =
-                    make_float4(src[0], src[1], src[2], src[3]);
-            }
-          }
-        } else {
-          // ragged last chunk or unaligned Y: element stores
-          for (int i = 0; i < 8; ++i) {
-            const int lr = i * 4 + sub_r;
-            const int grow = mb * BM + q * 32 + lr;
-            if (grow >= p.M) continue;
-            const float* src = buf + lr * 33 + sub_c;
-            const int64_t off = (int64_t)grow * p.ldy + col0 + sub_c;
-            for (int e = 0; e < 4 && col0 + sub_c + e < p.N; ++e) {
-              if (BF16OUT)
-                reinterpret_cast<__nv_bfloat16*>(p.y)[off + e] = __float2bfloat16_rn(src[e]);
-              else
-                reinterpret_cast<float*>(p.y)[off + e] = src[e];
-            }
-          }
-        }
-        __syncwarp();
-      }
+      for (int c = 0; c < BN / 64; ++c)
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + (half * (BN / 64) + c) * 32, r[c]);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(saddr(acc_empty));
+      // 32 x 8 chunks: lane = row while writing, then 2 lanes per 8-column row
+      // segment, 16 rows per store instruction
+      float* buf = epi + ew * 32 * EPI_PITCH;
+      const int sub_r = lane >> 1, sub_c = (lane & 1) * 4;
+#pragma unroll
+      for (int c = 0; c < BN / 64; ++c) {
+        const int col0 = nb * BN + (half * (BN / 64) + c) * 32;
+        if (col0 >= p.N) continue;  // uniform across the warp
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) buf[lane * EPI_PITCH + i] = __uint_as_float(r[c][g8 * 8 + i]) * alpha;
+          __syncwarp();
+          const int cg = col0 + g8 * 8;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int lr = h * 16 + sub_r;
+            const int grow = mb * BM + q * 32 + lr;
+            const float* src = buf + lr * EPI_PITCH + sub_c;
+            const int64_t off = (int64_t)grow * p.ldy + cg + sub_c;
+            if (grow < p.M) {
+              if (p.y_vec && cg + 8 <= p.N) {
+                if (BF16OUT)
+                  *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.y) + off) =
+                      make_uint2(pack_bf16x2(src[0], src[1]), pack_bf16x2(src[2], src[3]));
+                else
+                  *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + off) =
+                      make_float4(src[0], src[1], src[2], src[3]);
+              } else {
+                // ragged last chunk or unaligned Y: element stores
+                for (int e = 0; e < 4 && cg + sub_c + e < p.N; ++e) {
+                  if (BF16OUT)
+                    reinterpret_cast<__nv_bfloat16*>(p.y)[off + e] = __float2bfloat16_rn(src[e]);
+                  else
+                    reinterpret_cast<float*>(p.y)[off + e] = src[e];
+                }
+              }
+            }
+          }
+          __syncwarp();
+        }
+      }
     }
   }
 
@@ -302,6 +304,18 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
                                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_scales_map(CUtensorMap* map, const uint8_t* scales, int64_t groups, int64_t katoms, uint32_t box_groups) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)(katoms * 64), (cuuint64_t)groups};   // 8-byte units
+  const cuuint64_t strides[1] = {(cuuint64_t)(katoms * 512)};
+  const cuuint32_t box[2] = {(cuuint32_t)256, box_groups};                      // 4 atoms x box_groups
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(scales), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace tc
