@@ -8,24 +8,30 @@
 // compensation (ARCQuant blog post, section 3.1-3.2: one GEMM over the
 // augmented K) runs through this kernel unchanged.
 //
-// Structure (persistent, one CTA per SM, 352 threads):
-//   warp 0     one lane issues TMA loads of A/W code tiles (128 B K-slices,
-//              128-byte swizzle) and bulk copies of the matching scale atoms
-//              into a 4-stage shared-memory ring;
-//   warp 2     one lane copies each stage's scale atoms into TMEM
-//              (tcgen05.cp 32x128b.warpx4) into one of two alternating
-//              buffers, and signals the MMA issuer through tcgen05.commit;
-//   warp 1     allocates 512 TMEM columns; one lane issues the 4 MMAs (K = 64
-//              each) of a stage once its scales are in TMEM; tcgen05.commit
-//              frees the stage (and, two stages later, its scale buffer) and,
-//              at the end of a tile, signals the epilogue;
-//   warps 3-10 read the 128 x 256 fp32 accumulator into registers
-//              (tcgen05.ld 32x32b.x32; two warps per TMEM lane quadrant, 128
-//              columns each) and release it at once, so that the next tile's
-//              MMAs start while they scale by s_a s_w, transpose 32 x 8 chunks
-//              through shared memory and store Y with 16-byte stores, two
-//              lanes per 32-byte row segment.
-// Copies and MMAs come from two issuing threads so that they overlap.
+// Structure (persistent, one CTA per SM, 512 threads in four warpgroups with
+// a register split):
+//   warps 0-3  scale warps, one per TMEM lane quadrant (80 registers): for
+//              every stage, each lane reads line l of the stage's 12 scale
+//              atoms from shared memory and writes them with tcgen05.st into
+//              its quadrant of the stage's own TMEM scale buffer, which is
+//              the layout a 32x128b.warpx4 copy of the same atoms produces
+//              (the atom's 32 lines repeated in all four quadrants).  Scale
+//              copies issued to the tensor pipe (tcgen05.cp) would queue
+//              behind the in-flight TMA traffic; these stores do not.
+//   warp 4     one lane loads each stage (56 registers): the scale atoms
+//              first, on their own barrier, then the A/W code tiles (128 B
+//              K-slices, 128-byte swizzle) by TMA, into a 4-stage ring;
+//   warp 5     allocates 512 TMEM columns; one lane issues the 4 MMAs (K = 64
+//              each) of a stage once its codes have landed and all four
+//              quadrants of its scales are written; tcgen05.commit frees the
+//              stage and its scale buffer and, at the end of a tile, signals
+//              the epilogue;
+//   warps 8-15 read the 128 x 256 fp32 accumulator into registers (184
+//              each; tcgen05.ld 32x32b.x32, two warps per TMEM lane quadrant,
+//              128 columns each) and release it at once, so that the next
+//              tile's MMAs start while they scale by s_a s_w, transpose 32 x 8
+//              chunks through shared memory and store Y with 16-byte stores,
+//              two lanes per 32-byte row segment.
 // Tiles are 128 x 256 x 256 (M x N x K); tile order walks M fastest so that the
 // CTAs in flight share W tiles through L2.  Every mbarrier wait is bounded: on
 // timeout the kernel records NVFP4_ERR_TIMEOUT, every role leaves its loop, and
@@ -52,13 +58,19 @@ constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;    // + alignment slack
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;                  // 256 fp32 columns
-constexpr uint32_t SF_COL = 256;                 // two scale buffers of 48 columns, alternating by stage:
-constexpr uint32_t SF_BUF = 48;                  //   SFA 4 k-blocks x 4 columns, then SFB 4 k-blocks x 8
-constexpr int NUM_THREADS = 352;
-
+constexpr uint32_t SF_COL = 256, SF_BUF = 48;    // one scale buffer per stage: SFA 4 k-blocks x 4
+                                                 // columns, then SFB 4 k-blocks x 8
+constexpr int NUM_THREADS = 512;
+// Registers: the launch gives every thread 128 (the whole register file); the
+// scale and control warpgroups hand some back for the epilogue's accumulator.
+constexpr int LAUNCH_REGS = 65536 / NUM_THREADS;
+constexpr int SF_REGS = 80, CTL_REGS = 56, EPI_REGS = 184;
+static_assert(128 * SF_REGS + 128 * CTL_REGS + 256 * EPI_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for 128B swizzle");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert((2 * STAGES + 2) * 8 + 8 <= 128 && 128 + 2 * 8 <= BAR_BYTES, "barrier block: ring, accumulator, scale buffers");
+static_assert((4 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier block");
+static_assert(SF_COL % 4 == 0 && SF_BUF % 4 == 0 && SF_COL + STAGES * SF_BUF <= TMEM_COLS,
+              "block-scaled MMA scale operands start on 4-column TMEM boundaries");
 
 struct TcParams {
   const uint8_t* sfa;
@@ -85,28 +97,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* epi = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + EPI_BYTES);
-  uint64_t* full = bars;               // [STAGES] TMA -> MMA
-  uint64_t* empty = bars + STAGES;     // [STAGES] MMA -> TMA
-  uint64_t* acc_full = bars + 2 * STAGES;
-  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* full = bars;               // [STAGES] code tiles landed -> MMA
+  uint64_t* empty = bars + STAGES;     // [STAGES] MMAs done -> TMA (stage and its scale buffer free)
+  uint64_t* sf_land = bars + 2 * STAGES;   // [STAGES] scale atoms landed -> scale warps
+  uint64_t* sf_full = bars + 3 * STAGES;   // [STAGES] scales in TMEM, all four quadrants -> MMA
+  uint64_t* acc_full = bars + 4 * STAGES;
+  uint64_t* acc_empty = acc_full + 1;  // the epilogue holds the accumulator in registers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint64_t* sf_full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + EPI_BYTES + 128);   // [2] scales in TMEM
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(saddr(&full[s]), 1);
       mbar_init(saddr(&empty[s]), 1);
+      mbar_init(saddr(&sf_land[s]), 1);
+      mbar_init(saddr(&sf_full[s]), 4);
     }
     mbar_init(saddr(acc_full), 1);
-    mbar_init(saddr(&sf_full[0]), 1);
-    mbar_init(saddr(&sf_full[1]), 1);
     mbar_init(saddr(acc_empty), EPI_WARPS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
+  if (warp == 5) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)),
                  "r"(TMEM_COLS)
                  : "memory");
@@ -117,102 +130,113 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------ TMA producer
-    int s = 0;
-    uint32_t ph = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
-      const int ngroups = min(2, p.b_groups - nb * 2);
-      for (int kt = 0; kt < p.k_tiles; ++kt) {
-        if (!mbar_wait(saddr(&empty[s]), ph ^ 1u, abort_flag, p.st)) goto producer_done;
-        const int jmax = min(4, (p.K - kt * BK) / 64);
-        const uint32_t sf_bytes = (uint32_t)jmax * 512u;
-        const uint32_t bar = saddr(&full[s]);
-        uint8_t* st_base = smem + s * STAGE_BYTES;
-        mbar_expect_tx(bar, A_BYTES + B_BYTES + sf_bytes * (1 + ngroups));
-        tma_load_2d(saddr(st_base), &tmA, kt * BK_BYTES, mb * BM, bar);
-        tma_load_2d(saddr(st_base + OFF_B), &tmB, kt * BK_BYTES, nb * BN, bar);
-        bulk_load(saddr(st_base + OFF_SFA), p.sfa + ((size_t)mb * p.katoms + kt * 4) * 512, sf_bytes, bar);
-        for (int g = 0; g < ngroups; ++g)
-          bulk_load(saddr(st_base + OFF_SFB + g * 2048),
-                    p.sfb + ((size_t)(nb * 2 + g) * p.katoms + kt * 4) * 512, sf_bytes, bar);
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
-      }
-    }
-  producer_done:;
-  } else if (warp == 1 && lane == 0) {
-    // -------------------------------------------------------- MMA issuer
-    const uint32_t idesc = idesc_nvf4(BN);
-    uint32_t sf_flip = 0;
-    int s = 0;
-    uint32_t ph = 0;
-    int local = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
-      const int nb = tile / p.m_blocks;
-      const int ngroups = min(2, p.b_groups - nb * 2);
-      if (!mbar_wait(saddr(acc_empty), (uint32_t)(local & 1) ^ 1u, abort_flag, p.st)) break;
-      tc_fence_after();
-      for (int kt = 0; kt < p.k_tiles; ++kt) {
-        if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) goto mma_done;
+  if (warp < 4) {
+    regs_dec<SF_REGS>();
+    // ------------------------------------------- scale warps: quadrant `warp`, every stage
+    // TMEM scale buffer s was last read by the MMAs of the step STAGES earlier,
+    // which completed before this step's loads were issued.
+    const uint32_t quad = (uint32_t)(warp * 32) << 16;
+    int g = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+        const int s = g % STAGES;
+        // every lane waits; the warp goes on only if all saw the phase (the
+        // TMEM stores are warp-collective)
+        ok = __all_sync(0xFFFFFFFFu,
+                        mbar_wait_inline(saddr(&sf_land[s]), (uint32_t)((g / STAGES) & 1), abort_flag, p.st)) != 0;
+        if (!ok) break;
         tc_fence_after();
-        const int jmax = min(4, (p.K - kt * BK) / 64);
         const uint8_t* st_base = smem + s * STAGE_BYTES;
-        const uint32_t a0 = saddr(st_base), b0 = saddr(st_base + OFF_B);
-        const uint32_t buf = sf_flip & 1u;
-        const uint32_t sfa = SF_COL + buf * SF_BUF, sfb = sfa + 16u;
-        if (!mbar_wait(saddr(&sf_full[buf]), (sf_flip >> 1) & 1u, abort_flag, p.st)) goto mma_done;
-        tc_fence_after();
-        ++sf_flip;
-        for (int j = 0; j < jmax; ++j)
-          tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a0) + (uint64_t)(2 * j), desc_sw128(b0) + (uint64_t)(2 * j),
-                      idesc, tmem + sfa + 4 * j, tmem + sfb + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
-        tc_commit(saddr(&empty[s]));  // stage reusable once these MMAs have read it
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
-      }
-      tc_commit(saddr(acc_full));     // accumulator complete
-    }
-  mma_done:;
-  } else if (warp == 2 && lane == 0) {
-    // ----------------------------------------------------- scale copies (separate issuer)
-    int s = 0;
-    uint32_t ph = 0;
-    uint32_t gs = 0;   // global stage counter
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      const int nb = tile / p.m_blocks;
-      const int ngroups = min(2, p.b_groups - nb * 2);
-      for (int kt = 0; kt < p.k_tiles; ++kt, ++gs) {
-        if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) goto sf_done;
-        if (gs >= 2) {
-          const uint32_t g2 = gs - 2;
-          if (!mbar_wait(saddr(&empty[g2 % STAGES]), (g2 / STAGES) & 1u, abort_flag, p.st)) goto sf_done;
+        uint32_t ra[16], rb[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 va = *reinterpret_cast<const uint4*>(st_base + OFF_SFA + j * 512 + lane * 16);
+          const uint4 v0 = *reinterpret_cast<const uint4*>(st_base + OFF_SFB + j * 512 + lane * 16);
+          const uint4 v1 = *reinterpret_cast<const uint4*>(st_base + OFF_SFB + 2048 + j * 512 + lane * 16);
+          ra[4 * j] = va.x; ra[4 * j + 1] = va.y; ra[4 * j + 2] = va.z; ra[4 * j + 3] = va.w;
+          rb[8 * j] = v0.x; rb[8 * j + 1] = v0.y; rb[8 * j + 2] = v0.z; rb[8 * j + 3] = v0.w;
+          rb[8 * j + 4] = v1.x; rb[8 * j + 5] = v1.y; rb[8 * j + 6] = v1.z; rb[8 * j + 7] = v1.w;
         }
-        tc_fence_after();
-        const int jmax = min(4, (p.K - kt * BK) / 64);
-        const uint8_t* st_base = smem + s * STAGE_BYTES;
-        const uint32_t sfa = SF_COL + (gs & 1u) * SF_BUF, sfb = sfa + 16u;
-        for (int j = 0; j < jmax; ++j) {
-          tc_cp_scales(tmem + sfa + 4 * j, desc_sf_atom(saddr(st_base + OFF_SFA + j * 512)));
-          for (int g = 0; g < ngroups; ++g)
-            tc_cp_scales(tmem + sfb + 8 * j + 4 * g, desc_sf_atom(saddr(st_base + OFF_SFB + g * 2048 + j * 512)));
-        }
-        tc_commit(saddr(&sf_full[gs & 1u]));
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
+        const uint32_t buf = SF_COL + (uint32_t)s * SF_BUF;
+        tmem_st16(tmem + quad + buf, ra);
+        tmem_st32(tmem + quad + buf + 16u, rb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(saddr(&sf_full[s]));
       }
     }
-  sf_done:;
-  } else if (warp >= 3) {
+  } else if (warp < 8) {
+    regs_dec<CTL_REGS>();
+    if (warp == 4 && lane == 0) {
+      // ------------------------------------------------------ TMA producer
+      // the small scale atoms first, on their own barrier: their trip to TMEM
+      // overlaps the code tiles' flight
+      int g = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
+        const int ngroups = min(2, p.b_groups - nb * 2);
+        for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+          const int s = g % STAGES;
+          if (!mbar_wait_inline(saddr(&empty[s]), (uint32_t)((g / STAGES) & 1) ^ 1u, abort_flag, p.st)) goto producer_done;
+          const int jmax = min(4, (p.K - kt * BK) / 64);
+          const uint32_t sf_bytes = (uint32_t)jmax * 512u;
+          uint8_t* st_base = smem + s * STAGE_BYTES;
+          const uint32_t sbar = saddr(&sf_land[s]);
+          mbar_expect_tx(sbar, sf_bytes * (1 + ngroups));
+          bulk_load(saddr(st_base + OFF_SFA), p.sfa + ((size_t)mb * p.katoms + kt * 4) * 512, sf_bytes, sbar);
+          for (int gi = 0; gi < ngroups; ++gi)
+            bulk_load(saddr(st_base + OFF_SFB + gi * 2048), p.sfb + ((size_t)(nb * 2 + gi) * p.katoms + kt * 4) * 512,
+                      sf_bytes, sbar);
+          const uint32_t bar = saddr(&full[s]);
+          mbar_expect_tx(bar, A_BYTES + B_BYTES);
+          tma_load_2d(saddr(st_base), &tmA, kt * BK_BYTES, mb * BM, bar);
+          tma_load_2d(saddr(st_base + OFF_B), &tmB, kt * BK_BYTES, nb * BN, bar);
+        }
+      }
+    producer_done:;
+    } else if (warp == 5 && lane == 0) {
+      // -------------------------------------------------------- MMA issuer
+      const uint32_t idesc = idesc_nvf4(BN);
+      int g = 0, local = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
+        if (!mbar_wait_inline(saddr(acc_empty), (uint32_t)(local & 1) ^ 1u, abort_flag, p.st)) break;
+        tc_fence_after();
+        for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+          const int s = g % STAGES;
+          const uint32_t ph = (uint32_t)((g / STAGES) & 1);
+          if (!mbar_wait_inline(saddr(&sf_full[s]), ph, abort_flag, p.st)) goto mma_done;
+          if (!mbar_wait_inline(saddr(&full[s]), ph, abort_flag, p.st)) goto mma_done;
+          tc_fence_after();
+          const int jmax = min(4, (p.K - kt * BK) / 64);
+          const uint8_t* st_base = smem + s * STAGE_BYTES;
+          const uint64_t da = desc_sw128(saddr(st_base)), db = desc_sw128(saddr(st_base + OFF_B));
+          const uint32_t buf = SF_COL + (uint32_t)s * SF_BUF;
+          for (int j = 0; j < jmax; ++j)
+            tc_mma_nvf4(tmem + ACC_COL, da + (uint64_t)(2 * j), db + (uint64_t)(2 * j), idesc, tmem + buf + 4 * j,
+                        tmem + buf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+          tc_commit(saddr(&empty[s]));
+        }
+        tc_commit(saddr(acc_full));
+      }
+    mma_done:;
+    }
+  } else {
+    regs_inc<EPI_REGS>();
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const int ew = warp - 8, half = ew / 4;
+    float* buf = epi + ew * 32 * EPI_PITCH;
+    const int sub_r = lane >> 1, sub_c = (lane & 1) * 4;
     int local = 0;
     const float alpha = (*p.a_s) * (*p.w_s);
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
       const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
-      if (!mbar_wait(saddr(acc_full), (uint32_t)(local & 1), abort_flag, p.st)) break;
+      if (!mbar_wait_inline(saddr(acc_full), (uint32_t)(local & 1), abort_flag, p.st)) break;
       tc_fence_after();
       // Each warp owns TMEM lanes (= tile rows) 32q..32q+31 and columns
       // [128 half, 128 half + 128): read them all, then free the accumulator.
-      const int ew = warp - 3, half = ew / 4;
       uint32_t r[BN / 64][32];
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c)
@@ -223,8 +247,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(saddr(acc_empty));
       // 32 x 8 chunks: lane = row while writing, then 2 lanes per 8-column row
       // segment, 16 rows per store instruction
-      float* buf = epi + ew * 32 * EPI_PITCH;
-      const int sub_r = lane >> 1, sub_c = (lane & 1) * 4;
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) {
         const int col0 = nb * BN + (half * (BN / 64) + c) * 32;
@@ -266,10 +288,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
+  if (warp == 5) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   }
@@ -306,18 +328,6 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool encode_scales_map(CUtensorMap* map, const uint8_t* scales, int64_t groups, int64_t katoms, uint32_t box_groups) {
-  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
-  if (encode == nullptr) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)(katoms * 64), (cuuint64_t)groups};   // 8-byte units
-  const cuuint64_t strides[1] = {(cuuint64_t)(katoms * 512)};
-  const cuuint32_t box[2] = {(cuuint32_t)256, box_groups};                      // 4 atoms x box_groups
-  const cuuint32_t estr[2] = {1, 1};
-  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t*>(scales), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace tc
 
 cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) {
@@ -342,6 +352,9 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) 
   p.k_tiles = (int)((g.K + BK - 1) / BK);
   p.st = g.st;
   auto kern = g.y_bf16 ? k_gemm_nvf4<true> : k_gemm_nvf4<false>;
+  // the register split assumes the launch allocates LAUNCH_REGS per thread
+  cudaFuncAttributes fa{};
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != LAUNCH_REGS) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(p.num_tiles, num_sms));
