@@ -147,7 +147,8 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K,
     NVFP4_TRY(cuda_status(launch_amax(x, dt, M, K, ldx, ws, 0, q->tensor_scale, dev_status, sms, s)));
     s_ptr = q->tensor_scale;
   }
-  return cuda_status(launch_quant(Q_PLAIN, x, dt, M, K, ldx, s_ptr, nullptr, qo, qo, ws, dev_status, sms, s));
+  return cuda_status(launch_quant(Q_PLAIN, x, dt, M, K, ldx, s_ptr, nullptr, qo, qo, ws, dev_status, sms, s,
+                                  scale_in == nullptr));
 }
 
 nvfp4_status nvfp4_quantize_residue(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
@@ -170,8 +171,10 @@ nvfp4_status nvfp4_quantize_residue(const void* x, nvfp4_dtype dt, int64_t M, in
     s_ptr = q->tensor_scale;
   }
   if (rscale_in != nullptr)
-    return cuda_status(launch_quant(Q_BOTH, x, dt, M, K, ldx, s_ptr, rscale_in, qo, ro, ws, dev_status, sms, s));
-  NVFP4_TRY(cuda_status(launch_quant(Q_MAIN_AMAXR, x, dt, M, K, ldx, s_ptr, nullptr, qo, ro, ws, dev_status, sms, s)));
+    return cuda_status(launch_quant(Q_BOTH, x, dt, M, K, ldx, s_ptr, rscale_in, qo, ro, ws, dev_status, sms, s,
+                                    scale_in == nullptr));
+  NVFP4_TRY(cuda_status(launch_quant(Q_MAIN_AMAXR, x, dt, M, K, ldx, s_ptr, nullptr, qo, ro, ws, dev_status, sms,
+                                     s, scale_in == nullptr)));
   return cuda_status(launch_quant(Q_RES_ONLY, x, dt, M, K, ldx, s_ptr, r->tensor_scale, qo, ro, ws, dev_status, sms, s));
 }
 

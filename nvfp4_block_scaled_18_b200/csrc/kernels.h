@@ -26,9 +26,11 @@ enum QuantMode { Q_PLAIN = 0, Q_MAIN_AMAXR = 1, Q_RES_ONLY = 2, Q_BOTH = 3 };
 cudaError_t launch_amax(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                         WsHeader* ws, int slot, float* s_out, int* st, int num_sms,
                         cudaStream_t stream);
+// after_amax: launched as a programmatic dependent of the k_amax launch just
+// before it on the same stream (the quantizer overlaps that kernel's tail).
 cudaError_t launch_quant(int mode, const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                          const float* s_ptr, const float* sr_ptr, const QOut& q, const QOut& r,
-                         WsHeader* ws, int* st, int num_sms, cudaStream_t stream);
+                         WsHeader* ws, int* st, int num_sms, cudaStream_t stream, bool after_amax = false);
 cudaError_t launch_rms_stats(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                              const void* gamma, float eps, WsHeader* ws, float* rinv, float* s_out,
                              bool want_scale, int* st, int num_sms, cudaStream_t stream);

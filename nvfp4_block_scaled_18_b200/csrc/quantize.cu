@@ -54,50 +54,108 @@ __device__ void finish_tensor_scale(uint32_t key, unsigned int* amax_cell, unsig
   }
 }
 
+// Streaming passes: every thread issues kUnroll independent loads before it
+// consumes any, so that each SM keeps tens of KB in flight (what HBM needs);
+// a CTA covers kUnroll x 256 consecutive units per iteration.
+constexpr int kUnroll = 4;
+
+// |x| maximum.  Contiguous rows (ldx == K) are one flat array of 8-element
+// units; otherwise rows are grid-strided over blockIdx.y.
 template <typename T>
 __global__ void __launch_bounds__(256) k_amax(const T* __restrict__ x, int64_t M, int64_t K,
                                               int64_t ldx, WsHeader* ws, int slot, float* s_out,
                                               int* st) {
+  tc::griddep_launch_dependents();   // the quantizer may launch; it waits for this grid's result
   const int64_t upr = K >> 3;
   uint32_t key = 0;
-  for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
-    for (int64_t c8 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c8 < upr;
-         c8 += (int64_t)gridDim.x * blockDim.x) {
-      float v[8];
-      load8(x + row * ldx + c8 * 8, v);
+  if (ldx == K) {
+    const int64_t units = M * upr;
+    const int64_t cta = (int64_t)(blockIdx.y * gridDim.x + blockIdx.x), ctas = (int64_t)gridDim.x * gridDim.y;
+    for (int64_t base = cta * 256 * kUnroll; base < units; base += ctas * 256 * kUnroll) {
+      Raw8<T> raw[kUnroll];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * 256 + threadIdx.x;
+        if (i < units) raw[u].load(x + i * 8);
+        else raw[u].zero();
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        float v[8];
+        raw[u].get(v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
+      }
+    }
+  } else {
+    for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
+      for (int64_t c8 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c8 < upr;
+           c8 += (int64_t)gridDim.x * blockDim.x) {
+        float v[8];
+        load8(x + row * ldx + c8 * 8, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
+      }
     }
   }
   finish_tensor_scale(key, &ws->amax_bits[slot], &ws->arrive[slot], s_out, st);
 }
 
-// One thread per 16-element block (two 16-byte bf16 loads); a CTA covers up to
-// 256 consecutive blocks of a row, rows grid-strided over blockIdx.y.
+// One thread per 16-element block (two 16-byte bf16 loads), blocks numbered
+// row-major over the whole tensor (M * K/16 < 2^31); each iteration loads
+// kUnroll blocks per thread, then encodes them.  Launched as a programmatic dependent of the kernel that computes
+// the tensor scale (when there is one): it issues its first loads, then waits
+// for that grid before reading the scale.
 template <typename T, int MODE>
 __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t M, int64_t K,
                                                int64_t ldx, const float* s_ptr,
                                                const float* sr_ptr, QOut q, QOut r, WsHeader* ws,
                                                int* st) {
-  const int nb = (int)(K >> 4);
+  const uint32_t nb = (uint32_t)(K >> 4);
+  const int64_t nblk = M * nb;
+  const int64_t cta = (int64_t)(blockIdx.y * gridDim.x + blockIdx.x), ctas = (int64_t)gridDim.x * gridDim.y;
+  Raw8<T> raw[kUnroll][2];
+  auto load_blocks = [&](int64_t base) {
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t j = base + u * 256 + threadIdx.x;
+      if (j < nblk) {
+        const uint32_t row = (uint32_t)j / nb, b = (uint32_t)j - row * nb;
+        const T* p = x + (int64_t)row * ldx + (int64_t)b * 16;
+        raw[u][0].load(p);
+        raw[u][1].load(p + 8);
+      } else {
+        raw[u][0].zero();
+        raw[u][1].zero();
+      }
+    }
+  };
+  int64_t base = cta * 256 * kUnroll;
+  load_blocks(base);   // the input does not depend on the preceding kernel
+  tc::griddep_wait();
   const float s = *s_ptr;
   const float s_r = (MODE == Q_RES_ONLY || MODE == Q_BOTH) ? *sr_ptr : 0.0f;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     if (MODE != Q_RES_ONLY && q.s != s_ptr) *q.s = s;
     if (MODE == Q_BOTH && r.s != sr_ptr) *r.s = s_r;
   }
-  const int b = (int)(blockIdx.x * blockDim.x + threadIdx.x);
   uint32_t bad = 0, rkey = 0;
-  if (b < nb) {
-    for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
+  for (bool first = true; base < nblk; base += ctas * 256 * kUnroll, first = false) {
+    if (!first) load_blocks(base);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t j = base + u * 256 + threadIdx.x;
+      if (j >= nblk) break;
+      const uint32_t row = (uint32_t)j / nb, b = (uint32_t)j - row * nb;
       float v[16];
-      load16(x + row * ldx + (int64_t)b * 16, v);
+      raw[u][0].get(v);
+      raw[u][1].get(v + 8);
 #pragma unroll
       for (int i = 0; i < 16; ++i) bad = max(bad, abs_key(v[i]));
       uint32_t db;
       float deq[16];
       const uint64_t codes = quant_block16(v, s, db, MODE == Q_PLAIN ? nullptr : deq);
-      if (MODE != Q_RES_ONLY) store_block16(q, row, b, codes, db);
+      if (MODE != Q_RES_ONLY) store_block16(q, row, (int)b, codes, db);
       if (MODE != Q_PLAIN) {
         float rv[16];
 #pragma unroll
@@ -108,7 +166,7 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
         } else {
           uint32_t dr;
           const uint64_t rc = quant_block16(rv, s_r, dr, nullptr);
-          store_block16(r, row, b, rc, dr);
+          store_block16(r, row, (int)b, rc, dr);
         }
       }
     }
@@ -419,10 +477,16 @@ cudaError_t launch_quant_small(bool residue, const void* x, nvfp4_dtype dt, int6
                  : launch_quant_cluster_t<float, false>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
 }
 
-static inline dim3 quant_grid(int64_t M, int64_t K, int num_sms) {
+// k_amax grid: contiguous input runs flat over 8-element units (x only);
+// strided rows use (x) units of a row, (y) rows.
+static inline dim3 quant_grid(int64_t M, int64_t K, int64_t ldx, int num_sms) {
   const int64_t upr = K >> 3;
-  const int64_t gx = std::min<int64_t>((upr + 255) / 256, 65535);
   const int64_t target = (int64_t)num_sms * 8;
+  if (ldx == K) {
+    const int64_t per_cta = 256 * kUnroll;
+    return dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(target, (M * upr + per_cta - 1) / per_cta)));
+  }
+  const int64_t gx = std::min<int64_t>((upr + 255) / 256, 65535);
   const int64_t gy = std::max<int64_t>(1, std::min<int64_t>({M, 65535, (target + gx - 1) / gx}));
   return dim3((unsigned)gx, (unsigned)gy);
 }
@@ -430,7 +494,7 @@ static inline dim3 quant_grid(int64_t M, int64_t K, int num_sms) {
 template <typename T>
 cudaError_t launch_amax_t(const void* x, int64_t M, int64_t K, int64_t ldx, WsHeader* ws, int slot,
                           float* s_out, int* st, int num_sms, cudaStream_t stream) {
-  k_amax<T><<<quant_grid(M, K, num_sms), 256, 0, stream>>>(static_cast<const T*>(x), M, K, ldx, ws,
+  k_amax<T><<<quant_grid(M, K, ldx, num_sms), 256, 0, stream>>>(static_cast<const T*>(x), M, K, ldx, ws,
                                                            slot, s_out, st);
   return cudaGetLastError();
 }
@@ -443,35 +507,52 @@ cudaError_t launch_amax(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int
              : launch_amax_t<float>(x, M, K, ldx, ws, slot, s_out, st, num_sms, stream);
 }
 
-// k_quant grid: one thread per 16-element block, (x) blocks of a row, (y) rows.
+// k_quant grid: flat over 16-element blocks, up to 8 CTAs per SM.
 static inline dim3 quant_block_grid(int64_t M, int64_t K, int num_sms) {
-  const int64_t gx = std::min<int64_t>(((K >> 4) + 255) / 256, 65535);
-  const int64_t target = (int64_t)num_sms * 8;
-  const int64_t gy = std::max<int64_t>(1, std::min<int64_t>({M, 65535, (target + gx - 1) / gx}));
-  return dim3((unsigned)gx, (unsigned)gy);
+  const int64_t per_cta = 256 * kUnroll;
+  return dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>((int64_t)num_sms * 8, (M * (K >> 4) + per_cta - 1) / per_cta)));
+}
+
+template <typename T, int MODE>
+cudaError_t launch_quant_m(const void* x, int64_t M, int64_t K, int64_t ldx, const float* s_ptr,
+                           const float* sr_ptr, const QOut& q, const QOut& r, WsHeader* ws, int* st,
+                           int num_sms, cudaStream_t stream, bool after_amax) {
+  if (M * (K >> 4) >= ((int64_t)1 << 31)) return cudaErrorNotSupported;   // block numbers are 32-bit
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = quant_block_grid(M, K, num_sms);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_amax ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_quant<T, MODE>, static_cast<const T*>(x), M, K, ldx, s_ptr, sr_ptr, q, r, ws,
+                            st);
 }
 
 template <typename T>
 cudaError_t launch_quant_t(int mode, const void* x, int64_t M, int64_t K, int64_t ldx,
                            const float* s_ptr, const float* sr_ptr, const QOut& q, const QOut& r,
-                           WsHeader* ws, int* st, int num_sms, cudaStream_t stream) {
-  const dim3 g = quant_block_grid(M, K, num_sms);
-  const T* xp = static_cast<const T*>(x);
+                           WsHeader* ws, int* st, int num_sms, cudaStream_t stream, bool after_amax) {
   switch (mode) {
-    case Q_PLAIN: k_quant<T, Q_PLAIN><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
-    case Q_MAIN_AMAXR: k_quant<T, Q_MAIN_AMAXR><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
-    case Q_RES_ONLY: k_quant<T, Q_RES_ONLY><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
-    default: k_quant<T, Q_BOTH><<<g, 256, 0, stream>>>(xp, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st); break;
+    case Q_PLAIN:
+      return launch_quant_m<T, Q_PLAIN>(x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream, after_amax);
+    case Q_MAIN_AMAXR:
+      return launch_quant_m<T, Q_MAIN_AMAXR>(x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream, after_amax);
+    case Q_RES_ONLY:
+      return launch_quant_m<T, Q_RES_ONLY>(x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream, after_amax);
+    default:
+      return launch_quant_m<T, Q_BOTH>(x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream, after_amax);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_quant(int mode, const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                          const float* s_ptr, const float* sr_ptr, const QOut& q, const QOut& r,
-                         WsHeader* ws, int* st, int num_sms, cudaStream_t stream) {
+                         WsHeader* ws, int* st, int num_sms, cudaStream_t stream, bool after_amax) {
   return dt == NVFP4_BF16
-             ? launch_quant_t<__nv_bfloat16>(mode, x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream)
-             : launch_quant_t<float>(mode, x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream);
+             ? launch_quant_t<__nv_bfloat16>(mode, x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream, after_amax)
+             : launch_quant_t<float>(mode, x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream, after_amax);
 }
 
 template <typename T>
