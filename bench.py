@@ -621,7 +621,8 @@ def profile_case(case: str) -> int:
     """A handful of launches of one kernel, inputs just above L2, for ncu:
     decode   -- nvfp4_quantize_gemm, M=1, (N,K)=(4096,14336), 5 weight copies (147 MB)
     prefill  -- nvfp4_gemm, M=8192, (N,K)=(14336,4096) (A 19 MB, W 33 MB, Y 470 MB)
-    quantize -- nvfp4_quantize of the 8192x4096 bf16 prefill activations (67 MB)."""
+    quantize -- nvfp4_quantize of the 8192x4096 bf16 prefill activations (67 MB)
+    reorder  -- nvfp4_rmsnorm_reorder_quantize of the same activations, S=256."""
     import nvfp4_block_scaled_18_b200 as nv
     from nvfp4_block_scaled_18_b200 import workloads as wl
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -648,6 +649,14 @@ def profile_case(case: str) -> int:
         y = torch.empty((M, N), device=dev)
         for _ in range(3):
             nv.nvfp4_gemm(qa, qw, y)
+    elif case == "reorder":
+        M, K, S = 8192, 4096, 256
+        x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
+        perm = torch.from_numpy(wl.calibrated_perm(wl.prefill_x(64, K))).to(dev)
+        q = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED, device=dev)
+        ws = nv.Workspace(M, K, dev)
+        for _ in range(3):
+            nv.nvfp4_rmsnorm_reorder_quantize(x, q, perm=perm, S=S, workspace=ws)
     else:
         M, K = 8192, 4096
         x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
@@ -674,7 +683,7 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="decode: launch every step directly on the stream (no CUDA graphs) and skip the "
                          "per-call detail; for profilers that cannot follow graph replays")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize"],
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder"],
                     help="run a few launches of one kernel on a small case (for ncu captures) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

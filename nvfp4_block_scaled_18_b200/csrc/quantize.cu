@@ -299,8 +299,12 @@ __device__ __forceinline__ int ilog2_key(uint32_t key) {
 }
 
 // Pass 1, one CTA per row (grid-stride): rinv of the row and the running
-// maximum of |y| = |fl32(fl32(x * rinv) * gamma)| over the tensor.
-template <typename T>
+// maximum of |y| = |fl32(fl32(x * rinv) * gamma)| over the tensor.  The three
+// per-row reductions (|x| maximum for the exponent, the exact sum of squares,
+// the |y| maximum) all need the whole row: with NC > 0 each thread keeps its
+// NC 8-element units of the row in registers, so the row is read once; NC = 0
+// is the general form that re-reads the row (from L1/L2) for each reduction.
+template <typename T, int NC>
 __global__ void __launch_bounds__(256) k_rms_stats(const T* __restrict__ x, int64_t M, int64_t K,
                                                    int64_t ldx, const T* __restrict__ gamma,
                                                    float eps, WsHeader* ws, float* rinv_out,
@@ -309,14 +313,32 @@ __global__ void __launch_bounds__(256) k_rms_stats(const T* __restrict__ x, int6
   __shared__ double redd[32];
   const int64_t upr = K >> 3;
   uint32_t ykey = 0, bad = 0;
+  // unit c8 of the row: NC > 0 -> c8 = threadIdx.x + 256 n, n < NC
+  [[maybe_unused]] Raw8<T> rowv[NC > 0 ? NC : 1];
   for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
     const T* xr = x + row * ldx;
     uint32_t key = 0;
-    for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
-      float v[8];
-      load8(xr + c8 * 8, v);
+    if constexpr (NC > 0) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
+      for (int n = 0; n < NC; ++n) {
+        const int64_t c8 = threadIdx.x + 256 * n;
+        if (c8 < upr) rowv[n].load(xr + c8 * 8);
+        else rowv[n].zero();
+      }
+#pragma unroll
+      for (int n = 0; n < NC; ++n) {
+        float v[8];
+        rowv[n].get(v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
+      }
+    } else {
+      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+        float v[8];
+        load8(xr + c8 * 8, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
+      }
     }
     key = block_max_u32(key, redu);
     bad = max(bad, key);
@@ -325,13 +347,25 @@ __global__ void __launch_bounds__(256) k_rms_stats(const T* __restrict__ x, int6
     if (key != 0u && key < 0x7F800000u) {
       e = ilog2_key(key);
       const double c = pow2_f64(17 - e);  // z = x * 2^(17-e), |z| < 2^18
-      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
-        float v[8];
-        load8(xr + c8 * 8, v);
+      auto add_sq = [&](const float v[8]) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const double z = __dmul_rn((double)v[i], c);
           qsum = __dadd_rn(qsum, floor(__dmul_rn(z, z)));
+        }
+      };
+      if constexpr (NC > 0) {
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+          float v[8];
+          rowv[n].get(v);   // units past the row are zero and add nothing
+          add_sq(v);
+        }
+      } else {
+        for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+          float v[8];
+          load8(xr + c8 * 8, v);
+          add_sq(v);
         }
       }
     }
@@ -340,12 +374,28 @@ __global__ void __launch_bounds__(256) k_rms_stats(const T* __restrict__ x, int6
     const float rinv = __double2float_rn(__drcp_rn(__dsqrt_rn(__dadd_rn(mean, (double)eps))));
     if (threadIdx.x == 0) rinv_out[row] = rinv;
     if (want_scale) {
-      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
-        float v[8], g[8];
-        load8(xr + c8 * 8, v);
-        load8(gamma + c8 * 8, g);
+      auto max_y = [&](const float v[8], const float g[8]) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) ykey = max(ykey, abs_key(__fmul_rn(__fmul_rn(v[i], rinv), g[i])));
+      };
+      if constexpr (NC > 0) {
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+          const int64_t c8 = threadIdx.x + 256 * n;
+          if (c8 < upr) {
+            float v[8], g[8];
+            rowv[n].get(v);
+            load8(gamma + c8 * 8, g);
+            max_y(v, g);
+          }
+        }
+      } else {
+        for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+          float v[8], g[8];
+          load8(xr + c8 * 8, v);
+          load8(gamma + c8 * 8, g);
+          max_y(v, g);
+        }
       }
     }
   }
@@ -354,7 +404,15 @@ __global__ void __launch_bounds__(256) k_rms_stats(const T* __restrict__ x, int6
 }
 
 // Pass 2, persistent CTAs looping over rows.  Shared memory holds the channel
-// permutation (loaded once per CTA), gamma, and the current row of x.
+// permutation as 16-bit indices (K <= 65536) and gamma in its own type (both
+// loaded once per CTA), and two row buffers: the next row's load (cp.async)
+// is in flight while the current row is encoded.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tc::saddr(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, int64_t M,
                                                        int64_t K, int64_t ldx,
@@ -363,9 +421,18 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
                                                        const int32_t* __restrict__ perm, int64_t S,
                                                        const float* s_ptr, QOut q, int* st) {
   extern __shared__ __align__(16) unsigned char smem[];
-  int32_t* sperm = reinterpret_cast<int32_t*>(smem);
-  float* sgamma = reinterpret_cast<float*>(smem + K * 4);
-  T* srow = reinterpret_cast<T*>(smem + K * 4 + (gamma ? K * 4 : 0));
+  const int64_t row_bytes = K * (int64_t)sizeof(T);   // a multiple of 16 (K % 16 == 0)
+  T* srow0 = reinterpret_cast<T*>(smem);
+  T* srow1 = reinterpret_cast<T*>(smem + row_bytes);
+  uint16_t* sperm = reinterpret_cast<uint16_t*>(smem + 2 * row_bytes);
+  T* sgamma = reinterpret_cast<T*>(smem + 2 * row_bytes + ((K * 2 + 15) & ~int64_t(15)));
+  auto fetch_row = [&](int64_t row, T* dst) {
+    const T* xr = x + row * ldx;
+    for (int64_t c = threadIdx.x; c < row_bytes / 16; c += blockDim.x)
+      cp_async16(reinterpret_cast<uint4*>(dst) + c, reinterpret_cast<const uint4*>(xr) + c);
+    cp_async_commit();
+  };
+  if ((int64_t)blockIdx.x < M) fetch_row(blockIdx.x, srow0);   // overlaps the table set-up
   const float s = *s_ptr;
   if (blockIdx.x == 0 && threadIdx.x == 0 && q.s != s_ptr) *q.s = s;
   for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
@@ -374,32 +441,32 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
       report_status(st, NVFP4_ERR_INVALID_ARG);
       p = 0;
     }
-    sperm[k] = p;
-    if (gamma) sgamma[k] = load1(gamma + k);
+    sperm[k] = (uint16_t)p;
+    if (gamma) sgamma[k] = gamma[k];
   }
   const int nb = (int)(K >> 4);     // blocks of the reordered row
   const int nbr = (int)(S >> 4);    // residue blocks (the first S reordered columns)
   uint32_t bad = 0;
-  for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
-    __syncthreads();  // previous row fully consumed (and sperm/sgamma ready)
-    const T* xr = x + row * ldx;
-    for (int64_t c = threadIdx.x; c < (K * (int64_t)sizeof(T)) / 16; c += blockDim.x)
-      reinterpret_cast<uint4*>(srow)[c] = __ldg(reinterpret_cast<const uint4*>(xr) + c);
-    __syncthreads();
+  int buf = 0;
+  for (int64_t row = blockIdx.x; row < M; row += gridDim.x, buf ^= 1) {
+    const T* srow = buf ? srow1 : srow0;
+    cp_async_wait_all();
+    __syncthreads();   // this row landed; every thread is done with the other buffer
+    if (row + gridDim.x < M) fetch_row(row + gridDim.x, buf ? srow0 : srow1);
     const float ri = gamma ? rinv[row] : 1.0f;
     // one thread per 16-element block of the reordered row
     for (int b = threadIdx.x; b < nb; b += blockDim.x) {
       float v[16];
-      int32_t pv[16];
+      uint16_t pv[16];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)   // 16-byte reads of the cached permutation (no bank conflicts)
-        *reinterpret_cast<int4*>(pv + 4 * j) = reinterpret_cast<const int4*>(sperm)[b * 4 + j];
+      for (int j = 0; j < 2; ++j)   // 16-byte reads of the cached permutation
+        *reinterpret_cast<uint4*>(pv + 8 * j) = reinterpret_cast<const uint4*>(sperm)[b * 2 + j];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const int32_t p = pv[i];
+        const int p = pv[i];
         float y = load1(srow + p);
         bad = max(bad, abs_key(y));
-        if (gamma) y = __fmul_rn(__fmul_rn(y, ri), sgamma[p]);
+        if (gamma) y = __fmul_rn(__fmul_rn(y, ri), load1(sgamma + p));
         v[i] = y;
       }
       uint32_t db;
@@ -417,6 +484,7 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
       }
     }
   }
+  cp_async_wait_all();
   if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
 }
 
@@ -555,15 +623,26 @@ cudaError_t launch_quant(int mode, const void* x, nvfp4_dtype dt, int64_t M, int
              : launch_quant_t<float>(mode, x, M, K, ldx, s_ptr, sr_ptr, q, r, ws, st, num_sms, stream, after_amax);
 }
 
+template <typename T, int NC>
+cudaError_t launch_rms_stats_nc(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                                float eps, WsHeader* ws, float* rinv, float* s_out, bool want_scale,
+                                int* st, int num_sms, cudaStream_t stream) {
+  const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * 8));
+  k_rms_stats<T, NC><<<g, 256, 0, stream>>>(static_cast<const T*>(x), M, K, ldx, static_cast<const T*>(gamma),
+                                            eps, ws, rinv, s_out, want_scale, st);
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_rms_stats_t(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
                                float eps, WsHeader* ws, float* rinv, float* s_out, bool want_scale,
                                int* st, int num_sms, cudaStream_t stream) {
-  const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * 8));
-  k_rms_stats<T><<<g, 256, 0, stream>>>(static_cast<const T*>(x), M, K, ldx,
-                                        static_cast<const T*>(gamma), eps, ws, rinv, s_out,
-                                        want_scale, st);
-  return cudaGetLastError();
+  // 8-element units per thread when the row is held in registers (256 threads)
+  const int64_t units = ((K >> 3) + 255) / 256;
+  if (units <= 2) return launch_rms_stats_nc<T, 2>(x, M, K, ldx, gamma, eps, ws, rinv, s_out, want_scale, st, num_sms, stream);
+  if (units <= 4) return launch_rms_stats_nc<T, 4>(x, M, K, ldx, gamma, eps, ws, rinv, s_out, want_scale, st, num_sms, stream);
+  if (units <= 8) return launch_rms_stats_nc<T, 8>(x, M, K, ldx, gamma, eps, ws, rinv, s_out, want_scale, st, num_sms, stream);
+  return launch_rms_stats_nc<T, 0>(x, M, K, ldx, gamma, eps, ws, rinv, s_out, want_scale, st, num_sms, stream);
 }
 
 cudaError_t launch_rms_stats(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
@@ -575,7 +654,8 @@ cudaError_t launch_rms_stats(const void* x, nvfp4_dtype dt, int64_t M, int64_t K
 }
 
 size_t reorder_smem_bytes(nvfp4_dtype dt, int64_t K, bool has_gamma) {
-  return (size_t)K * 4 + (has_gamma ? (size_t)K * 4 : 0) + (size_t)K * (dt == NVFP4_BF16 ? 2 : 4);
+  const size_t es = dt == NVFP4_BF16 ? 2 : 4;
+  return 2 * (size_t)K * es + (((size_t)K * 2 + 15) & ~size_t(15)) + (has_gamma ? (size_t)K * es : 0);
 }
 
 template <typename T>
@@ -587,9 +667,8 @@ cudaError_t launch_reorder_quant_t(const void* x, int64_t M, int64_t K, int64_t 
   cudaError_t e = cudaFuncSetAttribute(k_reorder_quant<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  // rows are processed one at a time per CTA (load, barrier, encode): keep
   // several CTAs per SM so that rows overlap
-  const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (200 * 1024) / smem));
+  const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (220 * 1024) / (smem + 1024)));
   const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * per_sm));
   k_reorder_quant<T><<<g, 256, smem, stream>>>(static_cast<const T*>(x), M, K, ldx,
                                                static_cast<const T*>(gamma), rinv, perm, S, s_ptr,
