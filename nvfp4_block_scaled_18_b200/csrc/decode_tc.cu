@@ -22,16 +22,16 @@
 //
 // Activation scales sit in shared memory as the four 512-byte scale atoms of
 // each k-tile (TILED layout of row group 0: line n holds row n's 4 block
-// scales of that K=64 chunk), one tcgen05.cp per MMA.  The scale operands of a
-// block-scaled MMA must start on a 4-column TMEM boundary, so one copy cannot
-// serve several MMAs.
+// scales of that K=64 chunk).  The scale operands of a block-scaled MMA start
+// on a 4-column TMEM boundary: each K=64 MMA reads one atom's 4 columns.
 //
 // Grid: (ks, ceil(N/128)), cluster (ks, 1, 1), ks <= 8.  CTA rank r of a
 // cluster handles k-tiles [r*kt/ks, (r+1)*kt/ks).  Roles (256 threads): every
 // warp takes part in the activation quantization; warp 0 lane 0 streams W
-// tiles and scale atoms through a TMA ring; warp 2 lane 0 copies each stage's
-// scale atoms into TMEM (one buffer per stage) while warp 1 lane 0 issues the
-// MMAs of the previous stage; warps 0-3 drain the accumulators and push their partial rows
+// tiles and scale atoms through a TMA ring; warps 4-7 (one per TMEM lane
+// quadrant) write each stage's W and activation scale atoms into the stage's
+// TMEM scale buffer with tcgen05.st while warp 1 lane 0 issues the MMAs of the
+// previous stage; warps 0-3 drain the accumulators and push their partial rows
 // into a dedicated area of the owning CTA's shared memory (row r of the tile
 // belongs to rank floor(r*ks/128)); each owner sums its rows and writes Y.
 // Per-CTA maxima travel the same way: each CTA sends its maximum to every
@@ -89,6 +89,7 @@ constexpr int PART_ROWS = max_part_rows();   // 133 (ks = 7)
 // TMEM columns: acc [0,32) (X products in 0-15, R products in 16-31), then one
 // scale buffer per ring stage: W scales [+0,+16), X/R scales [+16,+32)
 constexpr uint32_t ACC = 0, ACC_R = 16, SF_COL = 32, SF_BUF = 32, SFX_OFF = 16, TMEM_COLS = 128;
+static_assert(SFX_OFF == 16 && SF_BUF >= 32, "one 32-column TMEM store writes a stage's W and X scales");
 static_assert(SF_COL % 4 == 0 && SF_BUF % 4 == 0 && SFX_OFF % 4 == 0,
               "block-scaled MMA scale operands start on 4-column TMEM boundaries");
 static_assert(SF_COL + STAGES * SF_BUF <= TMEM_COLS, "TMEM columns");
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
   uint64_t* x_full = acc_full + 1;
-  uint64_t* sf_full = x_full + 1;                                   // [STAGES] scales copied to TMEM
+  uint64_t* sf_full = x_full + 1;                                   // [STAGES] scales written to TMEM
   uint64_t* xbar = sf_full + STAGES;                                // [2] peers' |x|, |r| maxima arrived
   uint64_t* pbar = xbar + 2;                                        // peers' partial rows arrived
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(saddr(&full[s]), 1);
       mbar_init(saddr(&empty[s]), 1);
-      mbar_init(saddr(&sf_full[s]), 1);
+      mbar_init(saddr(&sf_full[s]), 4);   // one arrival per scale warp
     }
     mbar_init(saddr(acc_full), 1);
     mbar_init(saddr(x_full), 1);
@@ -383,24 +384,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_w(kt, s);
       if (++s == STAGES) { s = 0; ph ^= 1u; }
     }
-  } else if (warp == 2 && lane == 0) {
-    // ------------------------------------------------ scale copies (own issuer)
-    // Stage s's scales go to TMEM buffer s.  A stage is refilled only after the
-    // MMAs that read it (and its scale buffer) have completed, so waiting for
-    // the stage's data is enough before overwriting the buffer.
+  } else if (warp >= 4) {
+    // ------------------------------------------- scales into TMEM (tcgen05.st)
+    // Warp w writes TMEM lane quadrant w - 4 of stage s's scale buffer: line l
+    // of each W atom, then of the k-tile's activation atoms, in every lane l of
+    // the quadrant (the layout a 32x128b.warpx4 copy of the same atoms gives).
+    // Scale copies issued to the tensor pipe would queue behind the stream of
+    // W tiles; these stores do not.  A stage is refilled only after the MMAs
+    // that read it (and its scale buffer) have completed, so waiting for the
+    // stage's data is enough before overwriting the buffer.
+    const uint32_t quad = (uint32_t)((warp - 4) * 32) << 16;
     int s = 0;
     uint32_t ph = 0;
     for (int kt = kt0; kt < kt1; ++kt) {
-      if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) break;
+      // every lane waits; the warp goes on only if all saw the phase (the
+      // TMEM store is warp-collective)
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(saddr(&full[s]), ph, abort_flag, p.st))) break;
       tc_fence_after();
-      const int t = kt - kt0, jmax = w_chunks(kt);
+      const int t = kt - kt0;
       const uint8_t* sb = smem + s * WSTAGE;
-      const uint32_t sfw = SF_COL + (uint32_t)s * SF_BUF, sfx = sfw + SFX_OFF;
-      for (int j = 0; j < jmax; ++j) {
-        tc_cp_scales(tmem + sfw + 4 * j, desc_sf_atom(saddr(sb + W_TILE + j * 512)));
-        tc_cp_scales(tmem + sfx + 4 * j, desc_sf_atom(saddr(sfxp + t * SF_TILE + j * 512)));
+      uint32_t r[32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(sb + W_TILE + j * 512 + lane * 16);
+        const uint4 a = *reinterpret_cast<const uint4*>(sfxp + t * SF_TILE + j * 512 + lane * 16);
+        r[4 * j] = w.x; r[4 * j + 1] = w.y; r[4 * j + 2] = w.z; r[4 * j + 3] = w.w;
+        r[16 + 4 * j] = a.x; r[16 + 4 * j + 1] = a.y; r[16 + 4 * j + 2] = a.z; r[16 + 4 * j + 3] = a.w;
       }
-      tc_commit(saddr(&sf_full[s]));
+      tmem_st32(tmem + quad + SF_COL + (uint32_t)s * SF_BUF, r);   // W scales, then X (and R) scales
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(saddr(&sf_full[s]));
       if (++s == STAGES) { s = 0; ph ^= 1u; }
     }
   } else if (warp == 1 && lane == 0) {
