@@ -20,10 +20,13 @@
 // hand-off between the two kernels from every decode call.
 // Plain mode (nvfp4_gemm): X codes arrive by TMA, X scales are gathered.
 //
-// Activation scales sit in shared memory as the four 512-byte scale atoms of
-// each k-tile (TILED layout of row group 0: line n holds row n's 4 block
-// scales of that K=64 chunk).  The scale operands of a block-scaled MMA start
-// on a 4-column TMEM boundary: each K=64 MMA reads one atom's 4 columns.
+// Activation scales sit in shared memory compactly: per k-tile and K=64 chunk,
+// the 4 block scales of each of the 32 operand rows (X rows 0-15, R rows
+// 16-31).  In TMEM they take the layout of a scale atom (lane l, column c:
+// row 32c + l), with rows 32 and up absent (zero).  The scale operands of a
+// block-scaled MMA start on a 4-column TMEM boundary: each K=64 MMA reads one
+// atom's 4 columns.  With a residue, each CTA pushes s_x s_w acc_x + s_r s_w
+// acc_r per row, so partial rows travel once.
 //
 // Grid: (ks, ceil(N/128)), cluster (ks, 1, 1), ks <= 8.  CTA rank r of a
 // cluster handles k-tiles [r*kt/ks, (r+1)*kt/ks).  Roles (256 threads): every
@@ -72,7 +75,8 @@ constexpr int SFW_BYTES = 4 * 512;           // one scale atom per K=64 chunk
 constexpr int WSTAGE = W_TILE + SFW_BYTES;   // 18 KB, keeps 1024-byte alignment
 constexpr int STAGES = 2;
 constexpr int X_TILE = NP * 128;             // codes of one operand (X or R) in one k-tile (SW128)
-constexpr int SF_TILE = 4 * 512;             // scale atoms of one k-tile (lines 0-15 X, 16-31 R)
+constexpr int SF_TILE = 4 * 128;             // activation scales of one k-tile: 4 K=64 chunks x 32 rows
+                                             // (rows 0-15 X, 16-31 R) x 4 block scales
 __host__ __device__ constexpr int b_tile(bool res) { return X_TILE * (res ? 2 : 1); }   // MMA B tile
 constexpr int BAR_BYTES = 256;
 constexpr int PITCH = NP;                    // floats per partial row (16-byte aligned rows)
@@ -97,7 +101,9 @@ constexpr int TMEM_CTAS = 512 / TMEM_COLS;
 
 static_assert(WSTAGE % 1024 == 0 && X_TILE % 1024 == 0, "SW128 tiles need 1024-byte alignment");
 static_assert(PART_ROWS == 133, "slot count for ks <= 8");
-__host__ __device__ constexpr int part_bytes(bool res) { return PART_ROWS * PITCH * 4 * (res ? 2 : 1); }
+// one pushed vector per row: the partial X product, or with a residue the
+// already scaled sum s_x s_w acc_x + s_r s_w acc_r
+constexpr int PART_BYTES = PART_ROWS * PITCH * 4;
 static_assert((3 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier block");
 
 struct DecodeParams {
@@ -127,7 +133,7 @@ struct DecodeParams {
 __device__ __forceinline__ int div_magic(int u, uint32_t m) { return (int)__umulhi((uint32_t)u, m); }
 
 __host__ __device__ constexpr int smem_bytes(int kt_max, bool res) {
-  return 1024 + STAGES * WSTAGE + kt_max * (b_tile(res) + SF_TILE) + part_bytes(res) + BAR_BYTES;
+  return 1024 + STAGES * WSTAGE + kt_max * (b_tile(res) + SF_TILE) + PART_BYTES + BAR_BYTES;
 }
 
 template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
@@ -140,10 +146,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* xcodes = smem + STAGES * WSTAGE;                         // KT x 2 KB
   constexpr int BT = b_tile(RES);                                   // B tile bytes per k-tile
   uint8_t* rcodes = xcodes + X_TILE;                                // R rows 16-31 of each B tile
-  uint8_t* sfxp = xcodes + KT * BT;                                 // KT x 2 KB scale atoms
-  uint8_t* sfrp = sfxp + NP * 16;                                   // R scales: atom lines 16-31
+  uint8_t* sfxp = xcodes + KT * BT;                                 // KT x 512 B activation scales
+  uint8_t* sfrp = sfxp + NP * 4;                                    // R scales: rows 16-31
   float* part = reinterpret_cast<float*>(sfxp + KT * SF_TILE);      // pushed partial rows
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(part) + part_bytes(RES));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(part) + PART_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
@@ -180,11 +186,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) mbar_init(saddr(&xbar[i]), 1);
     mbar_init(saddr(pbar), 1);
     // Arm the receive barriers with every byte the peers will send: one word
-    // per exchanged maximum, and 16 (X) or 32 (X and R) floats per owned row.
+    // per exchanged maximum, and 16 floats per owned row.
     if (x_exchange) mbar_expect_tx(saddr(&xbar[0]), (ks - 1u) * 4u);
     if (r_exchange) mbar_expect_tx(saddr(&xbar[1]), (ks - 1u) * 4u);
     const uint32_t owned = (uint32_t)(owner_row0(rank + 1) - owner_row0(rank));
-    mbar_expect_tx(saddr(pbar), (ks - 1u) * owned * (uint32_t)(NP * 4 * (RES ? 2 : 1)));
+    mbar_expect_tx(saddr(pbar), (ks - 1u) * owned * (uint32_t)(NP * 4));
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -288,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else if (n < p.M)
           word = *reinterpret_cast<const uint32_t*>(src + (size_t)n * nblk + chunk * 4);
       }
-      *reinterpret_cast<uint32_t*>((which ? sfrp : sfxp) + t * SF_TILE + j * 512 + n * 16) = word;   // R: lines 16-31
+      *reinterpret_cast<uint32_t*>((which ? sfrp : sfxp) + t * SF_TILE + j * 128 + n * 4) = word;   // R: rows 16-31
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   } else {
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<uint32_t*>(codes_area + t * BT + row * 128 + ((chunk16 ^ (row & 7)) << 4) +
                                    ((kk & 31) >> 1)) = codes;
       const int bt = kk >> 4;                              // 16-block within the k-tile
-      if ((c8 & 1) == 0) sf_area[t * SF_TILE + (bt >> 2) * 512 + row * 16 + (bt & 3)] = (uint8_t)db;
+      if ((c8 & 1) == 0) sf_area[t * SF_TILE + (bt >> 2) * 128 + row * 4 + (bt & 3)] = (uint8_t)db;
       if (writer) store_half_block(qo, row, (c0 >> 3) + c8, codes, db);
     };
 
@@ -407,9 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const uint4 w = *reinterpret_cast<const uint4*>(sb + W_TILE + j * 512 + lane * 16);
-        const uint4 a = *reinterpret_cast<const uint4*>(sfxp + t * SF_TILE + j * 512 + lane * 16);
         r[4 * j] = w.x; r[4 * j + 1] = w.y; r[4 * j + 2] = w.z; r[4 * j + 3] = w.w;
-        r[16 + 4 * j] = a.x; r[16 + 4 * j + 1] = a.y; r[16 + 4 * j + 2] = a.z; r[16 + 4 * j + 3] = a.w;
+        // activation rows are 0-31 only: line l carries row l's 4 scales
+        r[16 + 4 * j] = *reinterpret_cast<const uint32_t*>(sfxp + t * SF_TILE + j * 128 + lane * 4);
+        r[16 + 4 * j + 1] = 0u; r[16 + 4 * j + 2] = 0u; r[16 + 4 * j + 3] = 0u;
       }
       tmem_st32(tmem + quad + SF_COL + (uint32_t)s * SF_BUF, r);   // W scales, then X (and R) scales
       tmem_st_wait();
@@ -461,26 +468,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t dst = mapa_shared(saddr(part + slot * PITCH), o);
     const uint32_t dst_bar = mapa_shared(saddr(pbar), o);
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-    for (int acc_i = 0; acc_i < (RES ? 2 : 1); ++acc_i) {
-      uint32_t v[16];
-      tmem_ld16(lane_addr + (acc_i ? ACC_R : ACC), v);
+    uint32_t v[16];
+    tmem_ld16(lane_addr + ACC, v);
+    if constexpr (RES) {
+      // combine X and R products here: each row travels once, already scaled
+      uint32_t vr[16];
+      tmem_ld16(lane_addr + ACC_R, vr);
       tmem_ld_wait();
-      if (!ok) {
+      const float ws = *p.w_s;
+      const float alpha = __fmul_rn(sx, ws), alpha_r = __fmul_rn(sr, ws);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = 0u;
-      }
-      const int off = acc_i * PART_ROWS * PITCH;
-      if (local) {
+      for (int i = 0; i < 16; ++i)
+        v[i] = __float_as_uint(__fmaf_rn(__uint_as_float(v[i]), alpha, __fmul_rn(__uint_as_float(vr[i]), alpha_r)));
+    } else {
+      tmem_ld_wait();
+    }
+    if (!ok) {
 #pragma unroll
-        for (int i = 0; i < 16; i += 4)
-          *reinterpret_cast<uint4*>(part + slot * PITCH + off + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-      } else {
+      for (int i = 0; i < 16; ++i) v[i] = 0u;
+    }
+    if (local) {
 #pragma unroll
-        for (int i = 0; i < 16; i += 4)
-          st_async_f32x4(dst + (uint32_t)((off + i) * 4), __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                         __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]), dst_bar);
-      }
+      for (int i = 0; i < 16; i += 4)
+        *reinterpret_cast<uint4*>(part + slot * PITCH + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; i += 4)
+        st_async_f32x4(dst + (uint32_t)(i * 4), __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                       __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]), dst_bar);
     }
   }
   tc_fence_before();
@@ -493,19 +508,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   {
     const int r0 = owner_row0(rank), r1 = owner_row0(rank + 1);
     const int nrows = r1 - r0;
-    const float ws = *p.w_s;
-    const float alpha = sx * ws, alpha_r = RES ? sr * ws : 0.0f;
+    const float alpha = __fmul_rn(sx, *p.w_s);
     for (int idx = threadIdx.x; idx < nrows * p.M; idx += kThreads) {
       const int m = idx / nrows, i = idx - m * nrows;
       const int n = rt * 128 + r0 + i;
       if (n >= p.N) continue;
-      float sum = 0.0f, sum_r = 0.0f;
-      for (uint32_t src = 0; src < ks; ++src) {
-        const int slot = (int)src * rows_max + i;
-        sum += part[slot * PITCH + m];
-        if (RES) sum_r += part[PART_ROWS * PITCH + slot * PITCH + m];
-      }
-      const float out = RES ? fmaf(sum, alpha, sum_r * alpha_r) : sum * alpha;
+      float sum = 0.0f;
+      for (uint32_t src = 0; src < ks; ++src) sum += part[((int)src * rows_max + i) * PITCH + m];
+      const float out = RES ? sum : sum * alpha;   // residue partials arrive scaled
       if (BF16OUT)
         reinterpret_cast<__nv_bfloat16*>(p.y)[(int64_t)m * p.ldy + n] = __float2bfloat16_rn(out);
       else
