@@ -77,9 +77,14 @@ constexpr int STAGES = 2;
 constexpr int X_TILE = NP * 128;             // codes of one operand (X or R) in one k-tile (SW128)
 constexpr int SF_TILE = 4 * 128;             // activation scales of one k-tile: 4 K=64 chunks x 32 rows
                                              // (rows 0-15 X, 16-31 R) x 4 block scales
-__host__ __device__ constexpr int b_tile(bool res) { return X_TILE * (res ? 2 : 1); }   // MMA B tile
+// Residue row offset `ro`: 0 without a residue; otherwise R's rows start at
+// operand row ro (8: X rows 0-7 and R rows 8-15 share one 16-row operand when
+// M <= 8; 16: X rows 0-15, R rows 16-31).
+__host__ __device__ constexpr int b_tile(int ro) { return ro == 16 ? 2 * X_TILE : X_TILE; }   // MMA B tile
+__host__ __device__ constexpr int operand_rows(int ro) { return ro ? ro : NP; }   // rows per operand (X, R)
 constexpr int BAR_BYTES = 256;
-constexpr int PITCH = NP;                    // floats per partial row (16-byte aligned rows)
+// floats per pushed partial row: M rounded up to 4 (16-byte rows)
+__host__ __device__ constexpr int part_pitch(int M) { return (M + 3) & ~3; }
 constexpr int MAX_KS = 8;   // portable cluster size: larger clusters wait for free slots inside one GPC
 
 // Partial-row slots an owner holds: one slot of ceil(128/ks) rows per source
@@ -92,7 +97,7 @@ constexpr int max_part_rows() {
 constexpr int PART_ROWS = max_part_rows();   // 133 (ks = 7)
 // TMEM columns: acc [0,32) (X products in 0-15, R products in 16-31), then one
 // scale buffer per ring stage: W scales [+0,+16), X/R scales [+16,+32)
-constexpr uint32_t ACC = 0, ACC_R = 16, SF_COL = 32, SF_BUF = 32, SFX_OFF = 16, TMEM_COLS = 128;
+constexpr uint32_t ACC = 0, SF_COL = 32, SF_BUF = 32, SFX_OFF = 16, TMEM_COLS = 128;   // R products: column ro
 static_assert(SFX_OFF == 16 && SF_BUF >= 32, "one 32-column TMEM store writes a stage's W and X scales");
 static_assert(SF_COL % 4 == 0 && SF_BUF % 4 == 0 && SFX_OFF % 4 == 0,
               "block-scaled MMA scale operands start on 4-column TMEM boundaries");
@@ -103,7 +108,7 @@ static_assert(WSTAGE % 1024 == 0 && X_TILE % 1024 == 0, "SW128 tiles need 1024-b
 static_assert(PART_ROWS == 133, "slot count for ks <= 8");
 // one pushed vector per row: the partial X product, or with a residue the
 // already scaled sum s_x s_w acc_x + s_r s_w acc_r
-constexpr int PART_BYTES = PART_ROWS * PITCH * 4;
+__host__ __device__ constexpr int part_bytes(int M) { return PART_ROWS * part_pitch(M) * 4; }
 static_assert((3 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier block");
 
 struct DecodeParams {
@@ -132,11 +137,11 @@ struct DecodeParams {
 // stays below 1/d, so the quotient is exact.
 __device__ __forceinline__ int div_magic(int u, uint32_t m) { return (int)__umulhi((uint32_t)u, m); }
 
-__host__ __device__ constexpr int smem_bytes(int kt_max, bool res) {
-  return 1024 + STAGES * WSTAGE + kt_max * (b_tile(res) + SF_TILE) + PART_BYTES + BAR_BYTES;
+__host__ __device__ constexpr int smem_bytes(int kt_max, int ro, int M) {
+  return 1024 + STAGES * WSTAGE + kt_max * (b_tile(ro) + SF_TILE) + part_bytes(M) + BAR_BYTES;
 }
 
-template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
+template <typename T, bool FUSED, int RES, bool BF16OUT, int R>
 __global__ void __launch_bounds__(kThreads, 1)
     k_decode_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                 const __grid_constant__ CUtensorMap tmR, const DecodeParams p) {
@@ -145,11 +150,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int KT = p.kt_max;
   uint8_t* xcodes = smem + STAGES * WSTAGE;                         // KT x 2 KB
   constexpr int BT = b_tile(RES);                                   // B tile bytes per k-tile
-  uint8_t* rcodes = xcodes + X_TILE;                                // R rows 16-31 of each B tile
+  constexpr int OPR = operand_rows(RES);                            // rows of X (and of R)
+  uint8_t* rcodes = xcodes + RES * 128;                             // R rows of each B tile
   uint8_t* sfxp = xcodes + KT * BT;                                 // KT x 512 B activation scales
-  uint8_t* sfrp = sfxp + NP * 4;                                    // R scales: rows 16-31
+  uint8_t* sfrp = sfxp + RES * 4;                                   // R scales: rows RES..
+  const int pitch = part_pitch(p.M);
   float* part = reinterpret_cast<float*>(sfxp + KT * SF_TILE);      // pushed partial rows
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(part) + PART_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(part) + part_bytes(p.M));
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* acc_full = bars + 2 * STAGES;
@@ -186,11 +193,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) mbar_init(saddr(&xbar[i]), 1);
     mbar_init(saddr(pbar), 1);
     // Arm the receive barriers with every byte the peers will send: one word
-    // per exchanged maximum, and 16 floats per owned row.
+    // per exchanged maximum, and `pitch` floats per owned row.
     if (x_exchange) mbar_expect_tx(saddr(&xbar[0]), (ks - 1u) * 4u);
     if (r_exchange) mbar_expect_tx(saddr(&xbar[1]), (ks - 1u) * 4u);
     const uint32_t owned = (uint32_t)(owner_row0(rank + 1) - owner_row0(rank));
-    mbar_expect_tx(saddr(pbar), (ks - 1u) * owned * (uint32_t)(NP * 4));
+    mbar_expect_tx(saddr(pbar), (ks - 1u) * owned * (uint32_t)(pitch * 4));
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -281,10 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- gather the activation scales into atoms: line n of atom j of k-tile t
     // starts with the 4 block scales of row n in K chunk 4(kt0+t)+j
     const int nblk = p.K >> 4;
-    for (int idx = threadIdx.x; idx < nkt * NP * 4 * (RES ? 2 : 1); idx += kThreads) {
-      const int which = idx / (nkt * NP * 4);
-      const int e = idx - which * (nkt * NP * 4);
-      const int t = e / (NP * 4), n = (e >> 2) & (NP - 1), j = e & 3;
+    for (int idx = threadIdx.x; idx < nkt * OPR * 4 * (RES ? 2 : 1); idx += kThreads) {
+      const int which = idx / (nkt * OPR * 4);
+      const int e = idx - which * (nkt * OPR * 4);
+      const int t = e / (OPR * 4), n = (e >> 2) & (OPR - 1), j = e & 3;
       const int chunk = 4 * (kt0 + t) + j;
       const uint8_t* src = which ? p.sfr : p.sfx;
       uint32_t word = 0u;
@@ -294,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else if (n < p.M)
           word = *reinterpret_cast<const uint32_t*>(src + (size_t)n * nblk + chunk * 4);
       }
-      *reinterpret_cast<uint32_t*>((which ? sfrp : sfxp) + t * SF_TILE + j * 128 + n * 4) = word;   // R: rows 16-31
+      *reinterpret_cast<uint32_t*>((which ? sfrp : sfxp) + t * SF_TILE + j * 128 + n * 4) = word;   // R: rows RES..
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   } else {
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------- MMA issuer
     bool ok = true;
     if (!FUSED) ok = mbar_wait(saddr(x_full), 0u, abort_flag, p.st);
-    const uint32_t idesc = idesc_nvf4(RES ? 2 * NP : NP);
+    const uint32_t idesc = idesc_nvf4(RES == 16 ? 2 * NP : NP);
     int s = 0;
     uint32_t ph = 0;
     for (int kt = kt0; ok && kt < kt1; ++kt) {
@@ -465,20 +472,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o = (uint32_t)row * ks / 128u;
     const int slot = (int)rank * rows_max + (row - owner_row0(o));
     const bool local = o == rank;
-    const uint32_t dst = mapa_shared(saddr(part + slot * PITCH), o);
+    const uint32_t dst = mapa_shared(saddr(part + slot * pitch), o);
     const uint32_t dst_bar = mapa_shared(saddr(pbar), o);
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     uint32_t v[16];
     tmem_ld16(lane_addr + ACC, v);
-    if constexpr (RES) {
+    if constexpr (RES != 0) {
       // combine X and R products here: each row travels once, already scaled
       uint32_t vr[16];
-      tmem_ld16(lane_addr + ACC_R, vr);
-      tmem_ld_wait();
+      if constexpr (RES == 16) {
+        tmem_ld16(lane_addr + ACC + 16, vr);
+        tmem_ld_wait();
+      } else {   // R products in columns 8-15 of the same load
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vr[i] = v[8 + i];
+      }
       const float ws = *p.w_s;
       const float alpha = __fmul_rn(sx, ws), alpha_r = __fmul_rn(sr, ws);
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
+      for (int i = 0; i < RES; ++i)
         v[i] = __float_as_uint(__fmaf_rn(__uint_as_float(v[i]), alpha, __fmul_rn(__uint_as_float(vr[i]), alpha_r)));
     } else {
       tmem_ld_wait();
@@ -487,15 +500,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = 0u;
     }
+    // the first `pitch` (>= M) products of the row
     if (local) {
 #pragma unroll
       for (int i = 0; i < 16; i += 4)
-        *reinterpret_cast<uint4*>(part + slot * PITCH + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        if (i < pitch)
+          *reinterpret_cast<uint4*>(part + slot * pitch + i) = make_uint4(v[i], v[i + 1], v[i + 2], v[i + 3]);
     } else {
 #pragma unroll
       for (int i = 0; i < 16; i += 4)
-        st_async_f32x4(dst + (uint32_t)(i * 4), __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
-                       __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]), dst_bar);
+        if (i < pitch)
+          st_async_f32x4(dst + (uint32_t)(i * 4), __uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                         __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]), dst_bar);
     }
   }
   tc_fence_before();
@@ -514,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n = rt * 128 + r0 + i;
       if (n >= p.N) continue;
       float sum = 0.0f;
-      for (uint32_t src = 0; src < ks; ++src) sum += part[((int)src * rows_max + i) * PITCH + m];
+      for (uint32_t src = 0; src < ks; ++src) sum += part[((int)src * rows_max + i) * pitch + m];
       const float out = RES ? sum : sum * alpha;   // residue partials arrive scaled
       if (BF16OUT)
         reinterpret_cast<__nv_bfloat16*>(p.y)[(int64_t)m * p.ldy + n] = __float2bfloat16_rn(out);
@@ -549,11 +565,12 @@ struct Choice {
 // their k-tiles and, fused (units_cap > 0), the cluster-wide maxima and the
 // encoding of the CTA's activation slice (every unit of which must fit in
 // units_cap registers arrays per thread).  The smaller split wins ties.
-Choice choose_split(int row_tiles, int k_tiles, bool res, int num_sms, int regs, int M, int K, int units_cap) {
+Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, int M, int K, int units_cap) {
+  const bool res = ro != 0;
   Choice best;
   for (int ks = 1; ks <= std::min(MAX_KS, k_tiles); ++ks) {
     const int kt_max = (k_tiles + ks - 1) / ks;
-    const int smem = smem_bytes(kt_max, res);
+    const int smem = smem_bytes(kt_max, ro, M);
     if (smem > 232448) continue;
     const int slice = std::min(kt_max * 256, K);
     const int64_t units = (int64_t)M * (slice / 8);
@@ -575,7 +592,7 @@ Choice choose_split(int row_tiles, int k_tiles, bool res, int num_sms, int regs,
   return best;
 }
 
-template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
+template <typename T, bool FUSED, int RES, bool BF16OUT, int R>
 int regs_of() {
   static int regs = -1;
   if (regs < 0) {
@@ -585,7 +602,7 @@ int regs_of() {
   return regs;
 }
 
-template <typename T, bool FUSED, bool RES, bool BF16OUT, int R>
+template <typename T, bool FUSED, int RES, bool BF16OUT, int R>
 cudaError_t launch_cfg(const DecodeArgs& a, DecodeParams p, const Choice& c, const CUtensorMap& tmW,
                        const CUtensorMap& tmX, const CUtensorMap& tmR, cudaStream_t stream) {
   if (a.dry_run) return cudaSuccess;
@@ -615,7 +632,7 @@ cudaError_t launch_cfg(const DecodeArgs& a, DecodeParams p, const Choice& c, con
   return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, tmR, p);
 }
 
-template <typename T, bool FUSED, bool RES, bool BF16OUT>
+template <typename T, bool FUSED, int RES, bool BF16OUT>
 cudaError_t launch_r(const DecodeArgs& a, const DecodeParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
                      const CUtensorMap& tmR, int num_sms, cudaStream_t stream) {
   const int row_tiles = (int)((a.N + 127) / 128);
@@ -648,15 +665,24 @@ cudaError_t launch_r(const DecodeArgs& a, const DecodeParams& p, const CUtensorM
   }
 }
 
+// residue row offset for this call (see b_tile)
+int residue_rows(const DecodeArgs& a) {
+  if (a.r_codes == nullptr && a.r_out.codes == nullptr) return 0;
+  return a.M <= 8 ? 8 : 16;
+}
+
 template <typename T, bool FUSED>
 cudaError_t launch_t(const DecodeArgs& a, const DecodeParams& p, const CUtensorMap& tmW, const CUtensorMap& tmX,
                      const CUtensorMap& tmR, int num_sms, cudaStream_t stream) {
-  const bool res = a.r_codes != nullptr || a.r_out.codes != nullptr;
-  if (res)
-    return a.y_bf16 ? launch_r<T, FUSED, true, true>(a, p, tmW, tmX, tmR, num_sms, stream)
-                    : launch_r<T, FUSED, true, false>(a, p, tmW, tmX, tmR, num_sms, stream);
-  return a.y_bf16 ? launch_r<T, FUSED, false, true>(a, p, tmW, tmX, tmR, num_sms, stream)
-                  : launch_r<T, FUSED, false, false>(a, p, tmW, tmX, tmR, num_sms, stream);
+  const int ro = residue_rows(a);
+  if (ro == 8)
+    return a.y_bf16 ? launch_r<T, FUSED, 8, true>(a, p, tmW, tmX, tmR, num_sms, stream)
+                    : launch_r<T, FUSED, 8, false>(a, p, tmW, tmX, tmR, num_sms, stream);
+  if (ro == 16)
+    return a.y_bf16 ? launch_r<T, FUSED, 16, true>(a, p, tmW, tmX, tmR, num_sms, stream)
+                    : launch_r<T, FUSED, 16, false>(a, p, tmW, tmX, tmR, num_sms, stream);
+  return a.y_bf16 ? launch_r<T, FUSED, 0, true>(a, p, tmW, tmX, tmR, num_sms, stream)
+                  : launch_r<T, FUSED, 0, false>(a, p, tmW, tmX, tmR, num_sms, stream);
 }
 
 }  // namespace
@@ -674,9 +700,10 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
   if (a.dry_run) {
     // configuration only
   } else if (!fused) {
-    if (!encode_codes_map(&tmX, a.x_codes, a.M, a.K, NP)) return cudaErrorInvalidValue;
+    const uint32_t box = (uint32_t)operand_rows(residue_rows(a));   // rows of X (and of R) per tile
+    if (!encode_codes_map(&tmX, a.x_codes, a.M, a.K, box)) return cudaErrorInvalidValue;
     if (a.r_codes != nullptr) {
-      if (!encode_codes_map(&tmR, a.r_codes, a.M, a.K, NP)) return cudaErrorInvalidValue;
+      if (!encode_codes_map(&tmR, a.r_codes, a.M, a.K, box)) return cudaErrorInvalidValue;
     } else {
       tmR = tmX;
     }
