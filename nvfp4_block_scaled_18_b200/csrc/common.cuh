@@ -118,6 +118,24 @@ __device__ __forceinline__ int64_t scale_offset(int64_t r, int64_t b, int64_t nb
   return ((r >> 7) * katoms + (b >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3);
 }
 
+// ------------------------------------------------- division by an invariant
+// n / d for any 32-bit n and 1 <= d < 2^32 by one multiply-high, one
+// subtract, one add and two shifts (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", PLDI 1994, section 4).
+struct DivMagic {
+  uint32_t m, s1, s2;
+};
+inline DivMagic make_div_magic(uint32_t d) {
+  uint32_t l = 0;
+  while (l < 32 && (uint64_t(1) << l) < d) ++l;                  // ceil(log2 d)
+  const uint64_t m = (((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d) + 1;
+  return DivMagic{(uint32_t)m, l < 1 ? l : 1u, l > 1 ? l - 1 : 0u};
+}
+__device__ __forceinline__ uint32_t div_invariant(uint32_t n, const DivMagic& dm) {
+  const uint32_t t1 = __umulhi(dm.m, n);
+  return (t1 + ((n - t1) >> dm.s1)) >> dm.s2;
+}
+
 // ------------------------------------------------------------ reductions
 
 __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {

@@ -68,6 +68,55 @@ __device__ __forceinline__ uint64_t quant_block16(const float v[16], float s, ui
   return (uint64_t)lo | ((uint64_t)hi << 32);
 }
 
+// quant_block16 for the streaming quantizer: the block maximum arrives as an
+// abs key (max of abs_key over the 16 values, so fl32 of it is max |v|), and
+// the E4M3 value d and the reciprocal fl32(1 / fl32(d * s)) of each of the 256
+// scale codes come from tables filled by make_scale_tables for this s.  Same
+// arithmetic as quant_block16, so the same codes and scales.
+__device__ __forceinline__ uint64_t quant_block16_tab(const float v[16], uint32_t amax_key, float s,
+                                                      const float* d_tab, const float* inv_tab, uint32_t& d_byte,
+                                                      float* deq) {
+  uint32_t db = 0;
+  if (s >= NVFP4_MIN_TENSOR_SCALE) db = f32_to_e4m3(__fdiv_rn(__uint_as_float(amax_key), __fmul_rn(6.0f, s)));
+  const float d = d_tab[db], inv = inv_tab[db];
+  const uint32_t lo =
+      f32x8_to_e2m1(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv), __fmul_rn(v[2], inv), __fmul_rn(v[3], inv),
+                    __fmul_rn(v[4], inv), __fmul_rn(v[5], inv), __fmul_rn(v[6], inv), __fmul_rn(v[7], inv));
+  const uint32_t hi =
+      f32x8_to_e2m1(__fmul_rn(v[8], inv), __fmul_rn(v[9], inv), __fmul_rn(v[10], inv), __fmul_rn(v[11], inv),
+                    __fmul_rn(v[12], inv), __fmul_rn(v[13], inv), __fmul_rn(v[14], inv), __fmul_rn(v[15], inv));
+  if (deq != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      deq[i] = __fmul_rn(__fmul_rn(e2m1_value(lo >> (4 * i)), d), s);
+      deq[8 + i] = __fmul_rn(__fmul_rn(e2m1_value(hi >> (4 * i)), d), s);
+    }
+  }
+  d_byte = db;
+  return (uint64_t)lo | ((uint64_t)hi << 32);
+}
+// Fill the 256-entry tables of quant_block16_tab for tensor scale s (all
+// threads of the block; the caller synchronises before use).
+__device__ __forceinline__ void make_scale_tables(float s, float* d_tab, float* inv_tab) {
+  for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+    const float d = e4m3_value((uint32_t)b);
+    d_tab[b] = d;
+    inv_tab[b] = (d != 0.0f) ? __frcp_rn(__fmul_rn(d, s)) : 0.0f;
+  }
+}
+// Max abs key of 16 values given as 8 words of packed bf16 pairs: the key of
+// a bf16 value is its 15 magnitude bits in the high half of the word.
+__device__ __forceinline__ uint32_t bf16x16_amax_key(const uint4& a, const uint4& b) {
+  uint32_t m = __vmaxu2(a.x & 0x7FFF7FFFu, a.y & 0x7FFF7FFFu);
+  m = __vmaxu2(m, a.z & 0x7FFF7FFFu);
+  m = __vmaxu2(m, a.w & 0x7FFF7FFFu);
+  m = __vmaxu2(m, b.x & 0x7FFF7FFFu);
+  m = __vmaxu2(m, b.y & 0x7FFF7FFFu);
+  m = __vmaxu2(m, b.z & 0x7FFF7FFFu);
+  m = __vmaxu2(m, b.w & 0x7FFF7FFFu);
+  return max(m & 0xFFFF0000u, m << 16);
+}
+
 // Load 16 consecutive elements (32-byte aligned for bf16, 64-byte for fp32) as fp32.
 __device__ __forceinline__ void load16(const __nv_bfloat16* p, float v[16]) {
   load8(p, v);

@@ -110,7 +110,7 @@ template <typename T, int MODE>
 __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t M, int64_t K,
                                                int64_t ldx, const float* s_ptr,
                                                const float* sr_ptr, QOut q, QOut r, WsHeader* ws,
-                                               int* st) {
+                                               int* st, DivMagic nb_div) {
   const uint32_t nb = (uint32_t)(K >> 4);
   const int64_t nblk = M * nb;
   const int64_t cta = (int64_t)(blockIdx.y * gridDim.x + blockIdx.x), ctas = (int64_t)gridDim.x * gridDim.y;
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t j = base + u * 256 + threadIdx.x;
       if (j < nblk) {
-        const uint32_t row = (uint32_t)j / nb, b = (uint32_t)j - row * nb;
+        const uint32_t row = div_invariant((uint32_t)j, nb_div), b = (uint32_t)j - row * nb;
         const T* p = x + (int64_t)row * ldx + (int64_t)b * 16;
         raw[u][0].load(p);
         raw[u][1].load(p + 8);
@@ -135,6 +135,13 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
   tc::griddep_wait();
   const float s = *s_ptr;
   const float s_r = (MODE == Q_RES_ONLY || MODE == Q_BOTH) ? *sr_ptr : 0.0f;
+  // per-code block scale and reciprocal for s (and for s_r)
+  __shared__ float d_tab[256], inv_tab[256];
+  __shared__ float dr_tab[(MODE == Q_RES_ONLY || MODE == Q_BOTH) ? 256 : 1];
+  __shared__ float invr_tab[(MODE == Q_RES_ONLY || MODE == Q_BOTH) ? 256 : 1];
+  make_scale_tables(s, d_tab, inv_tab);
+  if constexpr (MODE == Q_RES_ONLY || MODE == Q_BOTH) make_scale_tables(s_r, dr_tab, invr_tab);
+  __syncthreads();
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     if (MODE != Q_RES_ONLY && q.s != s_ptr) *q.s = s;
     if (MODE == Q_BOTH && r.s != sr_ptr) *r.s = s_r;
@@ -146,15 +153,22 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t j = base + u * 256 + threadIdx.x;
       if (j >= nblk) break;
-      const uint32_t row = (uint32_t)j / nb, b = (uint32_t)j - row * nb;
+      const uint32_t row = div_invariant((uint32_t)j, nb_div), b = (uint32_t)j - row * nb;
       float v[16];
       raw[u][0].get(v);
       raw[u][1].get(v + 8);
+      uint32_t key;
+      if constexpr (sizeof(T) == 2) {
+        key = bf16x16_amax_key(raw[u][0].u, raw[u][1].u);
+      } else {
+        key = 0u;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) bad = max(bad, abs_key(v[i]));
+        for (int i = 0; i < 16; ++i) key = max(key, abs_key(v[i]));
+      }
+      bad = max(bad, key);
       uint32_t db;
       float deq[16];
-      const uint64_t codes = quant_block16(v, s, db, MODE == Q_PLAIN ? nullptr : deq);
+      const uint64_t codes = quant_block16_tab(v, key, s, d_tab, inv_tab, db, MODE == Q_PLAIN ? nullptr : deq);
       if (MODE != Q_RES_ONLY) store_block16(q, row, (int)b, codes, db);
       if (MODE != Q_PLAIN) {
         float rv[16];
@@ -164,8 +178,11 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
 #pragma unroll
           for (int i = 0; i < 16; ++i) rkey = max(rkey, abs_key(rv[i]));
         } else {
+          uint32_t rk = 0u;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) rk = max(rk, abs_key(rv[i]));
           uint32_t dr;
-          const uint64_t rc = quant_block16(rv, s_r, dr, nullptr);
+          const uint64_t rc = quant_block16_tab(rv, rk, s_r, dr_tab, invr_tab, dr, nullptr);
           store_block16(r, row, (int)b, rc, dr);
         }
       }
@@ -596,7 +613,7 @@ cudaError_t launch_quant_m(const void* x, int64_t M, int64_t K, int64_t ldx, con
   cfg.attrs = attr;
   cfg.numAttrs = after_amax ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, k_quant<T, MODE>, static_cast<const T*>(x), M, K, ldx, s_ptr, sr_ptr, q, r, ws,
-                            st);
+                            st, make_div_magic((uint32_t)(K >> 4)));
 }
 
 template <typename T>
