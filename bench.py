@@ -169,7 +169,7 @@ def replica_throughput(work: float, ms: float, world: int, scale: float):
 
 # DRAM traffic / algorithmic bytes of k_decode_tc from its ncu capture (None once the kernel
 # changes after the capture)
-DECODE_TRAFFIC_RATIO = 33.091328e6 / (4096 * 14336 * 9 / 16 + 1 * 14336 * (2 + 9 / 16) + 4 * 1 * 4096)
+DECODE_TRAFFIC_RATIO = 33.093632e6 / (4096 * 14336 * 9 / 16 + 1 * 14336 * (2 + 9 / 16) + 4 * 1 * 4096)
 
 
 def decode_bytes(M, N, K):
@@ -761,7 +761,7 @@ def main():
         detail["resserve_residue_overhead"] = rs.measure()
         del rs
         # DRAM bytes per launch from the ncu capture of k_decode_tc (M=1, (4096,14336)):
-        # 33.091 MB measured against 33.077 MB algorithmic; scaled to the average call of a step
+        # 33.094 MB measured against 33.083 MB algorithmic; scaled to the average call of a step
         traffic = wk.step_bytes / len(wk.calls) * DECODE_TRAFFIC_RATIO if DECODE_TRAFFIC_RATIO else None
         roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": round(achieved / peaks["hbm_gbs"], 4),
