@@ -407,13 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // that read it (and its scale buffer) have completed, so waiting for the
     // stage's data is enough before overwriting the buffer.
     const uint32_t quad = (uint32_t)((warp - 4) * 32) << 16;
-    int s = 0;
-    uint32_t ph = 0;
-    for (int kt = kt0; kt < kt1; ++kt) {
-      // every lane waits; the warp goes on only if all saw the phase (the
-      // TMEM store is warp-collective)
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(saddr(&full[s]), ph, abort_flag, p.st))) break;
-      tc_fence_after();
+    auto write_stage = [&](int kt, int s) {
       const int t = kt - kt0;
       const uint8_t* sb = smem + s * WSTAGE;
       uint32_t r[32];
@@ -426,11 +420,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         r[16 + 4 * j + 1] = 0u; r[16 + 4 * j + 2] = 0u; r[16 + 4 * j + 3] = 0u;
       }
       tmem_st32(tmem + quad + SF_COL + (uint32_t)s * SF_BUF, r);   // W scales, then X (and R) scales
+    };
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kt = kt0; kt < kt1;) {
+      // every lane waits; the warp goes on only if all saw the phase (the
+      // TMEM store is warp-collective)
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(saddr(&full[s]), ph, abort_flag, p.st))) break;
+      tc_fence_after();
+      write_stage(kt, s);
+      // the next stage joins the batch if it has landed too: one wait covers
+      // both stores
+      const int s2 = s + 1 == STAGES ? 0 : s + 1;
+      const uint32_t ph2 = s2 == 0 ? ph ^ 1u : ph;
+      const bool two = kt + 1 < kt1 && __all_sync(0xFFFFFFFFu, mbar_test_wait(saddr(&full[s2]), ph2));
+      if (two) {
+        tc_fence_after();
+        write_stage(kt + 1, s2);
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(saddr(&sf_full[s]));
-      if (++s == STAGES) { s = 0; ph ^= 1u; }
+      if (lane == 0) {
+        mbar_arrive(saddr(&sf_full[s]));
+        if (two) mbar_arrive(saddr(&sf_full[s2]));
+      }
+      for (int n = 0; n < (two ? 2 : 1); ++n, ++kt)
+        if (++s == STAGES) { s = 0; ph ^= 1u; }
     }
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------- MMA issuer
