@@ -14,9 +14,10 @@
 // by cluster rank floor(r*ks/128); every CTA pushes its partial rows straight
 // into the owner's shared memory (distributed shared-memory stores), and after
 // one cluster barrier each owner sums its rows and writes Y.  Roles inside a
-// CTA (128 threads): warp 0 lane 0 issues TMA/bulk copies into a shared-memory
-// ring, warp 1 lane 0 copies scale atoms to TMEM and issues the MMAs, then all
-// four warps drain the accumulators.
+// CTA (256 threads): warp 0 lane 0 issues TMA/bulk copies into a shared-memory
+// ring; warps 4-7 (one per TMEM lane quadrant) write each k-tile's scale atoms
+// into one of two alternating TMEM scale buffers with tcgen05.st; warp 1 lane 0
+// issues the MMAs; then warps 0-3 drain the accumulators.
 //
 // Programmatic dependent launch: the kernel may start while the preceding
 // kernel on the stream (normally the activation quantizer) is still running.
@@ -36,7 +37,7 @@ namespace nvfp4 {
 using namespace tc;
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;   // warps 0-3: roles and the drain; warps 4-7: scales into TMEM
 constexpr int W_TILE = 128 * 128;   // 128 rows of W x 128 bytes (256 K-elements)
 constexpr int SF4 = 4 * 512;         // 4 scale atoms: one 128-row group x 256 K
 
@@ -49,10 +50,11 @@ struct Cfg {
   static constexpr int OFF_SFX = OFF_SFW + SF4;
   static constexpr int OFF_SFR = OFF_SFX + SF4;
   static constexpr int STAGE = ((OFF_SFR + (RES ? SF4 : 0)) + 1023) / 1024 * 1024;
-  // TMEM: acc [0,NP), acc_r [NP,2NP), scales of W, X, R (16 columns each)
+  // TMEM: acc [0,NP), acc_r [NP,2NP), then two scale buffers (alternating by
+  // k-tile) of W, X (and R) scales, 16 columns each
   static constexpr uint32_t ACC = 0, ACC_R = NP;
-  static constexpr uint32_t SFW_COL = 2 * NP, SFX_COL = 2 * NP + 16, SFR_COL = 2 * NP + 32;
-  static constexpr uint32_t COLS_USED = 2 * NP + 48;
+  static constexpr uint32_t SF_COL = (RES ? 2 : 1) * NP, SF_BUF = RES ? 48 : 32;
+  static constexpr uint32_t COLS_USED = SF_COL + 2 * SF_BUF;
   static constexpr uint32_t TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
   static constexpr int TMEM_CTAS = 512 / TMEM_COLS;               // CTAs whose TMEM fits on one SM
   static constexpr int BAR = 256;
@@ -78,7 +80,8 @@ struct Cfg {
   static constexpr int SMEM = SMEM_NEED > SMEM_MIN ? SMEM_NEED : SMEM_MIN;
   static constexpr int CTAS_PER_SM = (233472 / (SMEM + 1024)) < TMEM_CTAS ? (233472 / (SMEM + 1024)) : TMEM_CTAS;
   static_assert(1023 + STAGES * STAGE + PART_DED + BAR <= SMEM, "layout exceeds the shared-memory request");
-  static_assert((2 * STAGES + 1) * 8 + 8 <= BAR, "barrier block");
+  static_assert((2 * STAGES + 3) * 8 + 8 <= BAR, "barrier block");
+  static_assert(SF_COL % 4 == 0 && SF_BUF % 4 == 0, "block-scaled MMA scale operands start on 4-column TMEM boundaries");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(PART_OWN || PART <= STAGES * STAGE, "partials overlay the stage ring");
   static_assert(233472 / (SMEM + 1024) <= TMEM_CTAS, "TMEM must fit every co-resident CTA");
@@ -111,7 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* acc_full = bars + 2 * C::STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* sf_full = acc_full + 1;   // [2] a scale buffer written by all four quadrants
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   griddep_launch_dependents();   // the next kernel may set itself up; it waits for this one's results
@@ -128,6 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(saddr(&empty[s]), 1);
     }
     mbar_init(saddr(acc_full), 1);
+    mbar_init(saddr(&sf_full[0]), 4);
+    mbar_init(saddr(&sf_full[1]), 4);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -174,30 +180,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (RES) bulk_load(saddr(sb + C::OFF_SFR), p.sfr + (size_t)kt * 4 * 512, sf, bar);
       if (++s == C::STAGES) { s = 0; ph ^= 1u; }
     }
+  } else if (warp >= 4) {
+    // ------------------------------------------- scales into TMEM (tcgen05.st)
+    // Warp w writes TMEM lane quadrant w - 4 of scale buffer g & 1 for the
+    // CTA's g-th k-tile: line l of each W, X (and R) atom in every lane l of
+    // the quadrant (the layout of a 32x128b.warpx4 copy of the atoms).  Scale
+    // copies issued to the tensor pipe would queue behind the TMA stream;
+    // these stores do not.  The buffer is reused once the MMAs of k-tile g-2
+    // have completed.
+    const uint32_t quad = (uint32_t)((warp - 4) * 32) << 16;
+    for (int kt = kt0; kt < kt1; ++kt) {
+      const int g = kt - kt0, s = g % C::STAGES;
+      if (g >= 2) {
+        const int g2 = g - 2;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(saddr(&empty[g2 % C::STAGES]), (uint32_t)((g2 / C::STAGES) & 1),
+                                               abort_flag, p.st)))
+          break;
+      }
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(saddr(&full[s]), (uint32_t)((g / C::STAGES) & 1), abort_flag, p.st)))
+        break;
+      tc_fence_after();
+      const uint8_t* sb = smem + s * C::STAGE;
+      const uint32_t buf = C::SF_COL + (uint32_t)(g & 1) * C::SF_BUF;
+      uint32_t r[32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(sb + C::OFF_SFW + j * 512 + lane * 16);
+        const uint4 x = *reinterpret_cast<const uint4*>(sb + C::OFF_SFX + j * 512 + lane * 16);
+        r[4 * j] = w.x; r[4 * j + 1] = w.y; r[4 * j + 2] = w.z; r[4 * j + 3] = w.w;
+        r[16 + 4 * j] = x.x; r[16 + 4 * j + 1] = x.y; r[16 + 4 * j + 2] = x.z; r[16 + 4 * j + 3] = x.w;
+      }
+      tmem_st32(tmem + quad + buf, r);   // W scales, then X scales
+      if constexpr (RES) {
+        uint32_t rr[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sb + C::OFF_SFR + j * 512 + lane * 16);
+          rr[4 * j] = v.x; rr[4 * j + 1] = v.y; rr[4 * j + 2] = v.z; rr[4 * j + 3] = v.w;
+        }
+        tmem_st16(tmem + quad + buf + 32u, rr);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(saddr(&sf_full[g & 1]));
+    }
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------- MMA issuer
     const uint32_t idesc = idesc_nvf4(NP);
     int s = 0;
     uint32_t ph = 0;
     for (int kt = kt0; kt < kt1; ++kt) {
+      const int g = kt - kt0;
       if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) break;
+      if (!mbar_wait(saddr(&sf_full[g & 1]), (uint32_t)((g >> 1) & 1), abort_flag, p.st)) break;
       tc_fence_after();
       const int jmax = min(4, (p.K - kt * 256) / 64);
       const uint8_t* sb = smem + s * C::STAGE;
-      for (int j = 0; j < jmax; ++j) {
-        tc_cp_scales(tmem + C::SFW_COL + 4 * j, desc_sf_atom(saddr(sb + C::OFF_SFW + j * 512)));
-        tc_cp_scales(tmem + C::SFX_COL + 4 * j, desc_sf_atom(saddr(sb + C::OFF_SFX + j * 512)));
-        if (RES) tc_cp_scales(tmem + C::SFR_COL + 4 * j, desc_sf_atom(saddr(sb + C::OFF_SFR + j * 512)));
-      }
+      const uint32_t buf = C::SF_COL + (uint32_t)(g & 1) * C::SF_BUF;
       const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(sb + C::OFF_X));
       const uint64_t dr = desc_sw128(saddr(sb + C::OFF_R));
       for (int j = 0; j < jmax; ++j) {
         const uint32_t acc = (kt > kt0 || j > 0) ? 1u : 0u;
-        tc_mma_nvf4(tmem + C::ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + C::SFW_COL + 4 * j,
-                    tmem + C::SFX_COL + 4 * j, acc);
+        tc_mma_nvf4(tmem + C::ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + buf + 4 * j,
+                    tmem + buf + 16 + 4 * j, acc);
         if (RES)
-          tc_mma_nvf4(tmem + C::ACC_R, dw + (uint64_t)(2 * j), dr + (uint64_t)(2 * j), idesc,
-                      tmem + C::SFW_COL + 4 * j, tmem + C::SFR_COL + 4 * j, acc);
+          tc_mma_nvf4(tmem + C::ACC_R, dw + (uint64_t)(2 * j), dr + (uint64_t)(2 * j), idesc, tmem + buf + 4 * j,
+                      tmem + buf + 32 + 4 * j, acc);
       }
       tc_commit(saddr(&empty[s]));
       if (++s == C::STAGES) { s = 0; ph ^= 1u; }
@@ -222,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const int rows_max = (int)((128u + ks - 1) / ks);
   auto owner_row0 = [&](uint32_t o) { return (int)((o * 128u + ks - 1) / ks); };
-  {
+  if (warp < 4) {
     const int row = warp * 32 + lane;                              // TMEM lane = W row of the tile
     const uint32_t o = (uint32_t)row * ks / 128u;
     const int slot = (int)rank * rows_max + (row - owner_row0(o));
