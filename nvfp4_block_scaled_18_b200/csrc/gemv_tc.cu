@@ -58,8 +58,10 @@ struct Cfg {
   static constexpr uint32_t TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
   static constexpr int TMEM_CTAS = 512 / TMEM_COLS;               // CTAs whose TMEM fits on one SM
   static constexpr int BAR = 256;
-  // stages: as many as keep two CTAs per SM (four when TMEM allows only one CTA)
-  static constexpr int BUDGET = TMEM_CTAS >= 2 ? 114 * 1024 : 224 * 1024;
+  // stages: as many as keep two CTAs per SM (the request plus the 1 KB the
+  // runtime reserves per CTA must fit twice in the SM's 228 KB; four stages
+  // when TMEM allows only one CTA)
+  static constexpr int BUDGET = TMEM_CTAS >= 2 ? 233472 / 2 - 1024 : 224 * 1024;
   // pushed partial rows: every source rank has a slot of ceil(128/ks) rows in
   // its owner, ks * ceil(128/ks) <= 135 rows for ks <= 8
   static constexpr int PITCH = NP + 4;                            // floats per partial row (padded)
