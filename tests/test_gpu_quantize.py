@@ -55,6 +55,27 @@ def test_strided_rows(orc):
     assert_same_q(q, orc.quantize(x))
 
 
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("layout", [nv.SF_TILED, nv.SF_ROWMAJOR])
+def test_strided_rows_multi_launch(orc, dt, layout):
+    """Rows with a pitch larger than K through the multi-launch passes (the
+    strided amax loop and the block pass's row split), plain and residue."""
+    M, K, pad = 600, 4160, 64
+    x = wl.resserve_x(M, K)
+    big = torch.zeros((M, K + pad), dtype=dt, device="cuda")
+    big[:, :K] = to_dev(x, dt)
+    view = big[:, :K]
+    assert_same_q(run_quantize(view, layout), orc.quantize(x), "plain")
+    q, r = nv.NVFP4Tensor.empty(M, K, layout), nv.NVFP4Tensor.empty(M, K, layout)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_quantize_residue(view, q, r, workspace=nv.Workspace(M, K), dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    oq, orr = orc.quantize_residue(x)
+    assert_same_q(q, oq, "main")
+    assert_same_q(r, orr, "residue")
+
+
 @pytest.mark.parametrize("s", [0.01, 1.0 / 2688, 3.0e-7])
 def test_given_tensor_scale(orc, s):
     x = wl.decode_x(16, 1024)
