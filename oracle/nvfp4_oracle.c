@@ -256,3 +256,65 @@ ORC_API void orc_dequant_f64(const uint8_t* codes, const uint8_t* scales, float 
           orc_e2m1_decode(c) * orc_e4m3_decode(scales[r * nb + k / 16]) * (double)s;
     }
 }
+
+/* ------------------------------------------------------------------ MXFP4
+ * MX format (a NEXT row): 32-element blocks of E2M1 values sharing one E8M0
+ * scale, a power of two 2^(b-127) for bytes 0..254 (255 is NaN); no tensor
+ * scale (pages: ARCQuant blog sections 2.2 and 4.2 -- MX formats use E8M0
+ * scales with step 2^1 and 32-element blocks).  The pages do not give the
+ * scale rule; the reading taken is the shared-exponent rule of the MX format:
+ * the block scale is 2^(floor(log2 amax_b) - 2), 2 being the exponent of the
+ * largest E2M1 value, clamped to 2^-127..2^127, and 2^-127 for an all-zero
+ * block.  Elements are E2M1_RNE(x / scale), saturating at +-6 (an element in
+ * (6, 8) x scale clips to 6 x scale). */
+
+ORC_API double orc_e8m0_decode(uint8_t b) {
+  if (b == 255) return NAN;
+  return ldexp(1.0, (int)b - 127);
+}
+
+/* E8M0 byte of one 32-element block (maximum magnitude amax). */
+ORC_API uint8_t orc_mx_scale_byte(float amax) {
+  if (!(amax > 0.0f)) return 0;                       /* all-zero block: 2^-127 */
+  int e;
+  (void)frexp((double)amax, &e);                      /* amax = f 2^e, f in [0.5, 1) */
+  int x = (e - 1) - 2;                                /* floor(log2 amax) - 2 */
+  if (x < -127) x = -127;
+  if (x > 127) x = 127;
+  return (uint8_t)(x + 127);
+}
+
+/* Quantize rows x cols (cols a multiple of 32) to unpacked E2M1 codes and
+ * one E8M0 byte per 32-element block (row-major). */
+ORC_API void orc_mx_quantize(const float* x, int64_t rows, int64_t cols, int64_t ldx, uint8_t* codes,
+                             uint8_t* scales) {
+  const int64_t nb = cols / 32;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < nb; ++b) {
+      const float* xb = x + r * ldx + b * 32;
+      float amax = 0.0f;
+      for (int i = 0; i < 32; ++i) {
+        float a = fabsf(xb[i]);
+        if (a > amax) amax = a;
+      }
+      const uint8_t sb = orc_mx_scale_byte(amax);
+      scales[r * nb + b] = sb;
+      const int e = (int)sb - 127;
+      for (int i = 0; i < 32; ++i) {
+        /* x / 2^e is exact in binary64; the E2M1 rounding sees the exact quotient */
+        const double q = ldexp((double)xb[i], -e);
+        codes[r * cols + b * 32 + i] = orc_e2m1_encode((float)q);
+      }
+    }
+}
+
+/* deq[r][k] = v(code) * 2^(b-127), in binary64 (exact). */
+ORC_API void orc_mx_dequant_f64(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                double* out) {
+  const int64_t nb = cols / 32;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t k = 0; k < cols; ++k)
+      out[r * cols + k] = orc_e2m1_decode(codes[r * cols + k]) * orc_e8m0_decode(scales[r * nb + k / 32]);
+}

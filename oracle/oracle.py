@@ -24,7 +24,8 @@ Page citations (page title, section):
 
 Parity status: every function below is pinned by tests/test_oracle_*.py
 (exhaustive code tables, library cross-checks, brute force, closed forms and
-the pages' error bounds).
+the pages' error bounds); the MXFP4 functions at the end by
+tests/test_oracle_mx.py.
 """
 from __future__ import annotations
 
@@ -83,6 +84,12 @@ def _L():
             lib.orc_residue.argtypes = [f32p, i64, i64, i64, u8p, u8p, ctypes.c_float, f32p]
             lib.orc_rmsnorm.argtypes = [f32p, i64, i64, i64, f32p, ctypes.c_float, f32p, f32p]
             lib.orc_dequant_f64.argtypes = [u8p, u8p, ctypes.c_float, i64, i64, f64p]
+            lib.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
+            lib.orc_e8m0_decode.restype = ctypes.c_double
+            lib.orc_mx_scale_byte.argtypes = [ctypes.c_float]
+            lib.orc_mx_scale_byte.restype = ctypes.c_uint8
+            lib.orc_mx_quantize.argtypes = [f32p, i64, i64, i64, u8p, u8p]
+            lib.orc_mx_dequant_f64.argtypes = [u8p, u8p, i64, i64, f64p]
             _lib = lib
     return _lib
 
@@ -302,3 +309,67 @@ def gemm(a: QTensor, w: QTensor, rows=None) -> np.ndarray:
 def gemm_residue(a: QTensor, r: QTensor, w: QTensor, rows=None) -> np.ndarray:
     """Y = deq(Q(X)) deq(W)^T + deq(Q(R)) deq(W)^T ([RS] abstract)."""
     return gemm(a, w, rows) + gemm(r, w, rows)
+
+
+# ------------------------------------------------------------------ MXFP4
+# A NEXT row: 32-element blocks of E2M1 values under one E8M0 (power-of-two)
+# scale and no tensor scale ([ARC] sections 2.2 and 4.2: MX formats use E8M0
+# scales, step 2^1, and 32-element blocks).  Scale rule (a reading; the pages
+# do not give one): the shared exponent floor(log2 amax_b) - 2, clamped to
+# [-127, 127], with 2^-127 for an all-zero block; elements E2M1_RNE(x / scale),
+# saturating at 6.  Pinned by tests/test_oracle_mx.py.
+
+MX_BLOCK = 32
+
+
+def e8m0_decode(b: int) -> float:
+    """Value of an E8M0 byte: 2^(b - 127); 255 is NaN."""
+    return _L().orc_e8m0_decode(int(b) & 0xFF)
+
+
+def mx_scale_byte(amax: float) -> int:
+    """E8M0 byte of a block whose largest magnitude is amax (the reading above)."""
+    return _L().orc_mx_scale_byte(float(amax))
+
+
+def mx_quantize(x):
+    """MXFP4 quantization of an [M x K] array (K a multiple of 32).
+    Returns (codes uint8 [M x K] unpacked, scales uint8 [M x K/32] E8M0)."""
+    x = _f32(x)
+    M, K = x.shape
+    if K % MX_BLOCK:
+        raise ValueError("K must be a multiple of 32")
+    codes = np.empty((M, K), np.uint8)
+    scales = np.empty((M, K // MX_BLOCK), np.uint8)
+    _L().orc_mx_quantize(_p(x, ctypes.c_float), M, K, K, _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint8))
+    return codes, scales
+
+
+def mx_dequant(codes, scales) -> np.ndarray:
+    """Exact binary64 values v(code) * 2^(b - 127)."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    M, K = codes.shape
+    out = np.empty((M, K), np.float64)
+    _L().orc_mx_dequant_f64(_p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint8), M, K,
+                            _p(out, ctypes.c_double))
+    return out
+
+
+def mx_quantize_residue(x):
+    """ResServe's residue in MXFP4 ([RS] abstract: FP4 base plus FP4 residue):
+    R = fl32(x - deq(Q(x))), quantized with its own block scales.
+    Returns ((codes, scales) of X, (codes, scales) of R)."""
+    x = _f32(x)
+    qx = mx_quantize(x)
+    r = (x - mx_dequant(*qx).astype(np.float32)).astype(np.float32)
+    return qx, mx_quantize(r)
+
+
+def mx_gemm(qa, qw, qr=None) -> np.ndarray:
+    """Y = deq(Q(A)) deq(Q(W))^T (+ deq(Q(R)) deq(Q(W))^T), in binary64."""
+    wd = mx_dequant(*qw)
+    y = mx_dequant(*qa) @ wd.T
+    if qr is not None:
+        y = y + mx_dequant(*qr) @ wd.T
+    return y
