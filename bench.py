@@ -533,6 +533,21 @@ def measure_prefill_from(wk, peaks):
             "gemm_us": round(g_ms * 1e3, 2), "gemm_TFLOPs": round(flops / (g_ms * 1e-3) / 1e12, 1),
             "gemm_frac_fp4_peak": round(flops / (g_ms * 1e-3) / 1e12 / fp4_peak_tflops(peaks), 4),
             "quant_us": round(q_ms * 1e3, 2), "quant_GBps": round(q_bytes / (q_ms * 1e-3) / 1e9, 1)}
+    # MXFP4 quantizer (a NEXT row: 32-element blocks, E8M0 scales, one pass) on the
+    # first shape's activations, plain and with the residue
+    (_, M, N, Keff, S) = wk.calls[0]
+    x = wk.buf[(N, Keff - S)]["x"]
+    K = Keff - S
+    mc = torch.empty(M * K // 2, dtype=torch.uint8, device=x.device)
+    ms = torch.empty(M * K // 32, dtype=torch.uint8, device=x.device)
+    rc, rs = torch.empty_like(mc), torch.empty_like(ms)
+    mx_bytes = M * K * (2 + 0.5 + 1 / 32)
+    t_mx = time_back_to_back(lambda i: wk.nv.nvfp4_mx_quantize(x, mc, ms), 4)
+    t_mxr = time_back_to_back(lambda i: wk.nv.nvfp4_mx_quantize(x, mc, ms, rc, rs), 4)
+    out["mxfp4_quantize"] = {"shape": f"{M}x{K} bf16", "us": round(t_mx * 1e3, 2),
+                             "GBps": round(mx_bytes / (t_mx * 1e-3) / 1e9, 1),
+                             "residue_us": round(t_mxr * 1e3, 2),
+                             "residue_GBps": round((mx_bytes + M * K * (0.5 + 1 / 32)) / (t_mxr * 1e-3) / 1e9, 1)}
     achieved = flops_total / (gemm_ms_total * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak_tflops(peaks), 1),
             "unit": "TFLOP/s", "frac": round(achieved / fp4_peak_tflops(peaks), 4), "traffic": None,

@@ -217,6 +217,25 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize_noalloc(const void* x, nvfp4_dtype d
                                                     const float* scale_in, nvfp4_tensor* x_aug,
                                                     int* dev_status, void* stream);
 
+/* MXFP4 quantization (a NEXT row; ARCQuant post sections 2.2 and 4.2: MX
+ * formats use 32-element blocks and E8M0 power-of-two scales, no tensor scale).
+ * Scale rule (the pages give none; the MX shared-exponent rule):
+ *   per 32-block: b = clamp(floor(log2 amax_block) - 2 + 127, 0, 254), b = 0
+ *                 for an all-zero block; scale = 2^(b - 127)
+ *   per element:  code = E2M1_RNE_satfinite(x / scale)  (elements in (6, 8) x
+ *                 scale clip to 6 x scale)
+ * With r_codes != NULL also the residue R = fl32(x - v(code) scale), quantized
+ * the same way with its own block scales (ResServe abstract: FP4 base plus FP4
+ * residue).
+ * x: device, 16-byte aligned, ldx * sizeof(dt) a multiple of 16; K % 32 == 0.
+ * codes, r_codes: device, M x K/2 bytes, row-major, 16-byte aligned (element 2j
+ *   in the low nibble of byte j of its row).
+ * scales, r_scales: device, M x K/32 bytes, row-major (one E8M0 byte per block).
+ * A NaN/Inf input sets NVFP4_ERR_NONFINITE in *dev_status. */
+nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                               uint8_t* codes, uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales,
+                               int* dev_status, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* nvfp4_status_string(nvfp4_status status);
 

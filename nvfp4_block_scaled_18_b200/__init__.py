@@ -27,7 +27,7 @@ EXPORTED_SYMBOLS = ("nvfp4_scales_bytes", "nvfp4_workspace_size", "nvfp4_quantiz
                     "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize", "nvfp4_gemm",
                     "nvfp4_gemm_residue", "nvfp4_quantize_gemm", "nvfp4_quantize_residue_gemm",
                     "nvfp4_quantize_gemm_plan",
-                    "nvfp4_rmsnorm_reorder_quantize_noalloc",
+                    "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_mx_quantize",
                     "nvfp4_status_string", "nvfp4_version")
 NVFP4_NOALLOC_MAX_ROWS = 65536
 
@@ -73,8 +73,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.nvfp4_quantize_gemm_plan.restype = ctypes.c_int
         lib.nvfp4_quantize_residue_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, T, T, T, P,
                                                     ctypes.c_int, I64, P, P]
+        lib.nvfp4_mx_quantize.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, P, P, P, P]
         for fn in ("nvfp4_quantize", "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize",
-                   "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_gemm", "nvfp4_gemm_residue"):
+                   "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_gemm", "nvfp4_gemm_residue",
+                   "nvfp4_mx_quantize"):
             getattr(lib, fn).restype = ctypes.c_int
         lib.nvfp4_status_string.argtypes = [ctypes.c_int]
         lib.nvfp4_status_string.restype = ctypes.c_char_p
@@ -183,6 +185,21 @@ def nvfp4_quantize(x: torch.Tensor, q: NVFP4Tensor, scale_in: Optional[torch.Ten
     _check(lib.nvfp4_quantize(x.data_ptr(), _dtype_code(x), M, K, _ldx(x), _ptr(scale_in),
                               ctypes.byref(qc), ws_ptr, ws_n, _ptr(dev_status), _stream(stream)),
            "nvfp4_quantize")
+
+
+def nvfp4_mx_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                      r_codes: Optional[torch.Tensor] = None, r_scales: Optional[torch.Tensor] = None,
+                      dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """MXFP4: codes uint8 [M, K/2] (packed), scales uint8 [M, K/32] (E8M0), and
+    optionally the residue's codes and scales; all row-major on the device."""
+    lib = load_library()
+    M, K = x.shape
+    for t, n in ((codes, M * K // 2), (scales, M * K // 32), (r_codes, M * K // 2), (r_scales, M * K // 32)):
+        if t is not None and (t.dtype != torch.uint8 or t.numel() != n or not t.is_contiguous()):
+            raise ValueError("nvfp4_mx_quantize: output buffers must be contiguous uint8 of the MXFP4 sizes")
+    _check(lib.nvfp4_mx_quantize(x.data_ptr(), _dtype_code(x), M, K, _ldx(x), codes.data_ptr(), scales.data_ptr(),
+                                 _ptr(r_codes), _ptr(r_scales), _ptr(dev_status), _stream(stream)),
+           "nvfp4_mx_quantize")
 
 
 def nvfp4_quantize_residue(x: torch.Tensor, q: NVFP4Tensor, r: NVFP4Tensor,

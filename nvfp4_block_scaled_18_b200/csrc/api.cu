@@ -279,6 +279,17 @@ nvfp4_status nvfp4_quantize_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64
                                      dev_status, stream);
 }
 
+nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                               uint8_t* codes, uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales,
+                               int* dev_status, void* stream) {
+  NVFP4_TRY(check_input(x, dt, M, K, ldx));
+  if (K % 32 != 0 || codes == nullptr || scales == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if ((r_codes == nullptr) != (r_scales == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(codes) || (r_codes != nullptr && !aligned16(r_codes))) return NVFP4_ERR_ALIGNMENT;
+  return cuda_status(launch_mx_quant(x, dt, M, K, ldx, codes, scales, r_codes, r_scales, dev_status,
+                                     num_sms_current_device(), static_cast<cudaStream_t>(stream)));
+}
+
 const char* nvfp4_status_string(nvfp4_status st) {
   switch (st) {
     case NVFP4_OK: return "ok";

@@ -82,6 +82,11 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
 
 cudaError_t launch_gemv(const GemmArgs& g, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);
+// MXFP4 (32-element blocks, E8M0 scales): codes row-major M x K/2, scales row-major
+// M x K/32; r_codes == nullptr: no residue.
+cudaError_t launch_mx_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx, uint8_t* codes,
+                            uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales, int* st, int num_sms,
+                            cudaStream_t stream);
 cudaError_t launch_gemv_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);
 
 }  // namespace nvfp4
