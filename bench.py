@@ -548,6 +548,23 @@ def measure_prefill_from(wk, peaks):
                              "GBps": round(mx_bytes / (t_mx * 1e-3) / 1e9, 1),
                              "residue_us": round(t_mxr * 1e3, 2),
                              "residue_GBps": round((mx_bytes + M * K * (0.5 + 1 / 32)) / (t_mxr * 1e-3) / 1e9, 1)}
+    # MXFP4 GEMM (kind::mxf4, one E8M0 scale per 32 elements) on the same shape:
+    # both operands quantized on the device with TILED scales
+    from nvfp4_block_scaled_18_b200 import workloads as wl
+    nv = wk.nv
+    w = torch.from_numpy(wl.weights_normal(N, K)).to(x.device)
+    wc = torch.empty((N, K // 2), dtype=torch.uint8, device=x.device)
+    wsc = torch.empty(nv.mx_scales_bytes(N, K, nv.SF_TILED), dtype=torch.uint8, device=x.device)
+    nv.nvfp4_mx_quantize(w, wc.view(-1), wsc, sf_layout=nv.SF_TILED)
+    del w
+    xsc = torch.empty(nv.mx_scales_bytes(M, K, nv.SF_TILED), dtype=torch.uint8, device=x.device)
+    nv.nvfp4_mx_quantize(x, mc, xsc, sf_layout=nv.SF_TILED)
+    y = wk.buf[(N, K)]["y"]
+    t_mg = time_back_to_back(lambda i: nv.nvfp4_mx_gemm(mc.view(M, -1), xsc, wc, wsc, y), 4)
+    out["mxfp4_gemm"] = {"shape": f"M{M}_N{N}_K{K}", "us": round(t_mg * 1e3, 2),
+                         "TFLOPs": round(2.0 * M * N * K / (t_mg * 1e-3) / 1e12, 1),
+                         "frac_fp4_peak": round(2.0 * M * N * K / (t_mg * 1e-3) / 1e12 / fp4_peak_tflops(peaks), 4)}
+    del wc, wsc, xsc
     achieved = flops_total / (gemm_ms_total * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak_tflops(peaks), 1),
             "unit": "TFLOP/s", "frac": round(achieved / fp4_peak_tflops(peaks), 4), "traffic": None,

@@ -230,11 +230,31 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize_noalloc(const void* x, nvfp4_dtype d
  * x: device, 16-byte aligned, ldx * sizeof(dt) a multiple of 16; K % 32 == 0.
  * codes, r_codes: device, M x K/2 bytes, row-major, 16-byte aligned (element 2j
  *   in the low nibble of byte j of its row).
- * scales, r_scales: device, M x K/32 bytes, row-major (one E8M0 byte per block).
+ * scales, r_scales: device, nvfp4_mx_scales_bytes(M, K, sf_layout) bytes, one
+ *   E8M0 byte per block: ROWMAJOR (M x K/32) or TILED (the NVFP4 atom layout
+ *   with 32-element blocks: an atom holds 128 rows x 4 blocks = K 128; padding
+ *   bytes of a partial atom are left untouched).
  * A NaN/Inf input sets NVFP4_ERR_NONFINITE in *dev_status. */
 nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                uint8_t* codes, uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales,
-                               int* dev_status, void* stream);
+                               nvfp4_sf_layout sf_layout, int* dev_status, void* stream);
+
+/* Bytes of an MXFP4 scale buffer for a rows x cols matrix in `layout`
+ * (0 for an empty matrix). */
+size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout);
+
+/* MXFP4 W4A4 linear (ARCQuant post section 2.2: the MX block-scaled format on
+ * the same tensor cores): Y = deq(A) deq(W)^T, A = (a_codes, a_scales) M x K,
+ * W = (w_codes, w_scales) N x K, both quantized by nvfp4_mx_quantize with
+ * TILED scales; fp32 accumulation of the exact block products, output dtype
+ * out_dt with row stride ldy >= N.  One tensor-core kernel (128 x 256 tiles,
+ * kind::mxf4, one scale byte per 32 elements).
+ * Requirements: K % 128 == 0, K >= 256 (else NVFP4_ERR_UNSUPPORTED); codes and
+ * scales 16-byte aligned; y aligned to sizeof(out_dt).  The caller owns every
+ * buffer; nothing is allocated. */
+nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
+                           const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* y,
+                           nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* nvfp4_status_string(nvfp4_status status);

@@ -28,7 +28,7 @@ EXPORTED_SYMBOLS = ("nvfp4_scales_bytes", "nvfp4_workspace_size", "nvfp4_quantiz
                     "nvfp4_gemm_residue", "nvfp4_quantize_gemm", "nvfp4_quantize_residue_gemm",
                     "nvfp4_quantize_gemm_plan",
                     "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_mx_quantize",
-                    "nvfp4_status_string", "nvfp4_version")
+                    "nvfp4_mx_scales_bytes", "nvfp4_mx_gemm", "nvfp4_status_string", "nvfp4_version")
 NVFP4_NOALLOC_MAX_ROWS = 65536
 
 
@@ -73,10 +73,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.nvfp4_quantize_gemm_plan.restype = ctypes.c_int
         lib.nvfp4_quantize_residue_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, T, T, T, P,
                                                     ctypes.c_int, I64, P, P]
-        lib.nvfp4_mx_quantize.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, P, P, P, P]
+        lib.nvfp4_mx_quantize.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, P, P, ctypes.c_int, P, P]
+        lib.nvfp4_mx_scales_bytes.argtypes = [I64, I64, ctypes.c_int]
+        lib.nvfp4_mx_scales_bytes.restype = SZ
+        lib.nvfp4_mx_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, ctypes.c_int, I64, P, P]
         for fn in ("nvfp4_quantize", "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize",
                    "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_gemm", "nvfp4_gemm_residue",
-                   "nvfp4_mx_quantize"):
+                   "nvfp4_mx_quantize", "nvfp4_mx_gemm"):
             getattr(lib, fn).restype = ctypes.c_int
         lib.nvfp4_status_string.argtypes = [ctypes.c_int]
         lib.nvfp4_status_string.restype = ctypes.c_char_p
@@ -187,19 +190,45 @@ def nvfp4_quantize(x: torch.Tensor, q: NVFP4Tensor, scale_in: Optional[torch.Ten
            "nvfp4_quantize")
 
 
+def mx_scales_bytes(rows: int, cols: int, layout: int = SF_ROWMAJOR) -> int:
+    """Bytes of an MXFP4 scale buffer (one E8M0 byte per 32 elements)."""
+    return int(load_library().nvfp4_mx_scales_bytes(rows, cols, layout))
+
+
 def nvfp4_mx_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
                       r_codes: Optional[torch.Tensor] = None, r_scales: Optional[torch.Tensor] = None,
-                      dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
-    """MXFP4: codes uint8 [M, K/2] (packed), scales uint8 [M, K/32] (E8M0), and
-    optionally the residue's codes and scales; all row-major on the device."""
+                      dev_status: Optional[torch.Tensor] = None, stream=None,
+                      sf_layout: int = SF_ROWMAJOR) -> None:
+    """MXFP4: codes uint8 [M, K/2] (packed, row-major), scales uint8 (E8M0;
+    M x K/32 row-major, or the TILED atom layout), and optionally the
+    residue's codes and scales in the same layouts; all on the device."""
     lib = load_library()
     M, K = x.shape
-    for t, n in ((codes, M * K // 2), (scales, M * K // 32), (r_codes, M * K // 2), (r_scales, M * K // 32)):
+    ns = mx_scales_bytes(M, K, sf_layout) if K % 32 == 0 else M * K // 32
+    for t, n in ((codes, M * K // 2), (scales, ns), (r_codes, M * K // 2), (r_scales, ns)):
         if t is not None and (t.dtype != torch.uint8 or t.numel() != n or not t.is_contiguous()):
             raise ValueError("nvfp4_mx_quantize: output buffers must be contiguous uint8 of the MXFP4 sizes")
     _check(lib.nvfp4_mx_quantize(x.data_ptr(), _dtype_code(x), M, K, _ldx(x), codes.data_ptr(), scales.data_ptr(),
-                                 _ptr(r_codes), _ptr(r_scales), _ptr(dev_status), _stream(stream)),
+                                 _ptr(r_codes), _ptr(r_scales), sf_layout, _ptr(dev_status), _stream(stream)),
            "nvfp4_mx_quantize")
+
+
+def nvfp4_mx_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, w_codes: torch.Tensor,
+                  w_scales: torch.Tensor, y: torch.Tensor,
+                  dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """MXFP4 linear y = deq(A) deq(W)^T: a_codes uint8 [M, K/2], w_codes uint8
+    [N, K/2], both scale buffers in the TILED layout; y [M, N] fp32 or bf16."""
+    lib = load_library()
+    M, N, K = a_codes.shape[0], w_codes.shape[0], 2 * a_codes.shape[1]
+    if w_codes.shape[1] * 2 != K or tuple(y.shape) != (M, N):
+        raise ValueError("nvfp4_mx_gemm: shapes do not match")
+    for t, n in ((a_codes, M * K // 2), (w_codes, N * K // 2),
+                 (a_scales, mx_scales_bytes(M, K, SF_TILED)), (w_scales, mx_scales_bytes(N, K, SF_TILED))):
+        if t.dtype != torch.uint8 or t.numel() != n or not t.is_contiguous():
+            raise ValueError("nvfp4_mx_gemm: operands must be contiguous uint8 of the MXFP4 sizes")
+    _check(lib.nvfp4_mx_gemm(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(), w_scales.data_ptr(),
+                             M, N, K, y.data_ptr(), _out_dtype(y), _ldx(y), _ptr(dev_status), _stream(stream)),
+           "nvfp4_mx_gemm")
 
 
 def nvfp4_quantize_residue(x: torch.Tensor, q: NVFP4Tensor, r: NVFP4Tensor,

@@ -279,15 +279,46 @@ nvfp4_status nvfp4_quantize_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64
                                      dev_status, stream);
 }
 
+size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout) {
+  if (rows <= 0 || cols <= 0) return 0;
+  const int64_t nb = (cols + 31) / 32;
+  if (layout == NVFP4_SF_TILED) return (size_t)((rows + 127) / 128) * (size_t)((nb + 3) / 4) * 512;
+  return (size_t)rows * (size_t)nb;
+}
+
 nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                uint8_t* codes, uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales,
-                               int* dev_status, void* stream) {
+                               nvfp4_sf_layout sf_layout, int* dev_status, void* stream) {
   NVFP4_TRY(check_input(x, dt, M, K, ldx));
   if (K % 32 != 0 || codes == nullptr || scales == nullptr) return NVFP4_ERR_INVALID_ARG;
   if ((r_codes == nullptr) != (r_scales == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (sf_layout != NVFP4_SF_ROWMAJOR && sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_INVALID_ARG;
   if (!aligned16(codes) || (r_codes != nullptr && !aligned16(r_codes))) return NVFP4_ERR_ALIGNMENT;
-  return cuda_status(launch_mx_quant(x, dt, M, K, ldx, codes, scales, r_codes, r_scales, dev_status,
-                                     num_sms_current_device(), static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_mx_quant(x, dt, M, K, ldx, codes, scales, r_codes, r_scales,
+                                     sf_layout == NVFP4_SF_TILED, dev_status, num_sms_current_device(),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
+                           const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* y,
+                           nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream) {
+  if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr || y == nullptr ||
+      !dt_ok(out_dt))
+    return NVFP4_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || ldy < N || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
+    return NVFP4_ERR_INVALID_ARG;
+  if (K % 128 != 0 || K < 256) return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(a_scales) || !aligned16(w_scales))
+    return NVFP4_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(y) % dt_size(out_dt)) != 0) return NVFP4_ERR_ALIGNMENT;
+  GemmArgs g{};
+  g.a_codes = a_codes; g.a_scales = a_scales;
+  g.w_codes = w_codes; g.w_scales = w_scales;
+  g.y = y; g.ldy = ldy; g.y_bf16 = out_dt == NVFP4_BF16;
+  g.M = M; g.N = N; g.K = K; g.st = dev_status;
+  const cudaError_t e = launch_gemm_mx(g, num_sms_current_device(), static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
+  return cuda_status(e);
 }
 
 const char* nvfp4_status_string(nvfp4_status st) {

@@ -81,7 +81,7 @@ struct TcParams {
   int64_t ldy;
   int y_vec;       // Y base and row pitch allow 16-byte (fp32) / 8-byte (bf16) stores
   int M, N, K;
-  int katoms;      // scale atoms along K per 128-row group = ceil(K / 64)
+  int katoms;      // scale atoms along K per 128-row group: ceil(K / 64) (MX: K / 128)
   int b_groups;    // 128-row groups of W = ceil(N / 128)
   int m_blocks, n_blocks, num_tiles, k_tiles;
   int* st;
@@ -89,7 +89,10 @@ struct TcParams {
 
 // --------------------------------------------------------------- kernel
 
-template <bool BF16OUT>
+// MX: MXFP4 operands (32-element blocks, E8M0 scales, no tensor scales): the
+// same stages, with the scale atoms covering K = 128 each, so half of each
+// stage's scale area and of its TMEM scale buffer is used.
+template <bool BF16OUT, bool MX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const TcParams p) {
@@ -148,19 +151,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const uint8_t* st_base = smem + s * STAGE_BYTES;
-        uint32_t ra[16], rb[32];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 va = *reinterpret_cast<const uint4*>(st_base + OFF_SFA + j * 512 + lane * 16);
-          const uint4 v0 = *reinterpret_cast<const uint4*>(st_base + OFF_SFB + j * 512 + lane * 16);
-          const uint4 v1 = *reinterpret_cast<const uint4*>(st_base + OFF_SFB + 2048 + j * 512 + lane * 16);
-          ra[4 * j] = va.x; ra[4 * j + 1] = va.y; ra[4 * j + 2] = va.z; ra[4 * j + 3] = va.w;
-          rb[8 * j] = v0.x; rb[8 * j + 1] = v0.y; rb[8 * j + 2] = v0.z; rb[8 * j + 3] = v0.w;
-          rb[8 * j + 4] = v1.x; rb[8 * j + 5] = v1.y; rb[8 * j + 6] = v1.z; rb[8 * j + 7] = v1.w;
-        }
         const uint32_t buf = SF_COL + (uint32_t)s * SF_BUF;
-        tmem_st16(tmem + quad + buf, ra);
-        tmem_st32(tmem + quad + buf + 16u, rb);
+        if constexpr (MX) {
+          // two atoms per operand group: SFA atoms in columns 0-7, SFB atom a of
+          // group g in columns 8 + 8a + 4g
+          uint32_t rm[32];
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            const uint4 va = *reinterpret_cast<const uint4*>(st_base + OFF_SFA + a * 512 + lane * 16);
+            const uint4 v0 = *reinterpret_cast<const uint4*>(st_base + OFF_SFB + a * 512 + lane * 16);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(st_base + OFF_SFB + 2048 + a * 512 + lane * 16);
+            rm[4 * a] = va.x; rm[4 * a + 1] = va.y; rm[4 * a + 2] = va.z; rm[4 * a + 3] = va.w;
+            rm[8 + 8 * a] = v0.x; rm[8 + 8 * a + 1] = v0.y; rm[8 + 8 * a + 2] = v0.z; rm[8 + 8 * a + 3] = v0.w;
+            rm[12 + 8 * a] = v1.x; rm[12 + 8 * a + 1] = v1.y; rm[12 + 8 * a + 2] = v1.z; rm[12 + 8 * a + 3] = v1.w;
+          }
+#pragma unroll
+          for (int i = 24; i < 32; ++i) rm[i] = 0u;
+          tmem_st32(tmem + quad + buf, rm);
+        } else {
+          uint32_t ra[16], rb[32];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 va = *reinterpret_cast<const uint4*>(st_base + OFF_SFA + j * 512 + lane * 16);
+            const uint4 v0 = *reinterpret_cast<const uint4*>(st_base + OFF_SFB + j * 512 + lane * 16);
+            const uint4 v1 = *reinterpret_cast<const uint4*>(st_base + OFF_SFB + 2048 + j * 512 + lane * 16);
+            ra[4 * j] = va.x; ra[4 * j + 1] = va.y; ra[4 * j + 2] = va.z; ra[4 * j + 3] = va.w;
+            rb[8 * j] = v0.x; rb[8 * j + 1] = v0.y; rb[8 * j + 2] = v0.z; rb[8 * j + 3] = v0.w;
+            rb[8 * j + 4] = v1.x; rb[8 * j + 5] = v1.y; rb[8 * j + 6] = v1.z; rb[8 * j + 7] = v1.w;
+          }
+          tmem_st16(tmem + quad + buf, ra);
+          tmem_st32(tmem + quad + buf + 16u, rb);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -181,14 +202,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int s = g % STAGES;
           if (!mbar_wait_inline(saddr(&empty[s]), (uint32_t)((g / STAGES) & 1) ^ 1u, abort_flag, p.st)) goto producer_done;
           const int jmax = min(4, (p.K - kt * BK) / 64);
-          const uint32_t sf_bytes = (uint32_t)jmax * 512u;
+          const int atoms = MX ? (jmax + 1) / 2 : jmax, apt = MX ? 2 : 4;   // atoms of this / a full k-tile
+          const uint32_t sf_bytes = (uint32_t)atoms * 512u;
           uint8_t* st_base = smem + s * STAGE_BYTES;
           const uint32_t sbar = saddr(&sf_land[s]);
           mbar_expect_tx(sbar, sf_bytes * (1 + ngroups));
-          bulk_load(saddr(st_base + OFF_SFA), p.sfa + ((size_t)mb * p.katoms + kt * 4) * 512, sf_bytes, sbar);
+          bulk_load(saddr(st_base + OFF_SFA), p.sfa + ((size_t)mb * p.katoms + kt * apt) * 512, sf_bytes, sbar);
           for (int gi = 0; gi < ngroups; ++gi)
-            bulk_load(saddr(st_base + OFF_SFB + gi * 2048), p.sfb + ((size_t)(nb * 2 + gi) * p.katoms + kt * 4) * 512,
-                      sf_bytes, sbar);
+            bulk_load(saddr(st_base + OFF_SFB + gi * 2048),
+                      p.sfb + ((size_t)(nb * 2 + gi) * p.katoms + kt * apt) * 512, sf_bytes, sbar);
           const uint32_t bar = saddr(&full[s]);
           mbar_expect_tx(bar, A_BYTES + B_BYTES);
           tma_load_2d(saddr(st_base), &tmA, kt * BK_BYTES, mb * BM, bar);
@@ -213,9 +235,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint8_t* st_base = smem + s * STAGE_BYTES;
           const uint64_t da = desc_sw128(saddr(st_base)), db = desc_sw128(saddr(st_base + OFF_B));
           const uint32_t buf = SF_COL + (uint32_t)s * SF_BUF;
-          for (int j = 0; j < jmax; ++j)
-            tc_mma_nvf4(tmem + ACC_COL, da + (uint64_t)(2 * j), db + (uint64_t)(2 * j), idesc, tmem + buf + 4 * j,
-                        tmem + buf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < jmax; ++j) {
+            if constexpr (MX)   // K = 64 chunk j: atom j / 2, scale bytes 2 (j % 2) and 2 (j % 2) + 1
+              tc_mma_mxf4(tmem + ACC_COL, da + (uint64_t)(2 * j), db + (uint64_t)(2 * j),
+                          idesc_mxf4(BN, 2u * (uint32_t)(j & 1)), tmem + buf + 4 * (j >> 1),
+                          tmem + buf + 8 + 8 * (j >> 1), (kt > 0 || j > 0) ? 1u : 0u);
+            else
+              tc_mma_nvf4(tmem + ACC_COL, da + (uint64_t)(2 * j), db + (uint64_t)(2 * j), idesc, tmem + buf + 4 * j,
+                          tmem + buf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+          }
           tc_commit(saddr(&empty[s]));
         }
         tc_commit(saddr(acc_full));
@@ -230,7 +258,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float* buf = epi + ew * 32 * EPI_PITCH;
     const int sub_r = lane >> 1, sub_c = (lane & 1) * 4;
     int local = 0;
-    const float alpha = (*p.a_s) * (*p.w_s);
+    const float alpha = MX ? 1.0f : (*p.a_s) * (*p.w_s);   // MXFP4 has no tensor scales
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
       const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
       if (!mbar_wait_inline(saddr(acc_full), (uint32_t)(local & 1), abort_flag, p.st)) break;
@@ -330,9 +358,10 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
 
 }  // namespace tc
 
-cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) {
+template <bool MX>
+cudaError_t launch_gemm_impl(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   if (g.r_codes != nullptr) return cudaErrorNotSupported;  // own-scale residue: small-M paths only
-  if (g.K % 64 != 0 || g.K < BK) return cudaErrorNotSupported;
+  if (MX ? (g.K % 128 != 0 || g.K < 128) : (g.K % 64 != 0 || g.K < BK)) return cudaErrorNotSupported;
   CUtensorMap tmA, tmB;
   if (!encode_codes_map(&tmA, g.a_codes, g.M, g.K, BM) || !encode_codes_map(&tmB, g.w_codes, g.N, g.K, BN))
     return cudaErrorInvalidValue;
@@ -344,14 +373,14 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) 
     p.y_vec = (reinterpret_cast<uintptr_t>(g.y) % vec_bytes == 0) && ((size_t)g.ldy * esize) % vec_bytes == 0;
   }
   p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K;
-  p.katoms = (int)((g.K + 63) / 64);
+  p.katoms = MX ? (int)(g.K / 128) : (int)((g.K + 63) / 64);
   p.b_groups = (int)((g.N + 127) / 128);
   p.m_blocks = (int)((g.M + BM - 1) / BM);
   p.n_blocks = (int)((g.N + BN - 1) / BN);
   p.num_tiles = p.m_blocks * p.n_blocks;
   p.k_tiles = (int)((g.K + BK - 1) / BK);
   p.st = g.st;
-  auto kern = g.y_bf16 ? k_gemm_nvf4<true> : k_gemm_nvf4<false>;
+  auto kern = g.y_bf16 ? k_gemm_nvf4<true, MX> : k_gemm_nvf4<false, MX>;
   // the register split assumes the launch allocates LAUNCH_REGS per thread
   cudaFuncAttributes fa{};
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != LAUNCH_REGS) return cudaErrorNotSupported;
@@ -360,6 +389,14 @@ cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) 
   const int grid = std::max(1, std::min(p.num_tiles, num_sms));
   kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream) {
+  return launch_gemm_impl<false>(g, num_sms, stream);
+}
+
+cudaError_t launch_gemm_mx(const GemmArgs& g, int num_sms, cudaStream_t stream) {
+  return launch_gemm_impl<true>(g, num_sms, stream);
 }
 
 }  // namespace nvfp4

@@ -82,10 +82,13 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
 
 cudaError_t launch_gemv(const GemmArgs& g, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemm_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);
-// MXFP4 (32-element blocks, E8M0 scales): codes row-major M x K/2, scales row-major
-// M x K/32; r_codes == nullptr: no residue.
+// MXFP4 GEMM Y = deq(A) deq(W)^T: codes as for NVFP4, E8M0 scales in the TILED
+// atom layout with 32-element blocks (a_s, w_s unused); K % 128 == 0.
+cudaError_t launch_gemm_mx(const GemmArgs& g, int num_sms, cudaStream_t stream);
+// MXFP4 (32-element blocks, E8M0 scales): codes row-major M x K/2, scales
+// row-major M x K/32 or TILED; r_codes == nullptr: no residue.
 cudaError_t launch_mx_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx, uint8_t* codes,
-                            uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales, int* st, int num_sms,
+                            uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales, bool tiled, int* st, int num_sms,
                             cudaStream_t stream);
 cudaError_t launch_gemv_tc(const GemmArgs& g, int num_sms, cudaStream_t stream);
 

@@ -62,7 +62,7 @@ __device__ __forceinline__ uint32_t mx_block(const float v[32], uint4& packed, f
 template <typename T, bool RES>
 __global__ void __launch_bounds__(256) k_mx_quant(const T* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
                                                   uint8_t* codes, uint8_t* scales, uint8_t* r_codes,
-                                                  uint8_t* r_scales, int* st) {
+                                                  uint8_t* r_scales, bool tiled, int* st) {
   const int64_t nb = K / 32, nblk = M * nb;
   uint32_t bad = 0;
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < nblk; j += (int64_t)gridDim.x * blockDim.x) {
@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(256) k_mx_quant(const T* __restrict__ x, int64
     const uint32_t sb = mx_block(v, packed, RES ? deq : nullptr);
     bad = max(bad, sb);
     *reinterpret_cast<uint4*>(codes + row * (K / 2) + b * 16) = packed;
-    scales[row * nb + b] = (uint8_t)sb;
+    const int64_t so = scale_offset(row, b, nb, tiled);   // an atom holds 4 blocks, as for NVFP4
+    scales[so] = (uint8_t)sb;
     if (RES) {
       float r[32];
 #pragma unroll
@@ -84,7 +85,7 @@ __global__ void __launch_bounds__(256) k_mx_quant(const T* __restrict__ x, int64
       uint4 rp;
       const uint32_t rb = mx_block(r, rp, nullptr);
       *reinterpret_cast<uint4*>(r_codes + row * (K / 2) + b * 16) = rp;
-      r_scales[row * nb + b] = (uint8_t)rb;
+      r_scales[so] = (uint8_t)rb;
     }
   }
   if (bad >= 253u) report_status(st, NVFP4_ERR_NONFINITE);   // a NaN/Inf block maximum
@@ -92,26 +93,27 @@ __global__ void __launch_bounds__(256) k_mx_quant(const T* __restrict__ x, int64
 
 template <typename T>
 cudaError_t launch_mx_t(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* scales,
-                        uint8_t* r_codes, uint8_t* r_scales, int* st, int num_sms, cudaStream_t stream) {
+                        uint8_t* r_codes, uint8_t* r_scales, bool tiled, int* st, int num_sms,
+                        cudaStream_t stream) {
   const int64_t nblk = M * (K / 32);
   const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>((nblk + 255) / 256, (int64_t)num_sms * 8));
   if (r_codes != nullptr)
     k_mx_quant<T, true><<<g, 256, 0, stream>>>(static_cast<const T*>(x), M, K, ldx, codes, scales, r_codes,
-                                                r_scales, st);
+                                                r_scales, tiled, st);
   else
     k_mx_quant<T, false><<<g, 256, 0, stream>>>(static_cast<const T*>(x), M, K, ldx, codes, scales, nullptr,
-                                                 nullptr, st);
+                                                 nullptr, tiled, st);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_mx_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx, uint8_t* codes,
-                            uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales, int* st, int num_sms,
-                            cudaStream_t stream) {
+                            uint8_t* scales, uint8_t* r_codes, uint8_t* r_scales, bool tiled, int* st,
+                            int num_sms, cudaStream_t stream) {
   return dt == NVFP4_BF16
-             ? launch_mx_t<__nv_bfloat16>(x, M, K, ldx, codes, scales, r_codes, r_scales, st, num_sms, stream)
-             : launch_mx_t<float>(x, M, K, ldx, codes, scales, r_codes, r_scales, st, num_sms, stream);
+             ? launch_mx_t<__nv_bfloat16>(x, M, K, ldx, codes, scales, r_codes, r_scales, tiled, st, num_sms, stream)
+             : launch_mx_t<float>(x, M, K, ldx, codes, scales, r_codes, r_scales, tiled, st, num_sms, stream);
 }
 
 }  // namespace nvfp4

@@ -128,6 +128,18 @@ __device__ __forceinline__ void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t
       ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
       : "memory");
 }
+// MXFP4: E2M1 operands with one UE8M0 scale per 32 elements (scale_vec::2X).
+// An MMA (K = 64) reads 2 scale bytes per row from its TMEM scale column at the
+// byte offset given by the scale-factor IDs of the instruction descriptor.
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+      ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -187,6 +199,12 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
 // fp32 accumulator, M = 128, N = n.
 __device__ __forceinline__ uint32_t idesc_nvf4(int n) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+// kind::mxf4: E2M1 A and B, UE8M0 scales (bit 23), M = 128, N = n; sf_id: the
+// byte offset (0 or 2) of the MMA's two scale bytes in the A and B scale columns.
+__device__ __forceinline__ uint32_t idesc_mxf4(int n, uint32_t sf_id) {
+  return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(128 >> 4) << 24) | (sf_id << 29);
 }
 
 
