@@ -675,7 +675,8 @@ def profile_case(case: str) -> int:
     decode   -- nvfp4_quantize_gemm, M=1, (N,K)=(4096,14336), 5 weight copies (147 MB)
     prefill  -- nvfp4_gemm, M=8192, (N,K)=(14336,4096) (A 19 MB, W 33 MB, Y 470 MB)
     quantize -- nvfp4_quantize of the 8192x4096 bf16 prefill activations (67 MB)
-    reorder  -- nvfp4_rmsnorm_reorder_quantize of the same activations, S=256."""
+    reorder  -- nvfp4_rmsnorm_reorder_quantize of the same activations, S=256
+    mxgemm   -- nvfp4_mx_gemm, M=8192, (N,K)=(14336,4096), MXFP4 operands with TILED scales."""
     import nvfp4_block_scaled_18_b200 as nv
     from nvfp4_block_scaled_18_b200 import workloads as wl
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -702,6 +703,19 @@ def profile_case(case: str) -> int:
         y = torch.empty((M, N), device=dev)
         for _ in range(3):
             nv.nvfp4_gemm(qa, qw, y)
+    elif case == "mxgemm":
+        M, N, K = 8192, 14336, 4096
+        ops = []
+        for v in (wl.to_bf16(wl.prefill_x(M, K)).to(dev), torch.from_numpy(wl.weights_normal(N, K)).to(dev)):
+            rows = v.shape[0]
+            c = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev)
+            sc = torch.empty(nv.mx_scales_bytes(rows, K, nv.SF_TILED), dtype=torch.uint8, device=dev)
+            nv.nvfp4_mx_quantize(v, c.view(-1), sc, sf_layout=nv.SF_TILED)
+            ops.append((c, sc))
+            del v
+        y = torch.empty((M, N), device=dev)
+        for _ in range(3):
+            nv.nvfp4_mx_gemm(ops[0][0], ops[0][1], ops[1][0], ops[1][1], y)
     elif case == "reorder":
         M, K, S = 8192, 4096, 256
         x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
@@ -736,7 +750,7 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="decode: launch every step directly on the stream (no CUDA graphs) and skip the "
                          "per-call detail; for profilers that cannot follow graph replays")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder"],
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder", "mxgemm"],
                     help="run a few launches of one kernel on a small case (for ncu captures) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
