@@ -517,6 +517,46 @@ def prefill_e2e(wk, steps):
     return start.elapsed_time(end)
 
 
+def measure_arcquant(nv, dev, peaks):
+    """ARCQuant prefill: X 2048 x 4096 bf16 (2% channels x30), gamma, a perm from
+    512 calibration rows, W 11008 x 4096. For S in {0, 128, 256, 512}: the fused
+    RMSNorm + reorder + K->K+S quantizer, rotating over 16 activation copies
+    (268 MB, > 2x L2), and the augmented GEMM Y = s_aug s_w [QX|QR][QW|QW_o]^T
+    (tensor-bound; one operand copy)."""
+    from nvfp4_block_scaled_18_b200 import workloads as wl
+    M, K, N = wl.ARC_M, wl.ARC_K, wl.ARC_N
+    x, gamma, perm = wl.arc_inputs()
+    ncopy = 16
+    xs = [wl.to_bf16(x).to(dev) for _ in range(ncopy)]
+    g = wl.to_bf16(gamma).to(dev)
+    p = torch.from_numpy(np.ascontiguousarray(perm, dtype=np.int32)).to(dev)
+    w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
+    y = torch.empty((M, N), dtype=torch.float32, device=dev)
+    ws = nv.Workspace(M, K, dev)
+    out = {"shape": f"M{M}_N{N}_K{K}"}
+    for S in (0, 128, 256, 512):
+        qs = [nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED, device=dev) for _ in range(ncopy)]
+        w_aug = torch.cat([w[:, p.long()], w[:, p[:S].long()]], dim=1).contiguous()
+        qw = nv.NVFP4Tensor.empty(N, K + S, nv.SF_TILED, device=dev)
+        nv.nvfp4_quantize(w_aug, qw, workspace=nv.Workspace(N, K + S, dev))
+        del w_aug
+        t_q = time_back_to_back(lambda i: nv.nvfp4_rmsnorm_reorder_quantize(
+            xs[i], qs[i], gamma=g, eps=1e-5, perm=p, S=S, workspace=ws), ncopy)
+        t_g = time_back_to_back(lambda i: nv.nvfp4_gemm(qs[i % ncopy], qw, y), 4)
+        q_bytes = 2 * M * K + M * (K + S) * 9 // 16 + 6 * K
+        flops = 2.0 * M * N * (K + S)
+        out[f"S{S}"] = {"quant_us": round(t_q * 1e3, 2), "quant_GBps": round(q_bytes / (t_q * 1e-3) / 1e9, 1),
+                        "quant_frac_hbm": round(q_bytes / (t_q * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                        "gemm_us": round(t_g * 1e3, 2), "gemm_TFLOPs": round(flops / (t_g * 1e-3) / 1e12, 1),
+                        "gemm_frac_fp4_peak": round(flops / (t_g * 1e-3) / 1e12 / fp4_peak_tflops(peaks), 4)}
+        del qs, qw
+    base = out["S0"]["quant_us"] + out["S0"]["gemm_us"]
+    for S in (128, 256, 512):
+        o = out[f"S{S}"]
+        o["overhead_pct_vs_S0"] = round(100.0 * ((o["quant_us"] + o["gemm_us"]) / base - 1.0), 1)
+    return out
+
+
 def measure_prefill_from(wk, peaks):
     """Per-launch GEMM and quantizer times on the prefill workload."""
     out, flops_total, gemm_ms_total = {}, 0.0, 0.0
@@ -565,6 +605,10 @@ def measure_prefill_from(wk, peaks):
                          "TFLOPs": round(2.0 * M * N * K / (t_mg * 1e-3) / 1e12, 1),
                          "frac_fp4_peak": round(2.0 * M * N * K / (t_mg * 1e-3) / 1e12 / fp4_peak_tflops(peaks), 4)}
     del wc, wsc, xsc
+    try:
+        out["arcquant_prefill"] = measure_arcquant(nv, x.device, peaks)
+    except Exception as e:   # a detail leg: record the failure, keep the line
+        out["arcquant_prefill"] = {"error": f"{type(e).__name__}: {e}"}
     achieved = flops_total / (gemm_ms_total * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak_tflops(peaks), 1),
             "unit": "TFLOP/s", "frac": round(achieved / fp4_peak_tflops(peaks), 4), "traffic": None,
