@@ -113,3 +113,41 @@ def test_quantize_gemm_plan_rejects_without_device(lib):
     assert nv.nvfp4_quantize_gemm_plan(4, 4096, 320 + 16) == 0
     assert nv.nvfp4_quantize_gemm_plan(16, 128, 65536) == 0
     assert nv.nvfp4_quantize_gemm_plan(16, 128, 32768, x_dtype=torch.float32) == 0
+
+
+def test_mx_host_queries(lib):
+    # one E8M0 byte per 32 elements; TILED atoms hold 128 rows x 4 blocks (K = 128)
+    assert nv.mx_scales_bytes(4, 256, nv.SF_ROWMAJOR) == 4 * 8
+    assert nv.mx_scales_bytes(4, 256, nv.SF_TILED) == 2 * 512
+    assert nv.mx_scales_bytes(129, 160, nv.SF_TILED) == 2 * 2 * 512
+    assert nv.mx_scales_bytes(0, 256, nv.SF_TILED) == 0
+
+
+def test_mx_validation_before_launch(lib):
+    good = 1 << 20
+    q = lib.nvfp4_mx_quantize
+    assert q(good, 1, 4, 48, 48, good, good, None, None, 0, None, None) == 1          # K % 32
+    assert q(good, 1, 4, 64, 64, good, good, None, None, 5, None, None) == 1          # bad layout
+    assert q(good, 1, 4, 64, 64, good, good, good, None, 0, None, None) == 1          # residue half given
+    assert q(good, 1, 4, 64, 64, good + 8, good, None, None, 0, None, None) == 2      # misaligned codes
+    assert q(good, 1, 4, 64, 64, None, good, None, None, 0, None, None) == 1          # no codes
+    g = lib.nvfp4_mx_gemm
+    assert g(None, good, good, good, 128, 256, 256, good, 0, 256, None, None) == 1    # null operand
+    assert g(good, good, good, good, 128, 256, 192, good, 0, 256, None, None) == 3    # K % 128
+    assert g(good, good, good, good, 128, 256, 128, good, 0, 256, None, None) == 3    # K < 256
+    assert g(good, good, good, good, 128, 256, 256, good, 0, 200, None, None) == 1    # ldy < N
+    assert g(good, good + 4, good, good, 128, 256, 256, good, 0, 256, None, None) == 2  # misaligned scales
+    assert g(good, good, good, good, 128, 256, 256, good + 2, 0, 256, None, None) == 2  # misaligned fp32 y
+    assert g(good, good, good, good, 128, 256, 256, good, 7, 256, None, None) == 1    # bad out dtype
+    assert g(good, good, good, good, 0, 256, 256, good, 0, 256, None, None) == 1      # empty M
+
+
+def test_mx_binding_checks_shapes(lib):
+    ac = torch.zeros((128, 128), dtype=torch.uint8)
+    wc = torch.zeros((256, 64), dtype=torch.uint8)                  # K mismatch
+    s = torch.zeros(1024, dtype=torch.uint8)
+    y = torch.zeros((128, 256))
+    with pytest.raises(ValueError):
+        nv.nvfp4_mx_gemm(ac, s, wc, s, y)
+    with pytest.raises(ValueError):                                 # scales of the wrong size
+        nv.nvfp4_mx_gemm(ac, s, torch.zeros((256, 128), dtype=torch.uint8), s, y)
