@@ -76,6 +76,7 @@ nvfp4_status check_gemm_operands(const nvfp4_tensor* a, const nvfp4_tensor* r, c
   if (ldy < N) return NVFP4_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(y) % dt_size(out_dt)) != 0) return NVFP4_ERR_ALIGNMENT;
   if (K % 64 != 0) return NVFP4_ERR_UNSUPPORTED;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return NVFP4_ERR_UNSUPPORTED;  // 32-bit in the kernels
   return NVFP4_OK;
 }
 
@@ -252,7 +253,9 @@ nvfp4_status nvfp4_quantize_residue_gemm(const void* x, nvfp4_dtype dt, int64_t 
 }
 
 int nvfp4_quantize_gemm_plan(int64_t M, int64_t N, int64_t K, nvfp4_dtype dt, int residue, nvfp4_dtype out_dt) {
-  if (M < 1 || M > 16 || N < 1 || K < 256 || K % 64 != 0 || !dt_ok(dt) || !dt_ok(out_dt)) return 0;
+  if (M < 1 || M > 16 || N < 1 || N > INT32_MAX || K < 256 || K > INT32_MAX || K % 64 != 0 || !dt_ok(dt) ||
+      !dt_ok(out_dt))
+    return 0;
   if (M * (K / 8) > quant_small_max_units(dt)) return 0;
   static const uint8_t dummy[16] = {0};
   DecodeArgs d{};

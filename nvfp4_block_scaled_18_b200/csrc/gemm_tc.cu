@@ -361,7 +361,11 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
 template <bool MX>
 cudaError_t launch_gemm_impl(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   if (g.r_codes != nullptr) return cudaErrorNotSupported;  // own-scale residue: small-M paths only
-  if (MX ? (g.K % 128 != 0 || g.K < 128) : (g.K % 64 != 0 || g.K < BK)) return cudaErrorNotSupported;
+  if (MX ? (g.K % 128 != 0 || g.K < BK) : (g.K % 64 != 0 || g.K < BK)) return cudaErrorNotSupported;
+  // sizes, tile coordinates and the tile count are 32-bit in the kernel
+  if (g.M > INT32_MAX || g.N > INT32_MAX || g.K > INT32_MAX ||
+      ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN) > INT32_MAX)
+    return cudaErrorNotSupported;
   CUtensorMap tmA, tmB;
   if (!encode_codes_map(&tmA, g.a_codes, g.M, g.K, BM) || !encode_codes_map(&tmB, g.w_codes, g.N, g.K, BN))
     return cudaErrorInvalidValue;

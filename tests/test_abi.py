@@ -151,3 +151,11 @@ def test_mx_binding_checks_shapes(lib):
         nv.nvfp4_mx_gemm(ac, s, wc, s, y)
     with pytest.raises(ValueError):                                 # scales of the wrong size
         nv.nvfp4_mx_gemm(ac, s, torch.zeros((256, 128), dtype=torch.uint8), s, y)
+
+
+def test_sizes_beyond_32_bits_rejected(lib):
+    good = 1 << 20
+    a, w = _tensor(4, 64, good, good, good), _tensor(1 << 31, 64, good, good, good)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(w), good, 0, 1 << 31, None, None) == 3
+    assert lib.nvfp4_quantize_gemm_plan(1, 1 << 31, 4096, 1, 0, 0) == 0
+    assert lib.nvfp4_mx_gemm(good, good, good, good, 1 << 31, 256, 256, good, 0, 256, None, None) == 1
