@@ -662,52 +662,92 @@ def cpu_oracle_sample(workload: str = "decode", budget_s: float = 12.0):
                       f"+ fp64 dequantized GEMM, {t_total:.1f} s"}
 
 
+def arm_config(workload: str, world: int, calls_per_step: int) -> dict:
+    """The `config` of a bench line; both arms report the same one."""
+    if workload == "decode":
+        return {"workload": "decode GEMV (M in 1,2,4,8,16; (N,K) in (4096,4096),(14336,4096),(4096,14336)); "
+                            "online bf16->NVFP4 activation quantization + NVFP4 GEMM in one launch, fp32 out",
+                "calls_per_step": calls_per_step,
+                "l2": "every call streams its own weight copy; >= 260 MB of copies per shape (> L2)",
+                "parallelism": f"replicas x{world}"}
+    return {"workload": "large prefill W4A4 GEMM, M=8192, (N,K) in (14336,4096),(4096,14336),(28672,8192), "
+                        "each without and with the S=256 outlier-residue K extension; online quantization",
+            "calls_per_step": calls_per_step, "l2": "inputs > L2 (X 67-235 MB, Y 134-940 MB per call)",
+            "parallelism": f"replicas x{world}"}
+
+
 def reference_arm(args):
-    """--impl reference: the CPU oracle timed as the comparison arm (rank 0 only)."""
+    """--impl reference: the CPU oracle, as it stands, timed as the comparison arm
+    on the same workload, metric and unit (rank 0 only). Each step is one call of
+    the workload on a bounded sample: a row subset of W (decode), or a row subset
+    of X and of W (prefill), sized so that the whole run stays within minutes."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     import oracle
     from nvfp4_block_scaled_18_b200 import workloads as wl
     oracle.build()
-    budget = 150.0
+    budget = 120.0        # seconds of timed oracle work over warm-up and timed steps
     per_step = max(0.02, min(1.0, budget / max(1, args.steps + args.warmup)))
-    shapes = list(wl.DECODE_SHAPES)
-    Ms = list(wl.DECODE_M)
     cache = {}
+    # the W row subset of a step is sized by the oracle's cost per W element
+    # (dequantization to fp64 dominates): about 10 ns (decode), 20 ns (32 rows of X)
+    if args.workload == "decode":
+        shapes, Ms = list(wl.DECODE_SHAPES), list(wl.DECODE_M)
+        calls_per_step, unit, scale = len(shapes) * len(Ms), "GB/s", 1e9
 
-    def sample(i):
-        M, (N, K) = Ms[i % len(Ms)], shapes[(i // len(Ms)) % len(shapes)]
-        if (N, K) not in cache:
-            w = wl.weights_normal(N, K)
-            cache[(N, K)] = (oracle.quantize(w), w.shape[0])
-        qw, _ = cache[(N, K)]
-        # bound the work of a step: a row subset of W sized to the per-step budget
-        rows = max(8, min(N, int(per_step * 4e5 / max(1, K / 4096))))
-        sub = oracle.QTensor(qw.codes[:rows], qw.scales[:rows], qw.s)
-        x = wl.decode_x(M, K)
-        t0 = time.perf_counter()
-        oracle.gemm(oracle.quantize(x), sub)
-        return time.perf_counter() - t0, decode_bytes(M, rows, K)
+        def sample(i):
+            M, (N, K) = Ms[i % len(Ms)], shapes[(i // len(Ms)) % len(shapes)]
+            rows = max(8, min(N, int(per_step / (1e-8 * K))))
+            if (N, K) not in cache:      # the first rows of the workload's W
+                cache[(N, K)] = oracle.quantize(wl.weights_normal(rows, K))
+            sub = cache[(N, K)]
+            x = wl.decode_x(M, K)
+            t0 = time.perf_counter()
+            oracle.gemm(oracle.quantize(x), sub)
+            return time.perf_counter() - t0, decode_bytes(M, rows, K)
+        what = "one linear call per step (M 1..16 cycling over the shapes) on a W row subset"
+    else:
+        calls = [(N, K, S) for (N, K) in wl.PREFILL_SHAPES for S in (0, 256)]
+        calls_per_step, unit, scale = len(calls), "TFLOP/s", 1e12
+        x_rows = 32
+
+        def sample(i):
+            N, K, S = calls[i % len(calls)]
+            w_rows = max(16, min(N, int(per_step / (2e-8 * (K + S)))))
+            if (N, K, S) not in cache:   # the first rows of the workload's W
+                w = wl.weights_normal(w_rows, K)
+                if S:
+                    perm = wl.calibrated_perm(wl.prefill_x(64, K))
+                    cache[(N, K, S)] = (oracle.quantize(oracle.augment_weight(w, perm, S)), perm)
+                else:
+                    cache[(N, K, S)] = (oracle.quantize(w), None)
+            qw, perm = cache[(N, K, S)]
+            x = wl.prefill_x(x_rows, K)
+            t0 = time.perf_counter()
+            qx = oracle.rmsnorm_reorder_quantize(x, None, 1e-5, perm, S) if S else oracle.quantize(x)
+            oracle.gemm(qx, qw)
+            return time.perf_counter() - t0, 2.0 * x_rows * qw.codes.shape[0] * (K + S)
+        what = (f"one of the 6 prefill calls per step: {x_rows} rows of X (quantized, reordered for K+S) "
+                "against a W row subset")
 
     for i in range(args.warmup):
         sample(i)
-    t, b = 0.0, 0
+    t, work = 0.0, 0.0
     for i in range(args.steps):
-        dt, db = sample(i)
+        dt, dw = sample(i)
         t += dt
-        b += db
+        work += dw
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    value = b / t / 1e9
-    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
-            "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+    value = work / t / scale
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(t / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "decode GEMV, M=1..16, (N,K)=(4096,4096),(14336,4096),(4096,14336); "
-                                   "CPU oracle on a bounded row sample of W per step"},
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{args.steps} steps, each one linear call on a W row subset"},
-            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "config": arm_config(args.workload, world, calls_per_step),
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": f"{args.steps} steps, {what}; oracle quantize + fp64 dequantized GEMM"},
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -883,18 +923,11 @@ def main():
                               "where that is estimated faster), all 15 decode calls back to back",
                     "launches_per_step": wk.launches_per_step,
                     "peak_source": peaks["source"]}
-        config = {"workload": "decode GEMV (M in 1,2,4,8,16; (N,K) in (4096,4096),(14336,4096),(4096,14336)); "
-                              "online bf16->NVFP4 activation quantization + NVFP4 GEMM in one launch, fp32 out",
-                  "calls_per_step": len(wk.calls),
-                  "l2": "every call streams its own weight copy; >= 260 MB of copies per shape (> L2)",
-                  "parallelism": f"replicas x{world}"}
+        config = arm_config("decode", world, len(wk.calls))
         launches = wk.launches_per_step * steps
     else:
         detail, roofline = measure_prefill_from(wk, peaks)
-        config = {"workload": "large prefill W4A4 GEMM, M=8192, (N,K) in (14336,4096),(4096,14336),(28672,8192), "
-                              "each without and with the S=256 outlier-residue K extension; online quantization",
-                  "calls_per_step": len(wk.calls), "l2": "inputs > L2 (X 67-235 MB, Y 134-940 MB per call)",
-                  "parallelism": f"replicas x{world}"}
+        config = arm_config("prefill", world, len(wk.calls))
         launches = 3 * len(wk.calls) * steps
     line.update({"higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
                  "data": "synthetic", "config": config, "roofline": roofline,
