@@ -449,18 +449,56 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
       cp_async16(reinterpret_cast<uint4*>(dst) + c, reinterpret_cast<const uint4*>(xr) + c);
     cp_async_commit();
   };
+  // gamma goes to shared memory by cp.async in the first row's group (its
+  // pointer is 16-byte aligned and K * sizeof(T) a multiple of 16)
+  if (gamma)
+    for (int64_t c = threadIdx.x; c < row_bytes / 16; c += blockDim.x)
+      cp_async16(reinterpret_cast<uint4*>(sgamma) + c, reinterpret_cast<const uint4*>(gamma) + c);
   if ((int64_t)blockIdx.x < M) fetch_row(blockIdx.x, srow0);   // overlaps the table set-up
+  else cp_async_commit();
   const float s = *s_ptr;
   if (blockIdx.x == 0 && threadIdx.x == 0 && q.s != s_ptr) *q.s = s;
-  for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
-    int32_t p = perm ? perm[k] : (int32_t)k;
-    if (p < 0 || (int64_t)p >= K) {  // not a permutation of 0..K-1: report, never index out of range
-      report_status(st, NVFP4_ERR_INVALID_ARG);
-      p = 0;
+  // the permutation as 16-bit indices; an entry outside 0..K-1 is reported and
+  // replaced by 0, so no index is ever out of range
+  bool bad_perm = false;
+  if (perm != nullptr && (reinterpret_cast<uintptr_t>(perm) & 15u) == 0) {
+    // four 16-byte loads per thread in flight before any is used (K % 16 == 0)
+    constexpr int U = 4;
+    const int64_t n4 = K >> 2;
+    const uint4* p4 = reinterpret_cast<const uint4*>(perm);
+    for (int64_t c0 = threadIdx.x; c0 < n4; c0 += U * (int64_t)blockDim.x) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t c = c0 + u * (int64_t)blockDim.x;
+        v[u] = c < n4 ? __ldg(p4 + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t c = c0 + u * (int64_t)blockDim.x;
+        if (c < n4) {
+          uint32_t e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if ((uint64_t)e[i] >= (uint64_t)K) {   // also catches negative entries
+              bad_perm = true;
+              e[i] = 0u;
+            }
+          *reinterpret_cast<uint2*>(sperm + 4 * c) = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+        }
+      }
     }
-    sperm[k] = (uint16_t)p;
-    if (gamma) sgamma[k] = gamma[k];
+  } else {
+    for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
+      int32_t p = perm ? perm[k] : (int32_t)k;
+      if (p < 0 || (int64_t)p >= K) {
+        bad_perm = true;
+        p = 0;
+      }
+      sperm[k] = (uint16_t)p;
+    }
   }
+  if (bad_perm) report_status(st, NVFP4_ERR_INVALID_ARG);
   const int nb = (int)(K >> 4);     // blocks of the reordered row
   const int nbr = (int)(S >> 4);    // residue blocks (the first S reordered columns)
   uint32_t bad = 0;
@@ -684,8 +722,12 @@ cudaError_t launch_reorder_quant_t(const void* x, int64_t M, int64_t K, int64_t 
   cudaError_t e = cudaFuncSetAttribute(k_reorder_quant<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  // several CTAs per SM so that rows overlap
-  const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (220 * 1024) / (smem + 1024)));
+  // one wave of resident CTAs, several per SM so that rows overlap; a second
+  // wave would repeat the table set-up for only a few rows each
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_reorder_quant<T>, 256, smem);
+  if (e != cudaSuccess) return e;
+  per_sm = std::max(1, std::min(per_sm, 8));
   const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * per_sm));
   k_reorder_quant<T><<<g, 256, smem, stream>>>(static_cast<const T*>(x), M, K, ldx,
                                                static_cast<const T*>(gamma), rinv, perm, S, s_ptr,
