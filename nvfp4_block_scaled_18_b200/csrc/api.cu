@@ -203,8 +203,9 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64
     NVFP4_TRY(cuda_status(launch_amax(x, dt, M, K, ldx, ws, 0, x_aug->tensor_scale, dev_status, sms, s)));
   }
   const float* s_ptr = scale_in ? scale_in : x_aug->tensor_scale;
+  // a programmatic dependent of the statistics pass, when there is one
   return cuda_status(launch_reorder_quant(x, dt, M, K, ldx, gamma, rinv, perm, S, s_ptr, qout(x_aug),
-                                          dev_status, sms, s));
+                                          dev_status, sms, s, gamma != nullptr || scale_in == nullptr));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt,

@@ -45,7 +45,7 @@ size_t reorder_smem_bytes(nvfp4_dtype dt, int64_t K, bool has_gamma);
 cudaError_t launch_reorder_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                  const void* gamma, const float* rinv, const int32_t* perm,
                                  int64_t S, const float* s_ptr, const QOut& q, int* st, int num_sms,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, bool after_stats);
 
 // Operands of the decode GEMV / tensor-core GEMM.
 struct GemmArgs {

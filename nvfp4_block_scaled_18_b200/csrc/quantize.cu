@@ -328,6 +328,7 @@ __global__ void __launch_bounds__(256) k_rms_stats(const T* __restrict__ x, int6
                                                    float* s_out, bool want_scale, int* st) {
   __shared__ uint32_t redu[32];
   __shared__ double redd[32];
+  tc::griddep_launch_dependents();   // the reorder pass may launch; it waits for this grid's results
   const int64_t upr = K >> 3;
   uint32_t ykey = 0, bad = 0;
   // unit c8 of the row: NC > 0 -> c8 = threadIdx.x + 256 n, n < NC
@@ -456,8 +457,6 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
       cp_async16(reinterpret_cast<uint4*>(sgamma) + c, reinterpret_cast<const uint4*>(gamma) + c);
   if ((int64_t)blockIdx.x < M) fetch_row(blockIdx.x, srow0);   // overlaps the table set-up
   else cp_async_commit();
-  const float s = *s_ptr;
-  if (blockIdx.x == 0 && threadIdx.x == 0 && q.s != s_ptr) *q.s = s;
   // the permutation as 16-bit indices; an entry outside 0..K-1 is reported and
   // replaced by 0, so no index is ever out of range
   bool bad_perm = false;
@@ -499,6 +498,11 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
     }
   }
   if (bad_perm) report_status(st, NVFP4_ERR_INVALID_ARG);
+  // X, gamma and perm are inputs of the call; the tensor scale and the row
+  // factors come from the statistics pass, which may still be running
+  tc::griddep_wait();
+  const float s = *s_ptr;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && q.s != s_ptr) *q.s = s;
   const int nb = (int)(K >> 4);     // blocks of the reordered row
   const int nbr = (int)(S >> 4);    // residue blocks (the first S reordered columns)
   uint32_t bad = 0;
@@ -717,7 +721,7 @@ template <typename T>
 cudaError_t launch_reorder_quant_t(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
                                    const float* rinv, const int32_t* perm, int64_t S,
                                    const float* s_ptr, const QOut& q, int* st, int num_sms,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, bool after_stats) {
   const size_t smem = reorder_smem_bytes(sizeof(T) == 2 ? NVFP4_BF16 : NVFP4_F32, K, gamma != nullptr);
   cudaError_t e = cudaFuncSetAttribute(k_reorder_quant<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -729,19 +733,29 @@ cudaError_t launch_reorder_quant_t(const void* x, int64_t M, int64_t K, int64_t 
   if (e != cudaSuccess) return e;
   per_sm = std::max(1, std::min(per_sm, 8));
   const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * per_sm));
-  k_reorder_quant<T><<<g, 256, smem, stream>>>(static_cast<const T*>(x), M, K, ldx,
-                                               static_cast<const T*>(gamma), rinv, perm, S, s_ptr,
-                                               q, st);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // after the statistics pass only
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_stats ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_reorder_quant<T>, static_cast<const T*>(x), M, K, ldx,
+                            static_cast<const T*>(gamma), rinv, perm, S, s_ptr, q, st);
 }
 
 cudaError_t launch_reorder_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                  const void* gamma, const float* rinv, const int32_t* perm,
                                  int64_t S, const float* s_ptr, const QOut& q, int* st, int num_sms,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, bool after_stats) {
   return dt == NVFP4_BF16
-             ? launch_reorder_quant_t<__nv_bfloat16>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms, stream)
-             : launch_reorder_quant_t<float>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms, stream);
+             ? launch_reorder_quant_t<__nv_bfloat16>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms,
+                                                     stream, after_stats)
+             : launch_reorder_quant_t<float>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms, stream,
+                                             after_stats);
 }
 
 }  // namespace nvfp4
