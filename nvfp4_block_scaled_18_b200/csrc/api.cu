@@ -196,6 +196,12 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64
   const int sms = num_sms_current_device();
   WsHeader* ws = static_cast<WsHeader*>(workspace);
   float* rinv = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeaderBytes) : nullptr;
+  if (gamma != nullptr || scale_in == nullptr) {
+    // small enough for one launch: X read once, no second pass
+    const cudaError_t e = launch_reorder_onepass(x, dt, M, K, ldx, gamma, eps, perm, S, scale_in, qout(x_aug), ws,
+                                                 dev_status, sms, s);
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+  }
   if (gamma != nullptr) {
     NVFP4_TRY(cuda_status(launch_rms_stats(x, dt, M, K, ldx, gamma, eps, ws, rinv, x_aug->tensor_scale,
                                            scale_in == nullptr, dev_status, sms, s)));

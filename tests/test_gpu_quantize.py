@@ -278,3 +278,32 @@ def test_nonfinite_reported_multi_launch():
     torch.cuda.synchronize()
     assert st.item() == 5
     assert int(ws.buf.count_nonzero()) == 0
+
+
+# ------------------------------- ARCQuant quantizer: one launch or two passes
+
+# X that fits in the shared memory of one wave of CTAs is quantized by one
+# cooperative launch (rows read once, one grid-wide exchange of the maximum);
+# larger X by the statistics pass and the reorder pass.  Both must give the
+# oracle's codes and scales bit for bit and leave the workspace header zeroed.
+@pytest.mark.parametrize("M,K,norm,given", [(2048, 4096, True, False), (2048, 4096, True, True),
+                                            (2048, 4096, False, False), (3000, 4096, True, False),
+                                            (8192, 4096, True, False), (5, 512, True, False)])
+def test_reorder_one_launch_and_two_pass(orc, M, K, norm, given):
+    S = 256 if K >= 256 else 0
+    ch = wl.outlier_channels(K, 0.02)
+    x = wl.bf16_values(wl.activations_normal(M, K, 0.02, 30.0, wl.SEED_X, ch))
+    gamma = wl.bf16_values(wl.gamma_uniform(K)) if norm else None
+    perm = wl.calibrated_perm(wl.activations_normal(64, K, 0.02, 30.0, wl.SEED_CALIB, ch))
+    s_given = np.float32(0.05) if given else None
+    xa = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED)
+    ws = nv.Workspace(M, K)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_rmsnorm_reorder_quantize(
+        to_dev(x), xa, gamma=to_dev(gamma) if norm else None, eps=1e-5, perm=torch.from_numpy(perm).cuda(), S=S,
+        scale_in=torch.tensor([s_given], dtype=torch.float32, device="cuda") if given else None,
+        workspace=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0 and int(ws.buf[:256].count_nonzero()) == 0
+    ref = orc.rmsnorm_reorder_quantize(x, gamma, 1e-5, perm, S, s=s_given)
+    assert_same_q(xa, ref, f"M={M} K={K}")
