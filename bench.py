@@ -760,7 +760,9 @@ def profile_case(case: str) -> int:
     prefill  -- nvfp4_gemm, M=8192, (N,K)=(14336,4096) (A 19 MB, W 33 MB, Y 470 MB)
     quantize -- nvfp4_quantize of the 8192x4096 bf16 prefill activations (67 MB)
     reorder  -- nvfp4_rmsnorm_reorder_quantize of the same activations, S=256
-    mxgemm   -- nvfp4_mx_gemm, M=8192, (N,K)=(14336,4096), MXFP4 operands with TILED scales."""
+    mxgemm   -- nvfp4_mx_gemm, M=8192, (N,K)=(14336,4096), MXFP4 operands with TILED scales
+    arcquant -- nvfp4_rmsnorm_reorder_quantize on the ARCQuant prefill activations
+                (2048x4096 bf16, gamma, calibrated perm, S=256)."""
     import nvfp4_block_scaled_18_b200 as nv
     from nvfp4_block_scaled_18_b200 import workloads as wl
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -800,6 +802,16 @@ def profile_case(case: str) -> int:
         y = torch.empty((M, N), device=dev)
         for _ in range(3):
             nv.nvfp4_mx_gemm(ops[0][0], ops[0][1], ops[1][0], ops[1][1], y)
+    elif case == "arcquant":
+        x, gamma, perm = wl.arc_inputs()
+        M, K, S = wl.ARC_M, wl.ARC_K, 256
+        xs = [wl.to_bf16(x).to(dev) for _ in range(8)]   # 134 MB of activation copies (> L2)
+        g = wl.to_bf16(gamma).to(dev)
+        p = torch.from_numpy(np.ascontiguousarray(perm, dtype=np.int32)).to(dev)
+        q = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED, device=dev)
+        ws = nv.Workspace(M, K, dev)
+        for i in range(3):
+            nv.nvfp4_rmsnorm_reorder_quantize(xs[i], q, gamma=g, eps=1e-5, perm=p, S=S, workspace=ws)
     elif case == "reorder":
         M, K, S = 8192, 4096, 256
         x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
@@ -834,7 +846,7 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="decode: launch every step directly on the stream (no CUDA graphs) and skip the "
                          "per-call detail; for profilers that cannot follow graph replays")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder", "mxgemm"],
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder", "mxgemm", "arcquant"],
                     help="run a few launches of one kernel on a small case (for ncu captures) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
