@@ -588,10 +588,22 @@ def measure_prefill_from(wk, peaks):
                              "GBps": round(mx_bytes / (t_mx * 1e-3) / 1e9, 1),
                              "residue_us": round(t_mxr * 1e3, 2),
                              "residue_GBps": round((mx_bytes + M * K * (0.5 + 1 / 32)) / (t_mxr * 1e-3) / 1e9, 1)}
+    nv = wk.nv
+    # ResServe residue on the large-M GEMM (two accumulation passes per tile) on the same shape
+    q_r = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=x.device)
+    r_r = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=x.device)
+    nv.nvfp4_quantize_residue(x, q_r, r_r, workspace=wk.buf[(N, K)]["ws"])
+    qw_r, y_r = wk.buf[(N, K)]["qw"], wk.buf[(N, K)]["y"]
+    t_p = time_back_to_back(lambda i: nv.nvfp4_gemm(q_r, qw_r, y_r), 4)
+    t_r = time_back_to_back(lambda i: nv.nvfp4_gemm_residue(q_r, r_r, qw_r, y_r), 4)
+    out["resserve_gemm"] = {"shape": f"M{M}_N{N}_K{K}", "plain_us": round(t_p * 1e3, 2),
+                            "residue_us": round(t_r * 1e3, 2),
+                            "overhead_pct": round(100.0 * (t_r / t_p - 1.0), 1),
+                            "residue_TFLOPs": round(4.0 * M * N * K / (t_r * 1e-3) / 1e12, 1)}
+    del q_r, r_r
     # MXFP4 GEMM (kind::mxf4, one E8M0 scale per 32 elements) on the same shape:
     # both operands quantized on the device with TILED scales
     from nvfp4_block_scaled_18_b200 import workloads as wl
-    nv = wk.nv
     w = torch.from_numpy(wl.weights_normal(N, K)).to(x.device)
     wc = torch.empty((N, K // 2), dtype=torch.uint8, device=x.device)
     wsc = torch.empty(nv.mx_scales_bytes(N, K, nv.SF_TILED), dtype=torch.uint8, device=x.device)

@@ -148,8 +148,12 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y,
 
 /* ResServe compensated linear (ResServe abstract):
  *   Y = s_a s_w * A W^T + s_r s_w * R W^T,
- * both products accumulated on-chip and written once.  a and r are M x K,
- * w is N x K.  Other conventions as nvfp4_gemm. */
+ * both products accumulated on-chip and written once.  a and r are M x K (same
+ * scale layout), w is N x K.  M <= 128 runs the decode / few-row kernels with
+ * a second accumulator fed by the same W tiles; M > 128 (TILED scales) runs the
+ * 128x256-tile GEMM with two accumulation passes per tile, A W^T then R W^T,
+ * the first held in registers until the second is added.  Other conventions
+ * as nvfp4_gemm. */
 nvfp4_status nvfp4_gemm_residue(const nvfp4_tensor* a, const nvfp4_tensor* r,
                                 const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt, int64_t ldy,
                                 int* dev_status, void* stream);

@@ -106,7 +106,7 @@ nvfp4_status run_gemm(const nvfp4_tensor* a, const nvfp4_tensor* r, const nvfp4_
     e = launch_decode_tc(d, num_sms_current_device(), s);
   } else if (tiled && g.M <= 128) {
     e = launch_gemv_tc(g, num_sms_current_device(), s);           // tensor cores, operands swapped
-  } else if (tiled && r == nullptr) {
+  } else if (tiled) {
     e = launch_gemm_tc(g, num_sms_current_device(), s);           // tensor cores, 128x256 tiles
   } else {
     return NVFP4_ERR_UNSUPPORTED;
