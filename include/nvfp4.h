@@ -260,6 +260,17 @@ nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, cons
                            const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* y,
                            nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
 
+/* MXFP4 compensated linear (ResServe abstract: FP4 base plus FP4 residue; its
+ * largest gains are reported for MXFP4): Y = deq(A) deq(W)^T + deq(R) deq(W)^T,
+ * with (r_codes, r_scales) the residue from nvfp4_mx_quantize (TILED scales).
+ * MX has no tensor scales, so the residue's K-tiles continue the same fp32
+ * accumulation, Y = [A | R] [W | W]^T, written once.  Requirements and
+ * conventions as nvfp4_mx_gemm; r_codes and r_scales must not be NULL. */
+nvfp4_status nvfp4_mx_gemm_residue(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* r_codes,
+                                   const uint8_t* r_scales, const uint8_t* w_codes, const uint8_t* w_scales,
+                                   int64_t M, int64_t N, int64_t K, void* y, nvfp4_dtype out_dt, int64_t ldy,
+                                   int* dev_status, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* nvfp4_status_string(nvfp4_status status);
 

@@ -115,6 +115,31 @@ nvfp4_status run_gemm(const nvfp4_tensor* a, const nvfp4_tensor* r, const nvfp4_
   return cuda_status(e);
 }
 
+nvfp4_status run_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* r_codes,
+                         const uint8_t* r_scales, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M,
+                         int64_t N, int64_t K, void* y, nvfp4_dtype out_dt, int64_t ldy, int* dev_status,
+                         void* stream) {
+  if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr || y == nullptr ||
+      !dt_ok(out_dt))
+    return NVFP4_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || ldy < N || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
+    return NVFP4_ERR_INVALID_ARG;
+  if (K % 128 != 0 || K < 256) return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(a_scales) || !aligned16(w_scales))
+    return NVFP4_ERR_ALIGNMENT;
+  if (r_codes != nullptr && (!aligned16(r_codes) || !aligned16(r_scales))) return NVFP4_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(y) % dt_size(out_dt)) != 0) return NVFP4_ERR_ALIGNMENT;
+  GemmArgs g{};
+  g.a_codes = a_codes; g.a_scales = a_scales;
+  g.r_codes = r_codes; g.r_scales = r_scales;
+  g.w_codes = w_codes; g.w_scales = w_scales;
+  g.y = y; g.ldy = ldy; g.y_bf16 = out_dt == NVFP4_BF16;
+  g.M = M; g.N = N; g.K = K; g.st = dev_status;
+  const cudaError_t e = launch_gemm_mx(g, num_sms_current_device(), static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -312,23 +337,17 @@ nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t
 nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
                            const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* y,
                            nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream) {
-  if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr || y == nullptr ||
-      !dt_ok(out_dt))
-    return NVFP4_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0 || ldy < N || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
-    return NVFP4_ERR_INVALID_ARG;
-  if (K % 128 != 0 || K < 256) return NVFP4_ERR_UNSUPPORTED;
-  if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(a_scales) || !aligned16(w_scales))
-    return NVFP4_ERR_ALIGNMENT;
-  if ((reinterpret_cast<uintptr_t>(y) % dt_size(out_dt)) != 0) return NVFP4_ERR_ALIGNMENT;
-  GemmArgs g{};
-  g.a_codes = a_codes; g.a_scales = a_scales;
-  g.w_codes = w_codes; g.w_scales = w_scales;
-  g.y = y; g.ldy = ldy; g.y_bf16 = out_dt == NVFP4_BF16;
-  g.M = M; g.N = N; g.K = K; g.st = dev_status;
-  const cudaError_t e = launch_gemm_mx(g, num_sms_current_device(), static_cast<cudaStream_t>(stream));
-  if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
-  return cuda_status(e);
+  return run_mx_gemm(a_codes, a_scales, nullptr, nullptr, w_codes, w_scales, M, N, K, y, out_dt, ldy, dev_status,
+                     stream);
+}
+
+nvfp4_status nvfp4_mx_gemm_residue(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* r_codes,
+                                   const uint8_t* r_scales, const uint8_t* w_codes, const uint8_t* w_scales,
+                                   int64_t M, int64_t N, int64_t K, void* y, nvfp4_dtype out_dt, int64_t ldy,
+                                   int* dev_status, void* stream) {
+  if (r_codes == nullptr || r_scales == nullptr) return NVFP4_ERR_INVALID_ARG;
+  return run_mx_gemm(a_codes, a_scales, r_codes, r_scales, w_codes, w_scales, M, N, K, y, out_dt, ldy, dev_status,
+                     stream);
 }
 
 const char* nvfp4_status_string(nvfp4_status st) {

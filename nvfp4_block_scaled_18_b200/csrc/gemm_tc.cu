@@ -95,15 +95,18 @@ struct TcParams {
 // same stages, with the scale atoms covering K = 128 each, so half of each
 // stage's scale area and of its TMEM scale buffer is used.
 // RES: ResServe's full residue (Y = s_a s_w A W^T + s_r s_w R W^T).  Each tile
-// runs two accumulation passes into the same TMEM accumulator, A W^T and then
-// R W^T (the residue as a second run of K-tiles over the same W tiles); the
-// epilogue holds s_a s_w acc in registers while the second pass runs and adds
-// s_r s_w acc before the single store of Y.
+// runs two passes over its K-tiles, A W^T and then R W^T (the residue as a
+// second run of K-tiles over the same W tiles).  NVFP4: two uses of the TMEM
+// accumulator; the epilogue holds s_a s_w acc in registers while the second
+// pass runs and adds s_r s_w acc before the single store of Y.  MXFP4 has no
+// tensor scales, so the residue's K-tiles simply continue the same
+// accumulation: Y = [A | R] [W | W]^T.
 template <bool BF16OUT, bool MX, bool RES = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmR, const TcParams p) {
-  constexpr int NPASS = RES ? 2 : 1;   // accumulation passes per tile
+  constexpr int NPASS = RES ? 2 : 1;            // passes over the K-tiles per tile
+  constexpr int NUSE = (RES && !MX) ? 2 : 1;    // accumulator uses per tile
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* epi = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
@@ -236,9 +239,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local)
       for (int pass = 0; pass < NPASS; ++pass) {
         // accumulator use u: the epilogue has taken use u - 1 out of TMEM
-        const int u = NPASS * local + pass;
-        if (!mbar_wait_inline(saddr(acc_empty), (uint32_t)(u & 1) ^ 1u, abort_flag, p.st)) goto mma_done;
-        tc_fence_after();
+        const bool fresh = NUSE == 2 || pass == 0;   // this pass starts a use of the accumulator
+        const int u = NUSE * local + (NUSE == 2 ? pass : 0);
+        if (fresh) {
+          if (!mbar_wait_inline(saddr(acc_empty), (uint32_t)(u & 1) ^ 1u, abort_flag, p.st)) goto mma_done;
+          tc_fence_after();
+        }
         for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
           const int s = g % STAGES;
           const uint32_t ph = (uint32_t)((g / STAGES) & 1);
@@ -253,14 +259,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if constexpr (MX)   // K = 64 chunk j: atom j / 2, scale bytes 2 (j % 2) and 2 (j % 2) + 1
               tc_mma_mxf4(tmem + ACC_COL, da + (uint64_t)(2 * j), db + (uint64_t)(2 * j),
                           idesc_mxf4(BN, 2u * (uint32_t)(j & 1)), tmem + buf + 4 * (j >> 1),
-                          tmem + buf + 8 + 8 * (j >> 1), (kt > 0 || j > 0) ? 1u : 0u);
+                          tmem + buf + 8 + 8 * (j >> 1), (!fresh || kt > 0 || j > 0) ? 1u : 0u);
             else
               tc_mma_nvf4(tmem + ACC_COL, da + (uint64_t)(2 * j), db + (uint64_t)(2 * j), idesc, tmem + buf + 4 * j,
-                          tmem + buf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                          tmem + buf + 16 + 8 * j, (!fresh || kt > 0 || j > 0) ? 1u : 0u);
           }
           tc_commit(saddr(&empty[s]));
         }
-        tc_commit(saddr(acc_full));
+        if (NUSE == 2 || pass == NPASS - 1) tc_commit(saddr(acc_full));
       }
     mma_done:;
     }
@@ -273,11 +279,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int sub_r = lane >> 1, sub_c = (lane & 1) * 4;
     int local = 0;
     const float alpha = MX ? 1.0f : (*p.a_s) * (*p.w_s);   // MXFP4 has no tensor scales
-    const float alpha_r = RES ? (*p.r_s) * (*p.w_s) : 0.0f;
-    const float out_scale = RES ? 1.0f : alpha;              // RES: the registers hold the combined Y
+    const float alpha_r = NUSE == 2 ? (*p.r_s) * (*p.w_s) : 0.0f;
+    const float out_scale = NUSE == 2 ? 1.0f : alpha;        // two uses: the registers hold the combined Y
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
       const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
-      if (!mbar_wait_inline(saddr(acc_full), (uint32_t)((NPASS * local) & 1), abort_flag, p.st)) break;
+      if (!mbar_wait_inline(saddr(acc_full), (uint32_t)((NUSE * local) & 1), abort_flag, p.st)) break;
       tc_fence_after();
       // Each warp owns TMEM lanes (= tile rows) 32q..32q+31 and columns
       // [128 half, 128 half + 128): read them all, then free the accumulator.
@@ -289,13 +295,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(saddr(acc_empty));
-      if constexpr (RES) {
+      if constexpr (NUSE == 2) {
         // s_a s_w acc1 stays in registers; add s_r s_w acc2 column chunk by column chunk
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i) r[c][i] = __float_as_uint(__uint_as_float(r[c][i]) * alpha);
-        if (!mbar_wait_inline(saddr(acc_full), (uint32_t)((NPASS * local + 1) & 1), abort_flag, p.st)) break;
+        if (!mbar_wait_inline(saddr(acc_full), (uint32_t)((NUSE * local + 1) & 1), abort_flag, p.st)) break;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < BN / 64; ++c) {
@@ -397,8 +403,7 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
 
 template <bool MX>
 cudaError_t launch_gemm_impl(const GemmArgs& g, int num_sms, cudaStream_t stream) {
-  const bool res = g.r_codes != nullptr;   // ResServe residue: a second accumulation pass per tile
-  if (MX && res) return cudaErrorNotSupported;
+  const bool res = g.r_codes != nullptr;   // ResServe residue: a second pass over the K-tiles
   if (MX ? (g.K % 128 != 0 || g.K < BK) : (g.K % 64 != 0 || g.K < BK)) return cudaErrorNotSupported;
   // sizes, tile coordinates and the tile count are 32-bit in the kernel
   if (g.M > INT32_MAX || g.N > INT32_MAX || g.K > INT32_MAX ||
@@ -425,7 +430,7 @@ cudaError_t launch_gemm_impl(const GemmArgs& g, int num_sms, cudaStream_t stream
   p.num_tiles = p.m_blocks * p.n_blocks;
   p.k_tiles = (int)((g.K + BK - 1) / BK);
   p.st = g.st;
-  auto kern = res ? (g.y_bf16 ? k_gemm_nvf4<true, false, true> : k_gemm_nvf4<false, false, true>)
+  auto kern = res ? (g.y_bf16 ? k_gemm_nvf4<true, MX, true> : k_gemm_nvf4<false, MX, true>)
                   : (g.y_bf16 ? k_gemm_nvf4<true, MX> : k_gemm_nvf4<false, MX>);
   // the register split assumes the launch allocates LAUNCH_REGS per thread
   cudaFuncAttributes fa{};
