@@ -616,7 +616,14 @@ def measure_prefill_from(wk, peaks):
     out["mxfp4_gemm"] = {"shape": f"M{M}_N{N}_K{K}", "us": round(t_mg * 1e3, 2),
                          "TFLOPs": round(2.0 * M * N * K / (t_mg * 1e-3) / 1e12, 1),
                          "frac_fp4_peak": round(2.0 * M * N * K / (t_mg * 1e-3) / 1e12 / fp4_peak_tflops(peaks), 4)}
-    del wc, wsc, xsc
+    # the compensated MXFP4 linear: X with its residue, the residue's K-tiles in the same accumulation
+    rsc = torch.empty_like(xsc)
+    nv.nvfp4_mx_quantize(x, mc, xsc, rc, rsc, sf_layout=nv.SF_TILED)
+    t_mgr = time_back_to_back(lambda i: nv.nvfp4_mx_gemm_residue(mc.view(M, -1), xsc, rc.view(M, -1), rsc, wc, wsc,
+                                                                 y), 4)
+    out["mxfp4_gemm"].update({"residue_us": round(t_mgr * 1e3, 2),
+                              "residue_overhead_pct": round(100.0 * (t_mgr / t_mg - 1.0), 1)})
+    del wc, wsc, xsc, rsc
     try:
         out["arcquant_prefill"] = measure_arcquant(nv, x.device, peaks)
     except Exception as e:   # a detail leg: record the failure, keep the line
