@@ -588,10 +588,22 @@ def measure_prefill_from(wk, peaks):
                              "GBps": round(mx_bytes / (t_mx * 1e-3) / 1e9, 1),
                              "residue_us": round(t_mxr * 1e3, 2),
                              "residue_GBps": round((mx_bytes + M * K * (0.5 + 1 / 32)) / (t_mxr * 1e-3) / 1e9, 1)}
+    nv = wk.nv
+    # ResServe residue on the large-M GEMM (two accumulation passes per tile) on the same shape
+    q_r = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=x.device)
+    r_r = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=x.device)
+    nv.nvfp4_quantize_residue(x, q_r, r_r, workspace=wk.buf[(N, K)]["ws"])
+    qw_r, y_r = wk.buf[(N, K)]["qw"], wk.buf[(N, K)]["y"]
+    t_p = time_back_to_back(lambda i: nv.nvfp4_gemm(q_r, qw_r, y_r), 4)
+    t_r = time_back_to_back(lambda i: nv.nvfp4_gemm_residue(q_r, r_r, qw_r, y_r), 4)
+    out["resserve_gemm"] = {"shape": f"M{M}_N{N}_K{K}", "plain_us": round(t_p * 1e3, 2),
+                            "residue_us": round(t_r * 1e3, 2),
+                            "overhead_pct": round(100.0 * (t_r / t_p - 1.0), 1),
+                            "residue_TFLOPs": round(4.0 * M * N * K / (t_r * 1e-3) / 1e12, 1)}
+    del q_r, r_r
     # MXFP4 GEMM (kind::mxf4, one E8M0 scale per 32 elements) on the same shape:
     # both operands quantized on the device with TILED scales
     from nvfp4_block_scaled_18_b200 import workloads as wl
-    nv = wk.nv
     w = torch.from_numpy(wl.weights_normal(N, K)).to(x.device)
     wc = torch.empty((N, K // 2), dtype=torch.uint8, device=x.device)
     wsc = torch.empty(nv.mx_scales_bytes(N, K, nv.SF_TILED), dtype=torch.uint8, device=x.device)
@@ -604,7 +616,14 @@ def measure_prefill_from(wk, peaks):
     out["mxfp4_gemm"] = {"shape": f"M{M}_N{N}_K{K}", "us": round(t_mg * 1e3, 2),
                          "TFLOPs": round(2.0 * M * N * K / (t_mg * 1e-3) / 1e12, 1),
                          "frac_fp4_peak": round(2.0 * M * N * K / (t_mg * 1e-3) / 1e12 / fp4_peak_tflops(peaks), 4)}
-    del wc, wsc, xsc
+    # the compensated MXFP4 linear: X with its residue, the residue's K-tiles in the same accumulation
+    rsc = torch.empty_like(xsc)
+    nv.nvfp4_mx_quantize(x, mc, xsc, rc, rsc, sf_layout=nv.SF_TILED)
+    t_mgr = time_back_to_back(lambda i: nv.nvfp4_mx_gemm_residue(mc.view(M, -1), xsc, rc.view(M, -1), rsc, wc, wsc,
+                                                                 y), 4)
+    out["mxfp4_gemm"].update({"residue_us": round(t_mgr * 1e3, 2),
+                              "residue_overhead_pct": round(100.0 * (t_mgr / t_mg - 1.0), 1)})
+    del wc, wsc, xsc, rsc
     try:
         out["arcquant_prefill"] = measure_arcquant(nv, x.device, peaks)
     except Exception as e:   # a detail leg: record the failure, keep the line
@@ -760,7 +779,9 @@ def profile_case(case: str) -> int:
     prefill  -- nvfp4_gemm, M=8192, (N,K)=(14336,4096) (A 19 MB, W 33 MB, Y 470 MB)
     quantize -- nvfp4_quantize of the 8192x4096 bf16 prefill activations (67 MB)
     reorder  -- nvfp4_rmsnorm_reorder_quantize of the same activations, S=256
-    mxgemm   -- nvfp4_mx_gemm, M=8192, (N,K)=(14336,4096), MXFP4 operands with TILED scales."""
+    mxgemm   -- nvfp4_mx_gemm, M=8192, (N,K)=(14336,4096), MXFP4 operands with TILED scales
+    arcquant -- nvfp4_rmsnorm_reorder_quantize on the ARCQuant prefill activations
+                (2048x4096 bf16, gamma, calibrated perm, S=256)."""
     import nvfp4_block_scaled_18_b200 as nv
     from nvfp4_block_scaled_18_b200 import workloads as wl
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -800,6 +821,16 @@ def profile_case(case: str) -> int:
         y = torch.empty((M, N), device=dev)
         for _ in range(3):
             nv.nvfp4_mx_gemm(ops[0][0], ops[0][1], ops[1][0], ops[1][1], y)
+    elif case == "arcquant":
+        x, gamma, perm = wl.arc_inputs()
+        M, K, S = wl.ARC_M, wl.ARC_K, 256
+        xs = [wl.to_bf16(x).to(dev) for _ in range(8)]   # 134 MB of activation copies (> L2)
+        g = wl.to_bf16(gamma).to(dev)
+        p = torch.from_numpy(np.ascontiguousarray(perm, dtype=np.int32)).to(dev)
+        q = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED, device=dev)
+        ws = nv.Workspace(M, K, dev)
+        for i in range(3):
+            nv.nvfp4_rmsnorm_reorder_quantize(xs[i], q, gamma=g, eps=1e-5, perm=p, S=S, workspace=ws)
     elif case == "reorder":
         M, K, S = 8192, 4096, 256
         x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
@@ -834,7 +865,7 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="decode: launch every step directly on the stream (no CUDA graphs) and skip the "
                          "per-call detail; for profilers that cannot follow graph replays")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder", "mxgemm"],
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder", "mxgemm", "arcquant"],
                     help="run a few launches of one kernel on a small case (for ncu captures) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

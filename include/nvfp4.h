@@ -148,8 +148,12 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y,
 
 /* ResServe compensated linear (ResServe abstract):
  *   Y = s_a s_w * A W^T + s_r s_w * R W^T,
- * both products accumulated on-chip and written once.  a and r are M x K,
- * w is N x K.  Other conventions as nvfp4_gemm. */
+ * both products accumulated on-chip and written once.  a and r are M x K (same
+ * scale layout), w is N x K.  M <= 128 runs the decode / few-row kernels with
+ * a second accumulator fed by the same W tiles; M > 128 (TILED scales) runs the
+ * 128x256-tile GEMM with two accumulation passes per tile, A W^T then R W^T,
+ * the first held in registers until the second is added.  Other conventions
+ * as nvfp4_gemm. */
 nvfp4_status nvfp4_gemm_residue(const nvfp4_tensor* a, const nvfp4_tensor* r,
                                 const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt, int64_t ldy,
                                 int* dev_status, void* stream);
@@ -255,6 +259,17 @@ size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout)
 nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
                            const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* y,
                            nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
+
+/* MXFP4 compensated linear (ResServe abstract: FP4 base plus FP4 residue; its
+ * largest gains are reported for MXFP4): Y = deq(A) deq(W)^T + deq(R) deq(W)^T,
+ * with (r_codes, r_scales) the residue from nvfp4_mx_quantize (TILED scales).
+ * MX has no tensor scales, so the residue's K-tiles continue the same fp32
+ * accumulation, Y = [A | R] [W | W]^T, written once.  Requirements and
+ * conventions as nvfp4_mx_gemm; r_codes and r_scales must not be NULL. */
+nvfp4_status nvfp4_mx_gemm_residue(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* r_codes,
+                                   const uint8_t* r_scales, const uint8_t* w_codes, const uint8_t* w_scales,
+                                   int64_t M, int64_t N, int64_t K, void* y, nvfp4_dtype out_dt, int64_t ldy,
+                                   int* dev_status, void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* nvfp4_status_string(nvfp4_status status);

@@ -28,7 +28,7 @@ EXPORTED_SYMBOLS = ("nvfp4_scales_bytes", "nvfp4_workspace_size", "nvfp4_quantiz
                     "nvfp4_gemm_residue", "nvfp4_quantize_gemm", "nvfp4_quantize_residue_gemm",
                     "nvfp4_quantize_gemm_plan",
                     "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_mx_quantize",
-                    "nvfp4_mx_scales_bytes", "nvfp4_mx_gemm", "nvfp4_status_string", "nvfp4_version")
+                    "nvfp4_mx_scales_bytes", "nvfp4_mx_gemm", "nvfp4_mx_gemm_residue", "nvfp4_status_string", "nvfp4_version")
 NVFP4_NOALLOC_MAX_ROWS = 65536
 
 
@@ -77,9 +77,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.nvfp4_mx_scales_bytes.argtypes = [I64, I64, ctypes.c_int]
         lib.nvfp4_mx_scales_bytes.restype = SZ
         lib.nvfp4_mx_gemm.argtypes = [P, P, P, P, I64, I64, I64, P, ctypes.c_int, I64, P, P]
+        lib.nvfp4_mx_gemm_residue.argtypes = [P, P, P, P, P, P, I64, I64, I64, P, ctypes.c_int, I64, P, P]
         for fn in ("nvfp4_quantize", "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize",
                    "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_gemm", "nvfp4_gemm_residue",
-                   "nvfp4_mx_quantize", "nvfp4_mx_gemm"):
+                   "nvfp4_mx_quantize", "nvfp4_mx_gemm", "nvfp4_mx_gemm_residue"):
             getattr(lib, fn).restype = ctypes.c_int
         lib.nvfp4_status_string.argtypes = [ctypes.c_int]
         lib.nvfp4_status_string.restype = ctypes.c_char_p
@@ -213,22 +214,44 @@ def nvfp4_mx_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor
            "nvfp4_mx_quantize")
 
 
+def _mx_gemm_checks(a_codes, a_scales, w_codes, w_scales, y, where, r_codes=None, r_scales=None):
+    M, N, K = a_codes.shape[0], w_codes.shape[0], 2 * a_codes.shape[1]
+    if w_codes.shape[1] * 2 != K or tuple(y.shape) != (M, N):
+        raise ValueError(f"{where}: shapes do not match")
+    ops = [(a_codes, M * K // 2), (w_codes, N * K // 2),
+           (a_scales, mx_scales_bytes(M, K, SF_TILED)), (w_scales, mx_scales_bytes(N, K, SF_TILED))]
+    if r_codes is not None:
+        ops += [(r_codes, M * K // 2), (r_scales, mx_scales_bytes(M, K, SF_TILED))]
+    for t, n in ops:
+        if t.dtype != torch.uint8 or t.numel() != n or not t.is_contiguous():
+            raise ValueError(f"{where}: operands must be contiguous uint8 of the MXFP4 sizes")
+    return M, N, K
+
+
 def nvfp4_mx_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, w_codes: torch.Tensor,
                   w_scales: torch.Tensor, y: torch.Tensor,
                   dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
     """MXFP4 linear y = deq(A) deq(W)^T: a_codes uint8 [M, K/2], w_codes uint8
     [N, K/2], both scale buffers in the TILED layout; y [M, N] fp32 or bf16."""
     lib = load_library()
-    M, N, K = a_codes.shape[0], w_codes.shape[0], 2 * a_codes.shape[1]
-    if w_codes.shape[1] * 2 != K or tuple(y.shape) != (M, N):
-        raise ValueError("nvfp4_mx_gemm: shapes do not match")
-    for t, n in ((a_codes, M * K // 2), (w_codes, N * K // 2),
-                 (a_scales, mx_scales_bytes(M, K, SF_TILED)), (w_scales, mx_scales_bytes(N, K, SF_TILED))):
-        if t.dtype != torch.uint8 or t.numel() != n or not t.is_contiguous():
-            raise ValueError("nvfp4_mx_gemm: operands must be contiguous uint8 of the MXFP4 sizes")
+    M, N, K = _mx_gemm_checks(a_codes, a_scales, w_codes, w_scales, y, "nvfp4_mx_gemm")
     _check(lib.nvfp4_mx_gemm(a_codes.data_ptr(), a_scales.data_ptr(), w_codes.data_ptr(), w_scales.data_ptr(),
                              M, N, K, y.data_ptr(), _out_dtype(y), _ldx(y), _ptr(dev_status), _stream(stream)),
            "nvfp4_mx_gemm")
+
+
+def nvfp4_mx_gemm_residue(a_codes: torch.Tensor, a_scales: torch.Tensor, r_codes: torch.Tensor,
+                          r_scales: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, y: torch.Tensor,
+                          dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """MXFP4 compensated linear y = deq(A) deq(W)^T + deq(R) deq(W)^T (TILED scales)."""
+    lib = load_library()
+    if r_codes is None or r_scales is None:
+        raise ValueError("nvfp4_mx_gemm_residue: the residue operand is required")
+    M, N, K = _mx_gemm_checks(a_codes, a_scales, w_codes, w_scales, y, "nvfp4_mx_gemm_residue", r_codes, r_scales)
+    _check(lib.nvfp4_mx_gemm_residue(a_codes.data_ptr(), a_scales.data_ptr(), r_codes.data_ptr(),
+                                     r_scales.data_ptr(), w_codes.data_ptr(), w_scales.data_ptr(), M, N, K,
+                                     y.data_ptr(), _out_dtype(y), _ldx(y), _ptr(dev_status), _stream(stream)),
+           "nvfp4_mx_gemm_residue")
 
 
 def nvfp4_quantize_residue(x: torch.Tensor, q: NVFP4Tensor, r: NVFP4Tensor,

@@ -106,11 +106,36 @@ nvfp4_status run_gemm(const nvfp4_tensor* a, const nvfp4_tensor* r, const nvfp4_
     e = launch_decode_tc(d, num_sms_current_device(), s);
   } else if (tiled && g.M <= 128) {
     e = launch_gemv_tc(g, num_sms_current_device(), s);           // tensor cores, operands swapped
-  } else if (tiled && r == nullptr) {
+  } else if (tiled) {
     e = launch_gemm_tc(g, num_sms_current_device(), s);           // tensor cores, 128x256 tiles
   } else {
     return NVFP4_ERR_UNSUPPORTED;
   }
+  if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
+nvfp4_status run_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* r_codes,
+                         const uint8_t* r_scales, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M,
+                         int64_t N, int64_t K, void* y, nvfp4_dtype out_dt, int64_t ldy, int* dev_status,
+                         void* stream) {
+  if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr || y == nullptr ||
+      !dt_ok(out_dt))
+    return NVFP4_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || ldy < N || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
+    return NVFP4_ERR_INVALID_ARG;
+  if (K % 128 != 0 || K < 256) return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(a_scales) || !aligned16(w_scales))
+    return NVFP4_ERR_ALIGNMENT;
+  if (r_codes != nullptr && (!aligned16(r_codes) || !aligned16(r_scales))) return NVFP4_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(y) % dt_size(out_dt)) != 0) return NVFP4_ERR_ALIGNMENT;
+  GemmArgs g{};
+  g.a_codes = a_codes; g.a_scales = a_scales;
+  g.r_codes = r_codes; g.r_scales = r_scales;
+  g.w_codes = w_codes; g.w_scales = w_scales;
+  g.y = y; g.ldy = ldy; g.y_bf16 = out_dt == NVFP4_BF16;
+  g.M = M; g.N = N; g.K = K; g.st = dev_status;
+  const cudaError_t e = launch_gemm_mx(g, num_sms_current_device(), static_cast<cudaStream_t>(stream));
   if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
   return cuda_status(e);
 }
@@ -196,6 +221,12 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64
   const int sms = num_sms_current_device();
   WsHeader* ws = static_cast<WsHeader*>(workspace);
   float* rinv = workspace ? reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsHeaderBytes) : nullptr;
+  if (gamma != nullptr || scale_in == nullptr) {
+    // small enough for one launch: X read once, no second pass
+    const cudaError_t e = launch_reorder_onepass(x, dt, M, K, ldx, gamma, eps, perm, S, scale_in, qout(x_aug), ws,
+                                                 dev_status, sms, s);
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+  }
   if (gamma != nullptr) {
     NVFP4_TRY(cuda_status(launch_rms_stats(x, dt, M, K, ldx, gamma, eps, ws, rinv, x_aug->tensor_scale,
                                            scale_in == nullptr, dev_status, sms, s)));
@@ -203,8 +234,9 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64
     NVFP4_TRY(cuda_status(launch_amax(x, dt, M, K, ldx, ws, 0, x_aug->tensor_scale, dev_status, sms, s)));
   }
   const float* s_ptr = scale_in ? scale_in : x_aug->tensor_scale;
+  // a programmatic dependent of the statistics pass, when there is one
   return cuda_status(launch_reorder_quant(x, dt, M, K, ldx, gamma, rinv, perm, S, s_ptr, qout(x_aug),
-                                          dev_status, sms, s));
+                                          dev_status, sms, s, gamma != nullptr || scale_in == nullptr));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt,
@@ -305,23 +337,17 @@ nvfp4_status nvfp4_mx_quantize(const void* x, nvfp4_dtype dt, int64_t M, int64_t
 nvfp4_status nvfp4_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* w_codes,
                            const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* y,
                            nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream) {
-  if (a_codes == nullptr || a_scales == nullptr || w_codes == nullptr || w_scales == nullptr || y == nullptr ||
-      !dt_ok(out_dt))
-    return NVFP4_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0 || ldy < N || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
-    return NVFP4_ERR_INVALID_ARG;
-  if (K % 128 != 0 || K < 256) return NVFP4_ERR_UNSUPPORTED;
-  if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(a_scales) || !aligned16(w_scales))
-    return NVFP4_ERR_ALIGNMENT;
-  if ((reinterpret_cast<uintptr_t>(y) % dt_size(out_dt)) != 0) return NVFP4_ERR_ALIGNMENT;
-  GemmArgs g{};
-  g.a_codes = a_codes; g.a_scales = a_scales;
-  g.w_codes = w_codes; g.w_scales = w_scales;
-  g.y = y; g.ldy = ldy; g.y_bf16 = out_dt == NVFP4_BF16;
-  g.M = M; g.N = N; g.K = K; g.st = dev_status;
-  const cudaError_t e = launch_gemm_mx(g, num_sms_current_device(), static_cast<cudaStream_t>(stream));
-  if (e == cudaErrorNotSupported) return NVFP4_ERR_UNSUPPORTED;
-  return cuda_status(e);
+  return run_mx_gemm(a_codes, a_scales, nullptr, nullptr, w_codes, w_scales, M, N, K, y, out_dt, ldy, dev_status,
+                     stream);
+}
+
+nvfp4_status nvfp4_mx_gemm_residue(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* r_codes,
+                                   const uint8_t* r_scales, const uint8_t* w_codes, const uint8_t* w_scales,
+                                   int64_t M, int64_t N, int64_t K, void* y, nvfp4_dtype out_dt, int64_t ldy,
+                                   int* dev_status, void* stream) {
+  if (r_codes == nullptr || r_scales == nullptr) return NVFP4_ERR_INVALID_ARG;
+  return run_mx_gemm(a_codes, a_scales, r_codes, r_scales, w_codes, w_scales, M, N, K, y, out_dt, ldy, dev_status,
+                     stream);
 }
 
 const char* nvfp4_status_string(nvfp4_status st) {

@@ -81,6 +81,8 @@ struct TcParams {
   int64_t ldy;
   int y_vec;       // Y base and row pitch allow 16-byte (fp32) / 8-byte (bf16) stores
   int M, N, K;
+  const uint8_t* sfr;   // residue scales (RES)
+  const float* r_s;     // residue tensor scale (RES)
   int katoms;      // scale atoms along K per 128-row group: ceil(K / 64) (MX: K / 128)
   int b_groups;    // 128-row groups of W = ceil(N / 128)
   int m_blocks, n_blocks, num_tiles, k_tiles;
@@ -92,10 +94,19 @@ struct TcParams {
 // MX: MXFP4 operands (32-element blocks, E8M0 scales, no tensor scales): the
 // same stages, with the scale atoms covering K = 128 each, so half of each
 // stage's scale area and of its TMEM scale buffer is used.
-template <bool BF16OUT, bool MX>
+// RES: ResServe's full residue (Y = s_a s_w A W^T + s_r s_w R W^T).  Each tile
+// runs two passes over its K-tiles, A W^T and then R W^T (the residue as a
+// second run of K-tiles over the same W tiles).  NVFP4: two uses of the TMEM
+// accumulator; the epilogue holds s_a s_w acc in registers while the second
+// pass runs and adds s_r s_w acc before the single store of Y.  MXFP4 has no
+// tensor scales, so the residue's K-tiles simply continue the same
+// accumulation: Y = [A | R] [W | W]^T.
+template <bool BF16OUT, bool MX, bool RES = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_nvf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const TcParams p) {
+                const __grid_constant__ CUtensorMap tmR, const TcParams p) {
+  constexpr int NPASS = RES ? 2 : 1;            // passes over the K-tiles per tile
+  constexpr int NUSE = (RES && !MX) ? 2 : 1;    // accumulator uses per tile
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* epi = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
@@ -142,7 +153,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int g = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-      for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+      for (int t = 0; t < NPASS * p.k_tiles; ++t, ++g) {
         const int s = g % STAGES;
         // every lane waits; the warp goes on only if all saw the phase (the
         // TMEM stores are warp-collective)
@@ -198,7 +209,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
         const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
         const int ngroups = min(2, p.b_groups - nb * 2);
-        for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
+        for (int t = 0; t < NPASS * p.k_tiles; ++t, ++g) {
+          const int pass = t >= p.k_tiles ? 1 : 0, kt = t - pass * p.k_tiles;
+          const uint8_t* sfa = (RES && pass) ? p.sfr : p.sfa;            // A, then R
+          const CUtensorMap* tma = (RES && pass) ? &tmR : &tmA;
           const int s = g % STAGES;
           if (!mbar_wait_inline(saddr(&empty[s]), (uint32_t)((g / STAGES) & 1) ^ 1u, abort_flag, p.st)) goto producer_done;
           const int jmax = min(4, (p.K - kt * BK) / 64);
@@ -207,13 +221,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint8_t* st_base = smem + s * STAGE_BYTES;
           const uint32_t sbar = saddr(&sf_land[s]);
           mbar_expect_tx(sbar, sf_bytes * (1 + ngroups));
-          bulk_load(saddr(st_base + OFF_SFA), p.sfa + ((size_t)mb * p.katoms + kt * apt) * 512, sf_bytes, sbar);
+          bulk_load(saddr(st_base + OFF_SFA), sfa + ((size_t)mb * p.katoms + kt * apt) * 512, sf_bytes, sbar);
           for (int gi = 0; gi < ngroups; ++gi)
             bulk_load(saddr(st_base + OFF_SFB + gi * 2048),
                       p.sfb + ((size_t)(nb * 2 + gi) * p.katoms + kt * apt) * 512, sf_bytes, sbar);
           const uint32_t bar = saddr(&full[s]);
           mbar_expect_tx(bar, A_BYTES + B_BYTES);
-          tma_load_2d(saddr(st_base), &tmA, kt * BK_BYTES, mb * BM, bar);
+          tma_load_2d(saddr(st_base), tma, kt * BK_BYTES, mb * BM, bar);
           tma_load_2d(saddr(st_base + OFF_B), &tmB, kt * BK_BYTES, nb * BN, bar);
         }
       }
@@ -222,9 +236,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // -------------------------------------------------------- MMA issuer
       const uint32_t idesc = idesc_nvf4(BN);
       int g = 0, local = 0;
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
-        if (!mbar_wait_inline(saddr(acc_empty), (uint32_t)(local & 1) ^ 1u, abort_flag, p.st)) break;
-        tc_fence_after();
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local)
+      for (int pass = 0; pass < NPASS; ++pass) {
+        // accumulator use u: the epilogue has taken use u - 1 out of TMEM
+        const bool fresh = NUSE == 2 || pass == 0;   // this pass starts a use of the accumulator
+        const int u = NUSE * local + (NUSE == 2 ? pass : 0);
+        if (fresh) {
+          if (!mbar_wait_inline(saddr(acc_empty), (uint32_t)(u & 1) ^ 1u, abort_flag, p.st)) goto mma_done;
+          tc_fence_after();
+        }
         for (int kt = 0; kt < p.k_tiles; ++kt, ++g) {
           const int s = g % STAGES;
           const uint32_t ph = (uint32_t)((g / STAGES) & 1);
@@ -239,14 +259,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if constexpr (MX)   // K = 64 chunk j: atom j / 2, scale bytes 2 (j % 2) and 2 (j % 2) + 1
               tc_mma_mxf4(tmem + ACC_COL, da + (uint64_t)(2 * j), db + (uint64_t)(2 * j),
                           idesc_mxf4(BN, 2u * (uint32_t)(j & 1)), tmem + buf + 4 * (j >> 1),
-                          tmem + buf + 8 + 8 * (j >> 1), (kt > 0 || j > 0) ? 1u : 0u);
+                          tmem + buf + 8 + 8 * (j >> 1), (!fresh || kt > 0 || j > 0) ? 1u : 0u);
             else
               tc_mma_nvf4(tmem + ACC_COL, da + (uint64_t)(2 * j), db + (uint64_t)(2 * j), idesc, tmem + buf + 4 * j,
-                          tmem + buf + 16 + 8 * j, (kt > 0 || j > 0) ? 1u : 0u);
+                          tmem + buf + 16 + 8 * j, (!fresh || kt > 0 || j > 0) ? 1u : 0u);
           }
           tc_commit(saddr(&empty[s]));
         }
-        tc_commit(saddr(acc_full));
+        if (NUSE == 2 || pass == NPASS - 1) tc_commit(saddr(acc_full));
       }
     mma_done:;
     }
@@ -259,9 +279,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int sub_r = lane >> 1, sub_c = (lane & 1) * 4;
     int local = 0;
     const float alpha = MX ? 1.0f : (*p.a_s) * (*p.w_s);   // MXFP4 has no tensor scales
+    const float alpha_r = NUSE == 2 ? (*p.r_s) * (*p.w_s) : 0.0f;
+    const float out_scale = NUSE == 2 ? 1.0f : alpha;        // two uses: the registers hold the combined Y
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++local) {
       const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
-      if (!mbar_wait_inline(saddr(acc_full), (uint32_t)(local & 1), abort_flag, p.st)) break;
+      if (!mbar_wait_inline(saddr(acc_full), (uint32_t)((NUSE * local) & 1), abort_flag, p.st)) break;
       tc_fence_after();
       // Each warp owns TMEM lanes (= tile rows) 32q..32q+31 and columns
       // [128 half, 128 half + 128): read them all, then free the accumulator.
@@ -273,6 +295,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(saddr(acc_empty));
+      if constexpr (NUSE == 2) {
+        // s_a s_w acc1 stays in registers; add s_r s_w acc2 column chunk by column chunk
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[c][i] = __float_as_uint(__uint_as_float(r[c][i]) * alpha);
+        if (!mbar_wait_inline(saddr(acc_full), (uint32_t)((NUSE * local + 1) & 1), abort_flag, p.st)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c) {
+          uint32_t t[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + (half * (BN / 64) + c) * 32, t);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            r[c][i] = __float_as_uint(fmaf(alpha_r, __uint_as_float(t[i]), __uint_as_float(r[c][i])));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(saddr(acc_empty));
+      }
       // 32 x 8 chunks: lane = row while writing, then 2 lanes per 8-column row
       // segment, 16 rows per store instruction
 #pragma unroll
@@ -282,7 +325,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int g8 = 0; g8 < 4; ++g8) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) buf[lane * EPI_PITCH + i] = __uint_as_float(r[c][g8 * 8 + i]) * alpha;
+          for (int i = 0; i < 8; ++i) buf[lane * EPI_PITCH + i] = __uint_as_float(r[c][g8 * 8 + i]) * out_scale;
           __syncwarp();
           const int cg = col0 + g8 * 8;
 #pragma unroll
@@ -360,17 +403,20 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
 
 template <bool MX>
 cudaError_t launch_gemm_impl(const GemmArgs& g, int num_sms, cudaStream_t stream) {
-  if (g.r_codes != nullptr) return cudaErrorNotSupported;  // own-scale residue: small-M paths only
+  const bool res = g.r_codes != nullptr;   // ResServe residue: a second pass over the K-tiles
   if (MX ? (g.K % 128 != 0 || g.K < BK) : (g.K % 64 != 0 || g.K < BK)) return cudaErrorNotSupported;
   // sizes, tile coordinates and the tile count are 32-bit in the kernel
   if (g.M > INT32_MAX || g.N > INT32_MAX || g.K > INT32_MAX ||
       ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN) > INT32_MAX)
     return cudaErrorNotSupported;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmR;
   if (!encode_codes_map(&tmA, g.a_codes, g.M, g.K, BM) || !encode_codes_map(&tmB, g.w_codes, g.N, g.K, BN))
     return cudaErrorInvalidValue;
+  if (res ? !encode_codes_map(&tmR, g.r_codes, g.M, g.K, BM) : false) return cudaErrorInvalidValue;
+  if (!res) tmR = tmA;   // unused
   TcParams p{};
   p.sfa = g.a_scales; p.sfb = g.w_scales; p.a_s = g.a_s; p.w_s = g.w_s;
+  p.sfr = g.r_scales; p.r_s = g.r_s;
   p.y = g.y; p.ldy = g.ldy;
   {
     const size_t vec_bytes = g.y_bf16 ? 8 : 16, esize = g.y_bf16 ? 2 : 4;
@@ -384,14 +430,15 @@ cudaError_t launch_gemm_impl(const GemmArgs& g, int num_sms, cudaStream_t stream
   p.num_tiles = p.m_blocks * p.n_blocks;
   p.k_tiles = (int)((g.K + BK - 1) / BK);
   p.st = g.st;
-  auto kern = g.y_bf16 ? k_gemm_nvf4<true, MX> : k_gemm_nvf4<false, MX>;
+  auto kern = res ? (g.y_bf16 ? k_gemm_nvf4<true, MX, true> : k_gemm_nvf4<false, MX, true>)
+                  : (g.y_bf16 ? k_gemm_nvf4<true, MX> : k_gemm_nvf4<false, MX>);
   // the register split assumes the launch allocates LAUNCH_REGS per thread
   cudaFuncAttributes fa{};
   if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != LAUNCH_REGS) return cudaErrorNotSupported;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(p.num_tiles, num_sms));
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmR, p);
   return cudaGetLastError();
 }
 

@@ -42,10 +42,17 @@ cudaError_t launch_quant_small(bool residue, const void* x, nvfp4_dtype dt, int6
                                const float* s_in, const float* sr_in, const QOut& q, const QOut& r, int* st,
                                cudaStream_t stream);
 size_t reorder_smem_bytes(nvfp4_dtype dt, int64_t K, bool has_gamma);
+// ARCQuant quantizer in one cooperative launch when every row fits in the
+// shared memory of one wave of CTAs; cudaErrorNotSupported (nothing launched)
+// otherwise.  Identical results to the statistics pass + launch_reorder_quant.
+cudaError_t launch_reorder_onepass(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                   const void* gamma, float eps, const int32_t* perm, int64_t S,
+                                   const float* s_in, const QOut& q, WsHeader* ws, int* st, int num_sms,
+                                   cudaStream_t stream);
 cudaError_t launch_reorder_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                  const void* gamma, const float* rinv, const int32_t* perm,
                                  int64_t S, const float* s_ptr, const QOut& q, int* st, int num_sms,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, bool after_stats);
 
 // Operands of the decode GEMV / tensor-core GEMM.
 struct GemmArgs {

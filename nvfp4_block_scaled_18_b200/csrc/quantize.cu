@@ -328,6 +328,7 @@ __global__ void __launch_bounds__(256) k_rms_stats(const T* __restrict__ x, int6
                                                    float* s_out, bool want_scale, int* st) {
   __shared__ uint32_t redu[32];
   __shared__ double redd[32];
+  tc::griddep_launch_dependents();   // the reorder pass may launch; it waits for this grid's results
   const int64_t upr = K >> 3;
   uint32_t ykey = 0, bad = 0;
   // unit c8 of the row: NC > 0 -> c8 = threadIdx.x + 256 n, n < NC
@@ -430,6 +431,89 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// The channel permutation as 16-bit indices in shared memory (K <= 65536).  An
+// entry outside 0..K-1 is replaced by 0, so no index is ever out of range; the
+// return value says whether there was one.
+__device__ __forceinline__ bool load_perm16(const int32_t* __restrict__ perm, int64_t K, uint16_t* sperm) {
+  bool bad_perm = false;
+  if (perm != nullptr && (reinterpret_cast<uintptr_t>(perm) & 15u) == 0) {
+    // four 16-byte loads per thread in flight before any is used (K % 16 == 0)
+    constexpr int U = 4;
+    const int64_t n4 = K >> 2;
+    const uint4* p4 = reinterpret_cast<const uint4*>(perm);
+    for (int64_t c0 = threadIdx.x; c0 < n4; c0 += U * (int64_t)blockDim.x) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t c = c0 + u * (int64_t)blockDim.x;
+        v[u] = c < n4 ? __ldg(p4 + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t c = c0 + u * (int64_t)blockDim.x;
+        if (c < n4) {
+          uint32_t e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if ((uint64_t)e[i] >= (uint64_t)K) {   // also catches negative entries
+              bad_perm = true;
+              e[i] = 0u;
+            }
+          *reinterpret_cast<uint2*>(sperm + 4 * c) = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+        }
+      }
+    }
+  } else {
+    for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
+      int32_t p = perm ? perm[k] : (int32_t)k;
+      if (p < 0 || (int64_t)p >= K) {
+        bad_perm = true;
+        p = 0;
+      }
+      sperm[k] = (uint16_t)p;
+    }
+  }
+  return bad_perm;
+}
+
+// Encode one row held in shared memory: y'[j] = fl32(fl32(x[perm[j]] * ri) *
+// gamma[perm[j]]) (y' = x[perm] without gamma), one thread per 16-element block
+// of the reordered row; the first nbr blocks' residues are quantized under the
+// same scale and written as blocks nb .. nb + nbr - 1.
+template <typename T>
+__device__ __forceinline__ void encode_reordered_row(const T* srow, const uint16_t* sperm, const T* sgamma,
+                                                     float ri, float s, const QOut& q, int64_t row, int nb,
+                                                     int nbr, uint32_t& bad) {
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+    float v[16];
+    uint16_t pv[16];
+#pragma unroll
+    for (int j = 0; j < 2; ++j)   // 16-byte reads of the cached permutation
+      *reinterpret_cast<uint4*>(pv + 8 * j) = reinterpret_cast<const uint4*>(sperm)[b * 2 + j];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int p = pv[i];
+      float y = load1(srow + p);
+      bad = max(bad, abs_key(y));
+      if (sgamma) y = __fmul_rn(__fmul_rn(y, ri), load1(sgamma + p));
+      v[i] = y;
+    }
+    uint32_t db;
+    float deq[16];
+    const bool res = b < nbr;
+    const uint64_t codes = quant_block16(v, s, db, res ? deq : nullptr);
+    store_block16(q, row, b, codes, db);
+    if (res) {
+      float rv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) rv[i] = __fsub_rn(v[i], deq[i]);
+      uint32_t dr;
+      const uint64_t rc = quant_block16(rv, s, dr, nullptr);
+      store_block16(q, row, nb + b, rc, dr);
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, int64_t M,
                                                        int64_t K, int64_t ldx,
@@ -449,18 +533,19 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
       cp_async16(reinterpret_cast<uint4*>(dst) + c, reinterpret_cast<const uint4*>(xr) + c);
     cp_async_commit();
   };
+  // gamma goes to shared memory by cp.async in the first row's group (its
+  // pointer is 16-byte aligned and K * sizeof(T) a multiple of 16)
+  if (gamma)
+    for (int64_t c = threadIdx.x; c < row_bytes / 16; c += blockDim.x)
+      cp_async16(reinterpret_cast<uint4*>(sgamma) + c, reinterpret_cast<const uint4*>(gamma) + c);
   if ((int64_t)blockIdx.x < M) fetch_row(blockIdx.x, srow0);   // overlaps the table set-up
+  else cp_async_commit();
+  if (load_perm16(perm, K, sperm)) report_status(st, NVFP4_ERR_INVALID_ARG);
+  // X, gamma and perm are inputs of the call; the tensor scale and the row
+  // factors come from the statistics pass, which may still be running
+  tc::griddep_wait();
   const float s = *s_ptr;
   if (blockIdx.x == 0 && threadIdx.x == 0 && q.s != s_ptr) *q.s = s;
-  for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
-    int32_t p = perm ? perm[k] : (int32_t)k;
-    if (p < 0 || (int64_t)p >= K) {  // not a permutation of 0..K-1: report, never index out of range
-      report_status(st, NVFP4_ERR_INVALID_ARG);
-      p = 0;
-    }
-    sperm[k] = (uint16_t)p;
-    if (gamma) sgamma[k] = gamma[k];
-  }
   const int nb = (int)(K >> 4);     // blocks of the reordered row
   const int nbr = (int)(S >> 4);    // residue blocks (the first S reordered columns)
   uint32_t bad = 0;
@@ -470,38 +555,179 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
     cp_async_wait_all();
     __syncthreads();   // this row landed; every thread is done with the other buffer
     if (row + gridDim.x < M) fetch_row(row + gridDim.x, buf ? srow0 : srow1);
-    const float ri = gamma ? rinv[row] : 1.0f;
-    // one thread per 16-element block of the reordered row
-    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
-      float v[16];
-      uint16_t pv[16];
+    encode_reordered_row(srow, sperm, gamma ? sgamma : nullptr, gamma ? rinv[row] : 1.0f, s, q, row, nb, nbr,
+                         bad);
+  }
+  cp_async_wait_all();
+  if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
+}
+
+// One-launch ARCQuant quantizer, for inputs that fit in the shared memory of
+// one wave of CTAs.  The launch is cooperative, so every CTA is resident.
+// Each CTA:
+//   1. loads its rows (rows blockIdx.x + i * gridDim.x) once, with gamma and
+//      the permutation;
+//   2. derives each row's factor rinv and its part of the tensor maximum with
+//      the arithmetic of k_rms_stats (or the |x| maximum of k_amax without
+//      gamma);
+//   3. meets the other CTAs at one exchange of that maximum through the
+//      workspace header (atomics, a bounded wait; the last CTA to leave zeroes
+//      the header again);
+//   4. encodes its rows from shared memory as k_reorder_quant does.
+// So X is read from DRAM once and the result is identical to the two passes.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned int* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// 8 consecutive elements from shared memory as fp32.
+__device__ __forceinline__ void lds8(const __nv_bfloat16* p, float v[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+  v[4] = __uint_as_float(u.z << 16); v[5] = __uint_as_float(u.z & 0xFFFF0000u);
+  v[6] = __uint_as_float(u.w << 16); v[7] = __uint_as_float(u.w & 0xFFFF0000u);
+}
+__device__ __forceinline__ void lds8(const float* p, float v[8]) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Bytes of dynamic shared memory of k_reorder_onepass for `rows` rows per CTA.
+inline size_t onepass_smem_bytes(size_t es, int64_t K, bool has_gamma, int rows) {
+  return (size_t)rows * (size_t)K * es + (((size_t)K * 2 + 15) & ~size_t(15)) +
+         (has_gamma ? (size_t)K * es : 0) + (size_t)rows * 4;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_reorder_onepass(const T* __restrict__ x, int64_t M, int64_t K,
+                                                         int64_t ldx, const T* __restrict__ gamma, float eps,
+                                                         const int32_t* __restrict__ perm, int64_t S,
+                                                         const float* s_in, QOut q, WsHeader* ws,
+                                                         int rows_per_cta, int* st) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ uint32_t redu[32];
+  __shared__ double redd[32];
+  __shared__ float s_sh;
+  __shared__ int ok_sh;
+  const int64_t row_bytes = K * (int64_t)sizeof(T);   // a multiple of 16 (K % 16 == 0)
+  const int64_t rows_bytes = (int64_t)rows_per_cta * row_bytes;
+  T* srows = reinterpret_cast<T*>(smem);
+  uint16_t* sperm = reinterpret_cast<uint16_t*>(smem + rows_bytes);
+  const int64_t perm_bytes = (K * 2 + 15) & ~int64_t(15);
+  T* sgamma = reinterpret_cast<T*>(smem + rows_bytes + perm_bytes);
+  float* srinv = reinterpret_cast<float*>(smem + rows_bytes + perm_bytes + (gamma ? row_bytes : 0));
+  const int64_t G = gridDim.x;
+  int nrows = 0;   // rows of this CTA
+  while (nrows < rows_per_cta && (int64_t)blockIdx.x + nrows * G < M) ++nrows;
+
+  // 1. every load in flight at once
+  if (gamma)
+    for (int64_t c = threadIdx.x; c < row_bytes / 16; c += blockDim.x)
+      cp_async16(reinterpret_cast<uint4*>(sgamma) + c, reinterpret_cast<const uint4*>(gamma) + c);
+  for (int i = 0; i < nrows; ++i) {
+    const T* xr = x + ((int64_t)blockIdx.x + i * G) * ldx;
+    T* dst = srows + (int64_t)i * K;
+    for (int64_t c = threadIdx.x; c < row_bytes / 16; c += blockDim.x)
+      cp_async16(reinterpret_cast<uint4*>(dst) + c, reinterpret_cast<const uint4*>(xr) + c);
+  }
+  cp_async_commit();
+  if (load_perm16(perm, K, sperm)) report_status(st, NVFP4_ERR_INVALID_ARG);
+  cp_async_wait_all();
+  __syncthreads();
+
+  // 2. row factors and this CTA's part of the tensor maximum
+  const int64_t upr = K >> 3;
+  uint32_t ykey = 0, bad = 0;
+  for (int i = 0; i < nrows; ++i) {
+    const T* sr = srows + (int64_t)i * K;
+    uint32_t key = 0;
+    for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+      float v[8];
+      lds8(sr + c8 * 8, v);
 #pragma unroll
-      for (int j = 0; j < 2; ++j)   // 16-byte reads of the cached permutation
-        *reinterpret_cast<uint4*>(pv + 8 * j) = reinterpret_cast<const uint4*>(sperm)[b * 2 + j];
+      for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
+    }
+    key = block_max_u32(key, redu);
+    bad = max(bad, key);
+    if (gamma == nullptr) {
+      ykey = max(ykey, key);
+      continue;
+    }
+    double qsum = 0.0;
+    int e = 0;
+    if (key != 0u && key < 0x7F800000u) {
+      e = ilog2_key(key);
+      const double c = pow2_f64(17 - e);  // z = x * 2^(17-e), |z| < 2^18
+      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+        float v[8];
+        lds8(sr + c8 * 8, v);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int p = pv[i];
-        float y = load1(srow + p);
-        bad = max(bad, abs_key(y));
-        if (gamma) y = __fmul_rn(__fmul_rn(y, ri), load1(sgamma + p));
-        v[i] = y;
+        for (int j = 0; j < 8; ++j) {
+          const double z = __dmul_rn((double)v[j], c);
+          qsum = __dadd_rn(qsum, floor(__dmul_rn(z, z)));
+        }
       }
-      uint32_t db;
-      float deq[16];
-      const bool res = b < nbr;
-      const uint64_t codes = quant_block16(v, s, db, res ? deq : nullptr);
-      store_block16(q, row, b, codes, db);
-      if (res) {
-        float rv[16];
+    }
+    qsum = block_sum_f64(qsum, redd);  // exact: integers with total < 2^53
+    const double mean = __ddiv_rn(__dmul_rn(qsum, pow2_f64(2 * e - 34)), (double)K);
+    const float ri = __double2float_rn(__drcp_rn(__dsqrt_rn(__dadd_rn(mean, (double)eps))));
+    if (threadIdx.x == 0) srinv[i] = ri;
+    if (s_in == nullptr) {
+      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+        float v[8], g[8];
+        lds8(sr + c8 * 8, v);
+        lds8(sgamma + c8 * 8, g);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) rv[i] = __fsub_rn(v[i], deq[i]);
-        uint32_t dr;
-        const uint64_t rc = quant_block16(rv, s, dr, nullptr);
-        store_block16(q, row, nb + b, rc, dr);
+        for (int j = 0; j < 8; ++j) ykey = max(ykey, abs_key(__fmul_rn(__fmul_rn(v[j], ri), g[j])));
       }
     }
   }
-  cp_async_wait_all();
+
+  // 3. the tensor scale
+  if (s_in == nullptr) {
+    const uint32_t m = block_max_u32(ykey, redu);
+    if (threadIdx.x == 0) {
+      if (m != 0u) atomicMax(&ws->amax_bits[0], m);
+      __threadfence();
+      atomicAdd(&ws->arrive[0], 1u);
+      const uint64_t t0 = tc::globaltimer();
+      int ok = 1;
+      while (ld_acquire_gpu(&ws->arrive[0]) < (uint32_t)G) {
+        if (tc::globaltimer() - t0 > tc::kTimeoutNs) {
+          ok = 0;
+          report_status(st, NVFP4_ERR_TIMEOUT);
+          break;
+        }
+      }
+      const uint32_t a = atomicAdd(&ws->amax_bits[0], 0u);
+      s_sh = ok ? scale_from_key(a, blockIdx.x == 0, st) : 0.0f;
+      ok_sh = ok;
+      // the last CTA to leave zeroes the header for the next call
+      __threadfence();
+      if (atomicAdd(&ws->arrive[1], 1u) == (uint32_t)G - 1u) {
+        ws->amax_bits[0] = 0u;
+        ws->arrive[0] = 0u;
+        ws->arrive[1] = 0u;
+        __threadfence();
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    s_sh = *s_in;
+    ok_sh = 1;
+  }
+  __syncthreads();   // s_sh, ok_sh and srinv are visible to every thread
+  if (!ok_sh) return;
+  const float s = s_sh;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && q.s != s_in) *q.s = s;
+
+  // 4. encode
+  const int nb = (int)(K >> 4), nbr = (int)(S >> 4);
+  for (int i = 0; i < nrows; ++i)
+    encode_reordered_row(srows + (int64_t)i * K, sperm, gamma ? sgamma : nullptr, gamma ? srinv[i] : 1.0f, s, q,
+                         (int64_t)blockIdx.x + i * G, nb, nbr, bad);
   if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
 }
 
@@ -679,27 +905,91 @@ template <typename T>
 cudaError_t launch_reorder_quant_t(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
                                    const float* rinv, const int32_t* perm, int64_t S,
                                    const float* s_ptr, const QOut& q, int* st, int num_sms,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, bool after_stats) {
   const size_t smem = reorder_smem_bytes(sizeof(T) == 2 ? NVFP4_BF16 : NVFP4_F32, K, gamma != nullptr);
   cudaError_t e = cudaFuncSetAttribute(k_reorder_quant<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  // several CTAs per SM so that rows overlap
-  const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (220 * 1024) / (smem + 1024)));
+  // one wave of resident CTAs, several per SM so that rows overlap; a second
+  // wave would repeat the table set-up for only a few rows each
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_reorder_quant<T>, 256, smem);
+  if (e != cudaSuccess) return e;
+  per_sm = std::max(1, std::min(per_sm, 8));
   const unsigned g = (unsigned)std::max<int64_t>(1, std::min<int64_t>(M, (int64_t)num_sms * per_sm));
-  k_reorder_quant<T><<<g, 256, smem, stream>>>(static_cast<const T*>(x), M, K, ldx,
-                                               static_cast<const T*>(gamma), rinv, perm, S, s_ptr,
-                                               q, st);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // after the statistics pass only
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_stats ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_reorder_quant<T>, static_cast<const T*>(x), M, K, ldx,
+                            static_cast<const T*>(gamma), rinv, perm, S, s_ptr, q, st);
+}
+
+template <typename T>
+cudaError_t launch_reorder_onepass_t(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                                     float eps, const int32_t* perm, int64_t S, const float* s_in,
+                                     const QOut& q, WsHeader* ws, int* st, int num_sms, cudaStream_t stream) {
+  constexpr size_t kMaxSmem = 227 * 1024;   // opt-in dynamic shared memory per CTA
+  // the most CTAs per SM (up to 4) whose rows all fit in shared memory together
+  for (int per_sm = 4; per_sm >= 1; --per_sm) {
+    const int64_t g = std::min<int64_t>((int64_t)num_sms * per_sm, M);
+    const int64_t rows = (M + g - 1) / g;
+    if (rows > 4096) continue;
+    const size_t smem = onepass_smem_bytes(sizeof(T), K, gamma != nullptr, (int)rows);
+    if (smem > kMaxSmem) continue;
+    cudaError_t e = cudaFuncSetAttribute(k_reorder_onepass<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_reorder_onepass<T>, 256, smem);
+    if (e != cudaSuccess) return e;
+    if ((int64_t)occ * num_sms < g) continue;   // not all resident at once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)g);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs resident: they meet at the exchange
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, k_reorder_onepass<T>, static_cast<const T*>(x), M, K, ldx,
+                           static_cast<const T*>(gamma), eps, perm, S, s_in, q, ws, (int)rows, st);
+    if (e == cudaErrorCooperativeLaunchTooLarge) {
+      (void)cudaGetLastError();
+      return cudaErrorNotSupported;   // nothing ran; the two passes do the work
+    }
+    return e;
+  }
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_reorder_onepass(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
+                                   const void* gamma, float eps, const int32_t* perm, int64_t S,
+                                   const float* s_in, const QOut& q, WsHeader* ws, int* st, int num_sms,
+                                   cudaStream_t stream) {
+  return dt == NVFP4_BF16
+             ? launch_reorder_onepass_t<__nv_bfloat16>(x, M, K, ldx, gamma, eps, perm, S, s_in, q, ws, st, num_sms,
+                                                       stream)
+             : launch_reorder_onepass_t<float>(x, M, K, ldx, gamma, eps, perm, S, s_in, q, ws, st, num_sms, stream);
 }
 
 cudaError_t launch_reorder_quant(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                  const void* gamma, const float* rinv, const int32_t* perm,
                                  int64_t S, const float* s_ptr, const QOut& q, int* st, int num_sms,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, bool after_stats) {
   return dt == NVFP4_BF16
-             ? launch_reorder_quant_t<__nv_bfloat16>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms, stream)
-             : launch_reorder_quant_t<float>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms, stream);
+             ? launch_reorder_quant_t<__nv_bfloat16>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms,
+                                                     stream, after_stats)
+             : launch_reorder_quant_t<float>(x, M, K, ldx, gamma, rinv, perm, S, s_ptr, q, st, num_sms, stream,
+                                             after_stats);
 }
 
 }  // namespace nvfp4

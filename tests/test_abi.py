@@ -159,3 +159,12 @@ def test_sizes_beyond_32_bits_rejected(lib):
     assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(w), good, 0, 1 << 31, None, None) == 3
     assert lib.nvfp4_quantize_gemm_plan(1, 1 << 31, 4096, 1, 0, 0) == 0
     assert lib.nvfp4_mx_gemm(good, good, good, good, 1 << 31, 256, 256, good, 0, 256, None, None) == 1
+
+
+def test_mx_residue_validation_before_launch(lib):
+    good = 1 << 20
+    g = lib.nvfp4_mx_gemm_residue
+    assert g(good, good, None, good, good, good, 128, 256, 256, good, 0, 256, None, None) == 1   # no residue
+    assert g(good, good, good, None, good, good, 128, 256, 256, good, 0, 256, None, None) == 1
+    assert g(good, good, good + 4, good, good, good, 128, 256, 256, good, 0, 256, None, None) == 2
+    assert g(good, good, good, good, good, good, 128, 256, 192, good, 0, 256, None, None) == 3

@@ -147,3 +147,34 @@ def test_arcquant_augmented_gemm(orc, S):
     ys = y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].cpu().numpy()
     err = rel_fro(ys, orc.gemm(ox, ow))
     assert err <= REL_FRO_TOL, err
+
+
+# ------------------------------------------- ResServe residue on the large-M GEMM
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 1024), (200, 300, 320), (1000, 130, 576), (129, 1000, 4224)])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_residue_large_m(orc, M, N, K, out_dtype):
+    """Y = s_a s_w A W^T + s_r s_w R W^T for M > 128: the residue runs as a second
+    accumulation pass of the same tiles, combined before the single store."""
+    rng = np.random.default_rng(M * 7 + N + K)
+    x = (0.5 * rng.standard_t(3.0, (M, K))).astype(np.float32)
+    w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    q = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED)
+    r = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED)
+    nv.nvfp4_quantize_residue(to_dev(x, torch.float32), q, r, workspace=nv.Workspace(M, K))
+    qw = run_quantize(to_dev(w, torch.float32), nv.SF_TILED)
+    y = torch.full((M, N), float("nan"), dtype=out_dtype, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_gemm_residue(q, r, qw, y, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, nv.status_string(st.item())
+    oq, orr = orc.quantize_residue(x)
+    assert_same_q(q, oq, "Q(X)")
+    assert_same_q(r, orr, "Q(R)")
+    ref = orc.gemm_residue(oq, orr, orc.quantize(w))
+    yv = y.float().cpu().numpy()
+    if out_dtype == torch.float32:
+        assert rel_fro(yv, ref) <= REL_FRO_TOL
+    else:   # bf16 rounding of each output on top of the fp32 accumulation
+        atol = 1e-5 * np.sqrt(np.mean(ref ** 2))
+        assert np.all(np.abs(yv - ref) <= 2.0 ** -8 * np.abs(ref) + atol)

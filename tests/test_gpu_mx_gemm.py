@@ -148,3 +148,42 @@ def test_mx_gemm_rejects_unsupported_k(K):
     with pytest.raises(nv.NVFP4Error) as e:
         nv.nvfp4_mx_gemm(ac, asc, wc, wsc, y)
     assert e.value.status == 3
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (333, 520, 1280), (1, 256, 512), (256, 1024, 4096)])
+def test_mx_gemm_residue(orc, M, N, K):
+    """MXFP4 compensated linear: the residue's K-tiles continue the same accumulation."""
+    qa, qr = orc.mx_quantize_residue(wl.resserve_x(M, K))
+    qw = orc.mx_quantize(wl.weights_normal(N, K))
+    (ac, asc), (rc, rsc), (wc, wsc) = dev_operand(qa), dev_operand(qr), dev_operand(qw)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_mx_gemm_residue(ac.view(M, -1), asc, rc.view(M, -1), rsc, wc.view(N, -1), wsc, y, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert rel_fro(y.cpu().numpy(), orc.mx_gemm(qa, qw, qr)) <= REL_FRO_TOL
+
+
+def test_mx_residue_on_device_then_gemm(orc):
+    """X quantized with its residue on the device (TILED scales, checked bit for
+    bit), W likewise without residue, then the compensated MXFP4 linear."""
+    M, N, K = 300, 512, 2048
+    x, w = wl.resserve_x(M, K), wl.weights_normal(N, K)
+    ns_x, ns_w = nv.mx_scales_bytes(M, K, nv.SF_TILED), nv.mx_scales_bytes(N, K, nv.SF_TILED)
+    xc = torch.zeros(M * K // 2, dtype=torch.uint8, device="cuda")
+    xs = torch.zeros(ns_x, dtype=torch.uint8, device="cuda")
+    rc, rs = torch.zeros_like(xc), torch.zeros_like(xs)
+    wc = torch.zeros(N * K // 2, dtype=torch.uint8, device="cuda")
+    wsc = torch.zeros(ns_w, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_mx_quantize(to_dev(x), xc, xs, rc, rs, sf_layout=nv.SF_TILED)
+    nv.nvfp4_mx_quantize(to_dev(w), wc, wsc, sf_layout=nv.SF_TILED)
+    y = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_mx_gemm_residue(xc.view(M, -1), xs, rc.view(M, -1), rs, wc.view(N, -1), wsc, y)
+    torch.cuda.synchronize()
+    (oc, osc), (orc_c, ors) = orc.mx_quantize_residue(wl.bf16_values(x))
+    np.testing.assert_array_equal(rs.cpu().numpy(), tiled_from_rowmajor(ors))
+    b = rc.cpu().numpy().reshape(M, K // 2)
+    np.testing.assert_array_equal(b & 0xF, orc_c[:, 0::2])
+    np.testing.assert_array_equal(b >> 4, orc_c[:, 1::2])
+    qw = orc.mx_quantize(wl.bf16_values(w))
+    assert rel_fro(y.cpu().numpy(), orc.mx_gemm((oc, osc), qw, (orc_c, ors))) <= REL_FRO_TOL

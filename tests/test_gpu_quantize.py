@@ -278,3 +278,67 @@ def test_nonfinite_reported_multi_launch():
     torch.cuda.synchronize()
     assert st.item() == 5
     assert int(ws.buf.count_nonzero()) == 0
+
+
+# ------------------------------- ARCQuant quantizer: one launch or two passes
+
+# X that fits in the shared memory of one wave of CTAs is quantized by one
+# cooperative launch (rows read once, one grid-wide exchange of the maximum);
+# larger X by the statistics pass and the reorder pass.  Both must give the
+# oracle's codes and scales bit for bit and leave the workspace header zeroed.
+@pytest.mark.parametrize("M,K,norm,given", [(2048, 4096, True, False), (2048, 4096, True, True),
+                                            (2048, 4096, False, False), (3000, 4096, True, False),
+                                            (8192, 4096, True, False), (5, 512, True, False)])
+def test_reorder_one_launch_and_two_pass(orc, M, K, norm, given):
+    S = 256 if K >= 256 else 0
+    ch = wl.outlier_channels(K, 0.02)
+    x = wl.bf16_values(wl.activations_normal(M, K, 0.02, 30.0, wl.SEED_X, ch))
+    gamma = wl.bf16_values(wl.gamma_uniform(K)) if norm else None
+    perm = wl.calibrated_perm(wl.activations_normal(64, K, 0.02, 30.0, wl.SEED_CALIB, ch))
+    s_given = np.float32(0.05) if given else None
+    xa = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED)
+    ws = nv.Workspace(M, K)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_rmsnorm_reorder_quantize(
+        to_dev(x), xa, gamma=to_dev(gamma) if norm else None, eps=1e-5, perm=torch.from_numpy(perm).cuda(), S=S,
+        scale_in=torch.tensor([s_given], dtype=torch.float32, device="cuda") if given else None,
+        workspace=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0 and int(ws.buf[:256].count_nonzero()) == 0
+    ref = orc.rmsnorm_reorder_quantize(x, gamma, 1e-5, perm, S, s=s_given)
+    assert_same_q(xa, ref, f"M={M} K={K}")
+
+
+@pytest.mark.parametrize("M", [64, 4096])   # one launch / two passes
+def test_reorder_bad_perm_reported(M):
+    """A permutation entry outside 0..K-1 is reported (NVFP4_ERR_INVALID_ARG) and
+    never used as an index; both set-up paths (16-byte aligned and not)."""
+    K, S = 4096, 256
+    x = to_dev(wl.prefill_x(M, K))
+    gamma = to_dev(wl.bf16_values(wl.gamma_uniform(K)))
+    base = torch.arange(K + 1, dtype=torch.int32, device="cuda")
+    for perm in (base[:K].clone(), base[1:]):                  # aligned copy, 4-byte offset view
+        perm[7] = K + 5
+        perm[100] = -3
+        xa = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        nv.nvfp4_rmsnorm_reorder_quantize(x, xa, gamma=gamma, perm=perm, S=S, workspace=nv.Workspace(M, K),
+                                          dev_status=st)
+        torch.cuda.synchronize()
+        assert st.item() == 1
+
+
+def test_reorder_unaligned_perm_same_result(orc):
+    """The permutation set-up reads 16-byte vectors when it can and single
+    entries otherwise; both give the oracle's result."""
+    x, gamma, perm = wl.arc_inputs(M=256)
+    K, S = x.shape[1], 128
+    big = torch.zeros(K + 1, dtype=torch.int32, device="cuda")
+    big[1:] = torch.from_numpy(np.ascontiguousarray(perm, dtype=np.int32)).cuda()
+    xa = nv.NVFP4Tensor.empty(256, K + S, nv.SF_TILED)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_rmsnorm_reorder_quantize(to_dev(x), xa, gamma=to_dev(gamma), eps=1e-5, perm=big[1:], S=S,
+                                      workspace=nv.Workspace(256, K), dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert_same_q(xa, orc.rmsnorm_reorder_quantize(x, gamma, 1e-5, perm, S))
