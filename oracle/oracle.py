@@ -24,7 +24,9 @@ Page citations (page title, section):
 
 Parity status: every function below is pinned by tests/test_oracle_*.py
 (exhaustive code tables, library cross-checks, brute force, closed forms and
-the pages' error bounds); the MXFP4 functions at the end by
+the pages' error bounds); the rounding of the residue stages (dequant_f32,
+residue, mx_residue) by exact-rational recomputation in
+tests/test_oracle_residue_rounding.py; the MXFP4 functions at the end by
 tests/test_oracle_mx.py.
 """
 from __future__ import annotations
@@ -356,14 +358,20 @@ def mx_dequant(codes, scales) -> np.ndarray:
     return out
 
 
+def mx_residue(x, qx) -> np.ndarray:
+    """R = fl32(x - deq(Q(x))) in MXFP4 ([RS] abstract: what quantization lost).
+    deq = v(code) * 2^(b - 127) is exact in binary32, so only the subtraction rounds."""
+    x = _f32(x)
+    return (x - mx_dequant(*qx).astype(np.float32)).astype(np.float32)
+
+
 def mx_quantize_residue(x):
     """ResServe's residue in MXFP4 ([RS] abstract: FP4 base plus FP4 residue):
     R = fl32(x - deq(Q(x))), quantized with its own block scales.
     Returns ((codes, scales) of X, (codes, scales) of R)."""
     x = _f32(x)
     qx = mx_quantize(x)
-    r = (x - mx_dequant(*qx).astype(np.float32)).astype(np.float32)
-    return qx, mx_quantize(r)
+    return qx, mx_quantize(mx_residue(x, qx))
 
 
 def mx_gemm(qa, qw, qr=None) -> np.ndarray:
