@@ -448,7 +448,7 @@ class PrefillWorkload:
         g = torch.Generator(device="cpu").manual_seed(0)
         for (N, K) in self.shapes:
             x = wl.to_bf16(wl.prefill_x(self.M, K)).to(dev)
-            perm = torch.from_numpy(wl.calibrated_perm(wl.prefill_x(64, K))).to(dev)
+            perm = torch.from_numpy(wl.prefill_perm(K)).to(dev)
             w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
             qw = nv.NVFP4Tensor.empty(N, K, nv.SF_TILED, device=dev)
             nv.nvfp4_quantize(w, qw, workspace=nv.Workspace(N, K, dev))
@@ -834,7 +834,7 @@ def profile_case(case: str) -> int:
     elif case == "reorder":
         M, K, S = 8192, 4096, 256
         x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
-        perm = torch.from_numpy(wl.calibrated_perm(wl.prefill_x(64, K))).to(dev)
+        perm = torch.from_numpy(wl.prefill_perm(K)).to(dev)
         q = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED, device=dev)
         ws = nv.Workspace(M, K, dev)
         for _ in range(3):

@@ -120,3 +120,9 @@ def arc_inputs(M: int = ARC_M, K: int = ARC_K, n_calib: int = 512):
 def prefill_x(M: int, K: int) -> np.ndarray:
     """Large prefill activations: bf16 N(0,1), 1% channels x50."""
     return bf16_values(activations_normal(M, K, 0.01, 50.0))
+
+
+def prefill_perm(K: int, n_calib: int = 512) -> np.ndarray:
+    """Channel order for the large prefill's S-column extension, from n_calib
+    calibration rows (seed 1) of the prefill distribution (same outlier channels)."""
+    return calibrated_perm(activations_normal(n_calib, K, 0.01, 50.0, SEED_CALIB))

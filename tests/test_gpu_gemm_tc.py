@@ -149,6 +149,45 @@ def test_arcquant_augmented_gemm(orc, S):
     assert err <= REL_FRO_TOL, err
 
 
+@pytest.mark.parametrize("N,K", wl.PREFILL_SHAPES)
+def test_large_prefill_k_plus_s_end_to_end(orc, N, K):
+    """The large prefill with the S = 256 outlier-residue extension at full size
+    (ARCQuant blog post section 3.1: K -> K+S as one GEMM): the reorder quantizer
+    without normalisation writes X_aug (M x (K+S)), the GEMM multiplies it by
+    W_aug = [W' | W'_o].  Codes and scales are compared byte for byte on sampled
+    rows, Y on sampled rows and columns."""
+    S = 256
+    M = wl.PREFILL_M
+    x = wl.prefill_x(M, K)
+    perm = wl.prefill_perm(K)
+    xa = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws = nv.Workspace(M, K)
+    nv.nvfp4_rmsnorm_reorder_quantize(to_dev(x), xa, perm=torch.from_numpy(perm).cuda(), S=S, workspace=ws,
+                                      dev_status=st)
+    w_aug = orc.augment_weight(wl.weights_normal(N, K), perm, S)
+    qw = run_quantize(to_dev(w_aug, torch.float32), nv.SF_TILED)
+    y = run_gemm(xa, qw)
+    assert st.item() == 0, nv.status_string(st.item())
+    assert int(ws.buf.count_nonzero()) == 0, "workspace not left zeroed"
+    rng = np.random.default_rng(K + N)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 64, replace=False)]))
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 256, replace=False)]))
+    s_aug = orc.tensor_scale(np.abs(x).max())   # no normalisation: the reorder keeps amax
+    ox = orc.rmsnorm_reorder_quantize(x[rows], None, perm=perm, S=S, s=s_aug)
+    rows_t = torch.from_numpy(rows).cuda()
+    np.testing.assert_array_equal(xa.codes[rows_t].cpu().numpy(), ox.codes, err_msg="X_aug codes")
+    np.testing.assert_array_equal(xa.scales_rowmajor()[rows_t].cpu().numpy(), ox.scales, err_msg="X_aug scales")
+    assert np.float32(xa.tensor_scale.item()) == s_aug
+    ow = orc.quantize(w_aug[cols], orc.tensor_scale(np.abs(w_aug).max()))
+    cols_t = torch.from_numpy(cols).cuda()
+    np.testing.assert_array_equal(qw.codes[cols_t].cpu().numpy(), ow.codes, err_msg="W_aug codes")
+    np.testing.assert_array_equal(qw.scales_rowmajor()[cols_t].cpu().numpy(), ow.scales, err_msg="W_aug scales")
+    ys = y[rows_t][:, cols_t].cpu().numpy()
+    err = rel_fro(ys, orc.gemm(ox, ow))
+    assert err <= REL_FRO_TOL, err
+
+
 # ------------------------------------------- ResServe residue on the large-M GEMM
 
 @pytest.mark.parametrize("M,N,K", [(256, 512, 1024), (200, 300, 320), (1000, 130, 576), (129, 1000, 4224)])
