@@ -781,7 +781,12 @@ def profile_case(case: str) -> int:
     reorder  -- nvfp4_rmsnorm_reorder_quantize of the same activations, S=256
     mxgemm   -- nvfp4_mx_gemm, M=8192, (N,K)=(14336,4096), MXFP4 operands with TILED scales
     arcquant -- nvfp4_rmsnorm_reorder_quantize on the ARCQuant prefill activations
-                (2048x4096 bf16, gamma, calibrated perm, S=256)."""
+                (2048x4096 bf16, gamma, calibrated perm, S=256)
+    gemv     -- nvfp4_gemm on ROWMAJOR operands (CUDA-core GEMV), M=1, (N,K)=(4096,14336),
+                5 weight copies (165 MB)
+    gemv_tc  -- nvfp4_gemm_residue, M=64, (N,K)=(5120,27648) (ResServe decode), TILED
+                operands, 3 weight copies (239 MB)
+    mxquant  -- nvfp4_mx_quantize of the 8192x4096 bf16 prefill activations (67 MB), TILED."""
     import nvfp4_block_scaled_18_b200 as nv
     from nvfp4_block_scaled_18_b200 import workloads as wl
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -831,6 +836,40 @@ def profile_case(case: str) -> int:
         ws = nv.Workspace(M, K, dev)
         for i in range(3):
             nv.nvfp4_rmsnorm_reorder_quantize(xs[i], q, gamma=g, eps=1e-5, perm=p, S=S, workspace=ws)
+    elif case == "gemv":
+        M, N, K = 1, 4096, 14336
+        w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
+        ws = []
+        for _ in range(5):
+            q = nv.NVFP4Tensor.empty(N, K, nv.SF_ROWMAJOR, device=dev)
+            nv.nvfp4_quantize(w, q, workspace=nv.Workspace(N, K, dev))
+            ws.append(q)
+        qx = nv.NVFP4Tensor.empty(M, K, nv.SF_ROWMAJOR, device=dev)
+        nv.nvfp4_quantize(wl.to_bf16(wl.decode_x(M, K)).to(dev), qx, workspace=nv.Workspace(M, K, dev))
+        y = torch.empty((M, N), device=dev)
+        for i in range(10):
+            nv.nvfp4_gemm(qx, ws[i % 5], y)
+    elif case == "gemv_tc":
+        M, N, K = 64, 5120, 27648
+        w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
+        ws = []
+        for _ in range(3):
+            q = nv.NVFP4Tensor.empty(N, K, nv.SF_TILED, device=dev)
+            nv.nvfp4_quantize(w, q, workspace=nv.Workspace(N, K, dev))
+            ws.append(q)
+        q = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev)
+        r = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev)
+        nv.nvfp4_quantize_residue(wl.to_bf16(wl.resserve_x(M, K)).to(dev), q, r, workspace=nv.Workspace(M, K, dev))
+        y = torch.empty((M, N), device=dev)
+        for i in range(6):
+            nv.nvfp4_gemm_residue(q, r, ws[i % 3], y)
+    elif case == "mxquant":
+        M, K = 8192, 4096
+        x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
+        c = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        sc = torch.empty(nv.mx_scales_bytes(M, K, nv.SF_TILED), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            nv.nvfp4_mx_quantize(x, c.view(-1), sc, sf_layout=nv.SF_TILED)
     elif case == "reorder":
         M, K, S = 8192, 4096, 256
         x = wl.to_bf16(wl.prefill_x(M, K)).to(dev)
@@ -865,7 +904,8 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="decode: launch every step directly on the stream (no CUDA graphs) and skip the "
                          "per-call detail; for profilers that cannot follow graph replays")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder", "mxgemm", "arcquant"],
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder", "mxgemm", "arcquant", "gemv", "gemv_tc",
+                                               "mxquant"],
                     help="run a few launches of one kernel on a small case (for ncu captures) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
