@@ -125,6 +125,31 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64
                                             nvfp4_tensor* x_aug, void* workspace, size_t ws_bytes,
                                             int* dev_status, void* stream);
 
+/* Offline weight preparation for the augmented linear (ARCQuant post sections
+ * 3.1 and 6.3: the weight takes the activations' channel order and repeats its
+ * S outlier columns, so that one GEMM over K+S columns also multiplies the
+ * activation residue; OSFP4 page, abstract: a per-channel smoothing vector is
+ * absorbed as W diag(sigma) on the weight side and 1/sigma in the RMSNorm gain
+ * of the activation side):
+ *   W'[:, j] = fl32(W[:, perm[j]] * sigma[perm[j]])   (sigma NULL: W[:, perm[j]])
+ *   W_aug    = [W' | W'[:, 0..S)]                      (N x (K+S))
+ *   s_w      = scale_in ? *scale_in : fl32(amax|W'| / 2688)
+ *   w_aug    = Q(W_aug) under s_w, as nvfp4_quantize (its last S columns repeat
+ *              the first S columns' codes and block scales).
+ * w: device, N x K of dtype dt, row stride ldw >= K (elements), aligned to
+ *   the element size; K % 16 == 0.
+ * sigma: device float[K] or NULL; perm: device int32[K], a permutation of
+ *   0..K-1, or NULL (identity); an entry outside 0..K-1 is reported as
+ *   NVFP4_ERR_INVALID_ARG through dev_status and never indexed.
+ * S: 0 <= S <= K, S % 16 == 0.  w_aug: rows == N, cols == K + S, either scale
+ *   layout.  workspace: >= nvfp4_workspace_size(N, K) bytes when scale_in is
+ *   NULL.  The weight is read with gathers through perm: this is the offline
+ *   step, not tuned for speed. */
+nvfp4_status nvfp4_quantize_weight(const void* w, nvfp4_dtype dt, int64_t N, int64_t K, int64_t ldw,
+                                   const float* sigma, const int32_t* perm, int64_t S, const float* scale_in,
+                                   nvfp4_tensor* w_aug, void* workspace, size_t ws_bytes, int* dev_status,
+                                   void* stream);
+
 /* Block-scaled W4A4 linear: Y = s_a s_w * A W^T with A (M x K) and W (N x K)
  * NVFP4, fp32 accumulation, output dtype out_dt (row stride ldy).
  * ARCQuant's K -> K+S compensation is this call with K+S columns
@@ -270,6 +295,20 @@ nvfp4_status nvfp4_mx_gemm_residue(const uint8_t* a_codes, const uint8_t* a_scal
                                    const uint8_t* r_scales, const uint8_t* w_codes, const uint8_t* w_scales,
                                    int64_t M, int64_t N, int64_t K, void* y, nvfp4_dtype out_dt, int64_t ldy,
                                    int* dev_status, void* stream);
+
+/* Test support for the device-side bounded waits (failure detection around
+ * the method; the pages have no counterpart).  Every mbarrier wait of the
+ * tensor-core kernels (nvfp4_gemm, nvfp4_gemm_residue, the fused decode
+ * linears, the MXFP4 GEMMs) gives up after limit_ns nanoseconds (default 4 s;
+ * 0 restores it), records NVFP4_ERR_TIMEOUT in *dev_status and lets the launch
+ * finish: each CTA first lets its own bulk copies and MMAs in flight and the
+ * bytes its cluster peers send complete, then releases its tensor memory and
+ * exits, so the context stays usable.  withhold != 0 makes those kernels skip
+ * loading their weight tiles (the large-M GEMM: every operand tile), so that
+ * their waits run out: a way to exercise the timeout path that faults nothing.
+ * Output contents of a launch that timed out are unspecified.  The setting is
+ * process wide, read when a launch is made, and meant for tests only. */
+void nvfp4_test_wait_fault(uint64_t limit_ns, int withhold);
 
 /* Human-readable name of a status code (static string). */
 const char* nvfp4_status_string(nvfp4_status status);

@@ -28,7 +28,8 @@ EXPORTED_SYMBOLS = ("nvfp4_scales_bytes", "nvfp4_workspace_size", "nvfp4_quantiz
                     "nvfp4_gemm_residue", "nvfp4_quantize_gemm", "nvfp4_quantize_residue_gemm",
                     "nvfp4_quantize_gemm_plan",
                     "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_mx_quantize",
-                    "nvfp4_mx_scales_bytes", "nvfp4_mx_gemm", "nvfp4_mx_gemm_residue", "nvfp4_status_string", "nvfp4_version")
+                    "nvfp4_mx_scales_bytes", "nvfp4_mx_gemm", "nvfp4_mx_gemm_residue", "nvfp4_quantize_weight", "nvfp4_test_wait_fault", "nvfp4_status_string",
+                    "nvfp4_version")
 NVFP4_NOALLOC_MAX_ROWS = 65536
 
 
@@ -82,6 +83,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                    "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_gemm", "nvfp4_gemm_residue",
                    "nvfp4_mx_quantize", "nvfp4_mx_gemm", "nvfp4_mx_gemm_residue"):
             getattr(lib, fn).restype = ctypes.c_int
+        lib.nvfp4_quantize_weight.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, I64, P, T, P, SZ, P, P]
+        lib.nvfp4_quantize_weight.restype = ctypes.c_int
+        lib.nvfp4_test_wait_fault.argtypes = [ctypes.c_uint64, ctypes.c_int]
+        lib.nvfp4_test_wait_fault.restype = None
         lib.nvfp4_status_string.argtypes = [ctypes.c_int]
         lib.nvfp4_status_string.restype = ctypes.c_char_p
         lib.nvfp4_version.restype = ctypes.c_char_p
@@ -94,6 +99,14 @@ def status_string(status: int) -> str:
         return load_library().nvfp4_status_string(int(status)).decode()
     except RuntimeError:
         return STATUS_NAMES.get(status, "unknown")
+
+
+def nvfp4_test_wait_fault(limit_ns: int = 0, withhold: bool = False) -> None:
+    """Test support: bound every device-side wait of the tensor-core kernels by
+    limit_ns (0 = the default 4 s); withhold=True makes the following launches
+    skip their weight-tile loads so that the waits run out (NVFP4_ERR_TIMEOUT
+    in dev_status).  Process wide; for tests only."""
+    load_library().nvfp4_test_wait_fault(int(limit_ns), 1 if withhold else 0)
 
 
 def nvfp4_version() -> str:
@@ -288,6 +301,25 @@ def nvfp4_rmsnorm_reorder_quantize(x: torch.Tensor, x_aug: NVFP4Tensor,
                                               ctypes.byref(xc), ws_ptr, ws_n, _ptr(dev_status),
                                               _stream(stream)),
            "nvfp4_rmsnorm_reorder_quantize")
+
+
+def nvfp4_quantize_weight(w: torch.Tensor, w_aug: NVFP4Tensor, sigma: Optional[torch.Tensor] = None,
+                          perm: Optional[torch.Tensor] = None, S: int = 0,
+                          scale_in: Optional[torch.Tensor] = None, workspace: Optional[Workspace] = None,
+                          dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Offline weight preparation: w_aug = Q([W' | W'[:, :S]]), W'[:, j] = W[:, perm[j]] * sigma[perm[j]]."""
+    lib = load_library()
+    N, K = w.shape
+    if sigma is not None and sigma.dtype != torch.float32:
+        raise TypeError("sigma must be float32")
+    if perm is not None and perm.dtype != torch.int32:
+        raise TypeError("perm must be int32")
+    wc = w_aug.c()
+    ws_ptr, ws_n = (workspace.ptr(), workspace.nbytes) if workspace is not None else (None, 0)
+    _check(lib.nvfp4_quantize_weight(w.data_ptr(), _dtype_code(w), N, K, _ldx(w), _ptr(sigma), _ptr(perm), S,
+                                     _ptr(scale_in), ctypes.byref(wc), ws_ptr, ws_n, _ptr(dev_status),
+                                     _stream(stream)),
+           "nvfp4_quantize_weight")
 
 
 def nvfp4_rmsnorm_reorder_quantize_noalloc(x: torch.Tensor, x_aug: NVFP4Tensor,

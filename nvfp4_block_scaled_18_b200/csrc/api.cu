@@ -1,8 +1,10 @@
 // C-ABI entry points declared in include/nvfp4.h: argument validation on the
 // host, then kernel launches on the caller's stream.  No allocation, no
-// global state beyond a per-device SM-count cache.
+// global state beyond a per-device SM-count cache and the bounded-wait test
+// setting.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -12,6 +14,9 @@
 using namespace nvfp4;
 
 namespace {
+
+std::atomic<uint64_t> g_wait_limit_ns{tc_wait_default_ns()};
+std::atomic<int> g_wait_hold{0};
 
 int num_sms_current_device() {
   static int cache[64] = {0};
@@ -142,7 +147,16 @@ nvfp4_status run_mx_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const 
 
 }  // namespace
 
+namespace nvfp4 {
+WaitTest wait_test() { return WaitTest{g_wait_limit_ns.load(), g_wait_hold.load()}; }
+}  // namespace nvfp4
+
 extern "C" {
+
+void nvfp4_test_wait_fault(uint64_t limit_ns, int withhold) {
+  g_wait_limit_ns.store(limit_ns == 0 ? tc_wait_default_ns() : limit_ns);
+  g_wait_hold.store(withhold != 0 ? 1 : 0);
+}
 
 size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout) {
   if (rows <= 0 || cols <= 0) return 0;
@@ -237,6 +251,23 @@ nvfp4_status nvfp4_rmsnorm_reorder_quantize(const void* x, nvfp4_dtype dt, int64
   // a programmatic dependent of the statistics pass, when there is one
   return cuda_status(launch_reorder_quant(x, dt, M, K, ldx, gamma, rinv, perm, S, s_ptr, qout(x_aug),
                                           dev_status, sms, s, gamma != nullptr || scale_in == nullptr));
+}
+
+nvfp4_status nvfp4_quantize_weight(const void* w, nvfp4_dtype dt, int64_t N, int64_t K, int64_t ldw,
+                                   const float* sigma, const int32_t* perm, int64_t S, const float* scale_in,
+                                   nvfp4_tensor* w_aug, void* workspace, size_t ws_bytes, int* dev_status,
+                                   void* stream) {
+  if (w == nullptr || !dt_ok(dt) || N <= 0 || K <= 0 || ldw < K || K % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(w) % dt_size(dt)) != 0) return NVFP4_ERR_ALIGNMENT;
+  if (S < 0 || S > K || S % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if ((sigma != nullptr && (reinterpret_cast<uintptr_t>(sigma) & 3u)) ||
+      (perm != nullptr && (reinterpret_cast<uintptr_t>(perm) & 3u)))
+    return NVFP4_ERR_ALIGNMENT;
+  NVFP4_TRY(check_tensor(w_aug, N, K + S));
+  if (scale_in == nullptr) NVFP4_TRY(check_ws(workspace, ws_bytes, N, K));
+  return cuda_status(launch_weight_quant(w, dt, N, K, ldw, sigma, perm, S, scale_in, qout(w_aug),
+                                         static_cast<WsHeader*>(workspace), dev_status, num_sms_current_device(),
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_tensor* a, const nvfp4_tensor* w, void* y, nvfp4_dtype out_dt,

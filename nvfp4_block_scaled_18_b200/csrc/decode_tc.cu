@@ -73,7 +73,8 @@ constexpr int NP = 16;                       // activation rows, padded
 constexpr int W_TILE = 128 * 128;            // 128 W rows x 256 K-elements
 constexpr int SFW_BYTES = 4 * 512;           // one scale atom per K=64 chunk
 constexpr int WSTAGE = W_TILE + SFW_BYTES;   // 18 KB, keeps 1024-byte alignment
-constexpr int STAGES = 2;
+constexpr int MAX_STAGES = 8;                // W ring depth limit; the launch picks p.stages in [2, 8]
+constexpr int SF_BUFS = 2;                   // TMEM scale buffers, alternating by k-tile
 constexpr int X_TILE = NP * 128;             // codes of one operand (X or R) in one k-tile (SW128)
 constexpr int SF_TILE = 4 * 128;             // activation scales of one k-tile: 4 K=64 chunks x 32 rows
                                              // (rows 0-15 X, 16-31 R) x 4 block scales
@@ -95,13 +96,13 @@ constexpr int max_part_rows() {
   return m;
 }
 constexpr int PART_ROWS = max_part_rows();   // 133 (ks = 7)
-// TMEM columns: acc [0,32) (X products in 0-15, R products in 16-31), then one
-// scale buffer per ring stage: W scales [+0,+16), X/R scales [+16,+32)
+// TMEM columns: acc [0,32) (X products in 0-15, R products in 16-31), then two
+// scale buffers used by alternate k-tiles: W scales [+0,+16), X/R scales [+16,+32)
 constexpr uint32_t ACC = 0, SF_COL = 32, SF_BUF = 32, SFX_OFF = 16, TMEM_COLS = 128;   // R products: column ro
 static_assert(SFX_OFF == 16 && SF_BUF >= 32, "one 32-column TMEM store writes a stage's W and X scales");
 static_assert(SF_COL % 4 == 0 && SF_BUF % 4 == 0 && SFX_OFF % 4 == 0,
               "block-scaled MMA scale operands start on 4-column TMEM boundaries");
-static_assert(SF_COL + STAGES * SF_BUF <= TMEM_COLS, "TMEM columns");
+static_assert(SF_COL + SF_BUFS * SF_BUF <= TMEM_COLS, "TMEM columns");
 constexpr int TMEM_CTAS = 512 / TMEM_COLS;
 
 static_assert(WSTAGE % 1024 == 0 && X_TILE % 1024 == 0, "SW128 tiles need 1024-byte alignment");
@@ -109,7 +110,7 @@ static_assert(PART_ROWS == 133, "slot count for ks <= 8");
 // one pushed vector per row: the partial X product, or with a residue the
 // already scaled sum s_x s_w acc_x + s_r s_w acc_r
 __host__ __device__ constexpr int part_bytes(int M) { return PART_ROWS * part_pitch(M) * 4; }
-static_assert((3 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier block");
+static_assert((2 * MAX_STAGES + SF_BUFS + 5) * 8 + 16 + 8 <= BAR_BYTES, "barrier block");
 
 struct DecodeParams {
   const void* x;        // fused: activations, M x K (ldx), bf16 or fp32
@@ -130,15 +131,18 @@ struct DecodeParams {
   int katoms_w;         // scale atoms per 128-row group of W = K / 64
   int k_tiles;          // ceil(K / 256)
   int kt_max;           // k-tiles per CTA held in the activation area
+  int stages;           // W ring depth, 2..MAX_STAGES
   int* st;
+  uint64_t wait_ns;     // bound on every mbarrier wait
+  int hold;             // test of the timeout path: no W tile is loaded
 };
 
 // u / d for u < 2^16, d < 2^16 with m = ceil(2^32 / d): the error u*(m - 2^32/d)/2^32
 // stays below 1/d, so the quotient is exact.
 __device__ __forceinline__ int div_magic(int u, uint32_t m) { return (int)__umulhi((uint32_t)u, m); }
 
-__host__ __device__ constexpr int smem_bytes(int kt_max, int ro, int M) {
-  return 1024 + STAGES * WSTAGE + kt_max * (b_tile(ro) + SF_TILE) + part_bytes(M) + BAR_BYTES;
+__host__ __device__ constexpr int smem_bytes(int stages, int kt_max, int ro, int M) {
+  return 1024 + stages * WSTAGE + kt_max * (b_tile(ro) + SF_TILE) + part_bytes(M) + BAR_BYTES;
 }
 
 template <typename T, bool FUSED, int RES, bool BF16OUT, int R>
@@ -148,7 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int KT = p.kt_max;
-  uint8_t* xcodes = smem + STAGES * WSTAGE;                         // KT x 2 KB
+  const int NS = p.stages;                                          // W ring depth
+  uint8_t* xcodes = smem + NS * WSTAGE;                             // KT x 2 KB
   constexpr int BT = b_tile(RES);                                   // B tile bytes per k-tile
   constexpr int OPR = operand_rows(RES);                            // rows of X (and of R)
   uint8_t* rcodes = xcodes + RES * 128;                             // R rows of each B tile
@@ -157,15 +162,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pitch = part_pitch(p.M);
   float* part = reinterpret_cast<float*>(sfxp + KT * SF_TILE);      // pushed partial rows
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(part) + part_bytes(p.M));
-  uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* full = bars;                                            // [NS] W stage landed
+  uint64_t* empty = bars + MAX_STAGES;                              // [NS] MMAs of the stage's k-tile done
+  uint64_t* acc_full = bars + 2 * MAX_STAGES;
   uint64_t* x_full = acc_full + 1;
-  uint64_t* sf_full = x_full + 1;                                   // [STAGES] scales written to TMEM
-  uint64_t* xbar = sf_full + STAGES;                                // [2] peers' |x|, |r| maxima arrived
+  uint64_t* sf_full = x_full + 1;                                   // [SF_BUFS] scale buffer written to TMEM
+  uint64_t* xbar = sf_full + SF_BUFS;                               // [2] peers' |x|, |r| maxima arrived
   uint64_t* pbar = xbar + 2;                                        // peers' partial rows arrived
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  WaitState* abort_flag = reinterpret_cast<WaitState*>(pbar + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(abort_flag + 1);
   __shared__ uint32_t red[kWarps];
   __shared__ uint32_t xall[2][MAX_KS];                              // every CTA's |x|, |r| maximum
 
@@ -183,11 +188,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool r_exchange = FUSED && RES && p.sr_in == nullptr;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(saddr(&full[s]), 1);
       mbar_init(saddr(&empty[s]), 1);
-      mbar_init(saddr(&sf_full[s]), 4);   // one arrival per scale warp
     }
+    for (int b = 0; b < SF_BUFS; ++b) mbar_init(saddr(&sf_full[b]), 4);   // one arrival per scale warp
     mbar_init(saddr(acc_full), 1);
     mbar_init(saddr(x_full), 1);
     for (int i = 0; i < 2; ++i) mbar_init(saddr(&xbar[i]), 1);
@@ -198,7 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (r_exchange) mbar_expect_tx(saddr(&xbar[1]), (ks - 1u) * 4u);
     const uint32_t owned = (uint32_t)(owner_row0(rank + 1) - owner_row0(rank));
     mbar_expect_tx(saddr(pbar), (ks - 1u) * owned * (uint32_t)(pitch * 4));
-    *abort_flag = 0;
+    abort_flag->abort = 0;
+    abort_flag->limit_ns = p.wait_ns;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -253,7 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  const int pre = min(nkt, STAGES);
+  const int pre = p.hold ? 0 : min(nkt, NS);   // every stage of the ring is loaded at once
+  int issued = pre;   // W stages loaded (warp 0 lane 0)
   if (warp == 0 && lane == 0) {
     if (!FUSED) {
       mbar_expect_tx(saddr(x_full), (uint32_t)(nkt * BT));
@@ -277,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x < ks && threadIdx.x != rank)
       st_async_u32(mapa_shared(saddr(&xall[which][rank]), threadIdx.x), m,
                    mapa_shared(saddr(&xbar[which]), threadIdx.x));
-    (void)mbar_wait<true>(saddr(&xbar[which]), 0u, abort_flag, p.st);
+    (void)mbar_drain<true>(saddr(&xbar[which]), 0u, abort_flag, p.st);   // peers send on every path
     return max(m, warp_max_u32(lane < (int)ks && lane != (int)rank ? xall[which][lane] : 0u));
   };
 
@@ -390,25 +397,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------- W producer (rest of the ring)
-    int s = pre % STAGES;
-    uint32_t ph = (pre == STAGES) ? 1u : 0u;
-    for (int kt = kt0 + pre; kt < kt1; ++kt) {
+    int s = pre % NS;
+    uint32_t ph = (pre == NS) ? 1u : 0u;
+    for (int kt = kt0 + pre; !p.hold && kt < kt1; ++kt, ++issued) {
       if (!mbar_wait(saddr(&empty[s]), ph ^ 1u, abort_flag, p.st)) break;
       load_w(kt, s);
-      if (++s == STAGES) { s = 0; ph ^= 1u; }
+      if (++s == NS) { s = 0; ph ^= 1u; }
     }
+    // the last NS stages' copies (and the activation codes) may still be in
+    // flight if a consumer gave up: let them land before the CTA can exit
+    for (int g2 = max(0, issued - NS); g2 < issued; ++g2)
+      (void)mbar_drain(saddr(&full[g2 % NS]), (uint32_t)((g2 / NS) & 1), abort_flag, p.st);
+    if (!FUSED) (void)mbar_drain(saddr(x_full), 0u, abort_flag, p.st);
   } else if (warp >= 4) {
     // ------------------------------------------- scales into TMEM (tcgen05.st)
-    // Warp w writes TMEM lane quadrant w - 4 of stage s's scale buffer: line l
-    // of each W atom, then of the k-tile's activation atoms, in every lane l of
-    // the quadrant (the layout a 32x128b.warpx4 copy of the same atoms gives).
-    // Scale copies issued to the tensor pipe would queue behind the stream of
-    // W tiles; these stores do not.  A stage is refilled only after the MMAs
-    // that read it (and its scale buffer) have completed, so waiting for the
-    // stage's data is enough before overwriting the buffer.
+    // Warp w writes TMEM lane quadrant w - 4 of scale buffer t & 1 for the
+    // CTA's k-tile t: line l of each W atom, then of the k-tile's activation
+    // atoms, in every lane l of the quadrant (the layout a 32x128b.warpx4 copy
+    // of the same atoms gives).  Scale copies issued to the tensor pipe would
+    // queue behind the stream of W tiles; these stores do not.  Buffer t & 1
+    // was last read by the MMAs of k-tile t - 2, so its stores wait for that
+    // k-tile's commit (the ring has at least two stages, so that commit's phase
+    // is still the current one of its barrier).
     const uint32_t quad = (uint32_t)((warp - 4) * 32) << 16;
-    auto write_stage = [&](int kt, int s) {
-      const int t = kt - kt0;
+    auto write_tile = [&](int t, int s) {
       const uint8_t* sb = smem + s * WSTAGE;
       uint32_t r[32];
 #pragma unroll
@@ -419,64 +431,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         r[16 + 4 * j] = *reinterpret_cast<const uint32_t*>(sfxp + t * SF_TILE + j * 128 + lane * 4);
         r[16 + 4 * j + 1] = 0u; r[16 + 4 * j + 2] = 0u; r[16 + 4 * j + 3] = 0u;
       }
-      tmem_st32(tmem + quad + SF_COL + (uint32_t)s * SF_BUF, r);   // W scales, then X (and R) scales
+      tmem_st32(tmem + quad + SF_COL + (uint32_t)(t & 1) * SF_BUF, r);   // W scales, then X (and R) scales
     };
-    int s = 0;
-    uint32_t ph = 0;
-    for (int kt = kt0; kt < kt1;) {
+    auto buf_free = [&](int t) {   // the MMAs of k-tile t - 2 have completed
+      return t < 2 || mbar_test_wait(saddr(&empty[(t - 2) % NS]), (uint32_t)(((t - 2) / NS) & 1));
+    };
+    for (int t = 0; t < nkt;) {
       // every lane waits; the warp goes on only if all saw the phase (the
       // TMEM store is warp-collective)
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(saddr(&full[s]), ph, abort_flag, p.st))) break;
+      if (t >= 2 && !__all_sync(0xFFFFFFFFu, mbar_wait(saddr(&empty[(t - 2) % NS]),
+                                                       (uint32_t)(((t - 2) / NS) & 1), abort_flag, p.st)))
+        break;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(saddr(&full[t % NS]), (uint32_t)((t / NS) & 1), abort_flag, p.st)))
+        break;
       tc_fence_after();
-      write_stage(kt, s);
-      // the next stage joins the batch if it has landed too: one wait covers
-      // both stores
-      const int s2 = s + 1 == STAGES ? 0 : s + 1;
-      const uint32_t ph2 = s2 == 0 ? ph ^ 1u : ph;
-      const bool two = kt + 1 < kt1 && __all_sync(0xFFFFFFFFu, mbar_test_wait(saddr(&full[s2]), ph2));
+      write_tile(t, t % NS);
+      // k-tile t + 1 joins the batch if its stage has landed and its buffer is
+      // free: one wait covers both stores
+      const bool two = t + 1 < nkt &&
+                       __all_sync(0xFFFFFFFFu, buf_free(t + 1) && mbar_test_wait(saddr(&full[(t + 1) % NS]),
+                                                                                 (uint32_t)(((t + 1) / NS) & 1)));
       if (two) {
         tc_fence_after();
-        write_stage(kt + 1, s2);
+        write_tile(t + 1, (t + 1) % NS);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(saddr(&sf_full[s]));
-        if (two) mbar_arrive(saddr(&sf_full[s2]));
+        mbar_arrive(saddr(&sf_full[t & 1]));
+        if (two) mbar_arrive(saddr(&sf_full[(t + 1) & 1]));
       }
-      for (int n = 0; n < (two ? 2 : 1); ++n, ++kt)
-        if (++s == STAGES) { s = 0; ph ^= 1u; }
+      t += two ? 2 : 1;
     }
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------- MMA issuer
     bool ok = true;
     if (!FUSED) ok = mbar_wait(saddr(x_full), 0u, abort_flag, p.st);
     const uint32_t idesc = idesc_nvf4(RES == 16 ? 2 * NP : NP);
-    int s = 0;
-    uint32_t ph = 0;
-    for (int kt = kt0; ok && kt < kt1; ++kt) {
-      if (!mbar_wait(saddr(&full[s]), ph, abort_flag, p.st)) break;
-      if (!mbar_wait(saddr(&sf_full[s]), ph, abort_flag, p.st)) break;
+    for (int t = 0; ok && t < nkt; ++t) {
+      const int s = t % NS;
+      if (!mbar_wait(saddr(&full[s]), (uint32_t)((t / NS) & 1), abort_flag, p.st)) break;
+      if (!mbar_wait(saddr(&sf_full[t & 1]), (uint32_t)((t >> 1) & 1), abort_flag, p.st)) break;
       tc_fence_after();
-      const int t = kt - kt0, jmax = w_chunks(kt);
+      const int kt = kt0 + t, jmax = w_chunks(kt);
       const uint8_t* sb = smem + s * WSTAGE;
-      const uint32_t sfw = SF_COL + (uint32_t)s * SF_BUF, sfx = sfw + SFX_OFF;
+      const uint32_t sfw = SF_COL + (uint32_t)(t & 1) * SF_BUF, sfx = sfw + SFX_OFF;
       const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(xcodes + t * BT));
       for (int j = 0; j < jmax; ++j) {
-        const uint32_t acc = (kt > kt0 || j > 0) ? 1u : 0u;
+        const uint32_t acc = (t > 0 || j > 0) ? 1u : 0u;
         tc_mma_nvf4(tmem + ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + sfw + 4 * j,
                     tmem + sfx + 4 * j, acc);
       }
       tc_commit(saddr(&empty[s]));
-      if (++s == STAGES) { s = 0; ph ^= 1u; }
     }
     tc_commit(saddr(acc_full));
   }
   __syncwarp();
 
   // ------------------- push this CTA's partial rows to the CTA that owns them
-  const bool ok = mbar_wait(saddr(acc_full), 0u, abort_flag, p.st);
+  // the commit after the MMA loop is issued on every path: waiting for it also
+  // waits for every MMA in flight, before TMEM is read and released
+  const bool ok = mbar_drain(saddr(acc_full), 0u, abort_flag, p.st) && !wait_aborted(abort_flag);
   tc_fence_after();
   __syncwarp();     // the cluster barrier below is warp-aligned
   if (!peers_running) cluster_wait();   // uniform: no maximum was exchanged
@@ -534,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();  // own partial rows stored; TMEM reads done before the dealloc
   // Every peer's partial rows have landed here.  Each CTA also waits for all
   // bytes addressed to it before it exits, so no store targets an exited CTA.
-  (void)mbar_wait<true>(saddr(pbar), 0u, abort_flag, p.st);
+  (void)mbar_drain<true>(saddr(pbar), 0u, abort_flag, p.st);
 
   // ------------------------------------------------ owners sum their rows and store
   {
@@ -566,33 +582,47 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ host side
 
 constexpr double kFixedUs = 5.0;     // launch-to-exit latency of one wave of CTAs (measured, few k-tiles)
-constexpr double kTileUs = 0.8;      // issue time of one k-tile (8 scale copies, 4 MMAs, 1 commit) per CTA
+constexpr double kTileUs = 0.8;      // one k-tile (scale stores, 4 MMAs, 1 commit) per CTA, up to 4 CTAs per SM
 constexpr double kQuantUs = 4.0;     // one-launch quantizer plus the hand-off to the next kernel
 constexpr double kExchangeUs = 1.3;  // fused: one cluster-wide maximum (stores into peers + wait)
 constexpr double kUnitUs = 0.15;     // fused: encoding one 8-element unit per thread, per co-resident CTA
+// A request of at least this many bytes keeps at most TMEM_CTAS CTAs on an SM
+// (228 KB per SM, 1 KB reserved per CTA), so tcgen05.alloc never waits for a
+// CTA of another cluster.
+constexpr int kSmemFloor = 233472 / (TMEM_CTAS + 1) - 1024 + 16;
+static_assert((kSmemFloor + 1024) * (TMEM_CTAS + 1) > 233472, "smem floor");
 
 struct Choice {
-  int ks = 0, kt_max = 0, smem = 0;
+  int ks = 0, kt_max = 0, stages = 0, smem = 0;
   double cost = 1e30;
 };
 
+// CTAs of `smem` bytes and `regs` registers per thread that one SM holds.
+int ctas_per_sm(int smem, int regs) {
+  int per_sm = std::min({233472 / (smem + 1024), TMEM_CTAS, 2048 / kThreads});
+  if (regs > 0) per_sm = std::min(per_sm, 65536 / (((regs + 7) / 8) * 8 * kThreads));
+  return per_sm;
+}
+
 // Cluster split of K for a kernel instance with `regs` registers per thread:
-// waves of resident CTAs cost a fixed latency plus the per-CTA issue time of
-// their k-tiles and, fused (units_cap > 0), the cluster-wide maxima and the
-// encoding of the CTA's activation slice (every unit of which must fit in
-// units_cap registers arrays per thread).  The smaller split wins ties.
+// waves of resident CTAs cost a fixed latency plus the per-CTA time of their
+// k-tiles and, fused (units_cap > 0), the cluster-wide maxima and the encoding
+// of the CTA's activation slice (every unit of which must fit in units_cap
+// register arrays per thread).  The smaller split wins ties.  The W ring then
+// takes as many stages (up to the CTA's k-tiles) as keep the same number of
+// CTAs per SM: measured, a deeper ring gains a little where it costs no
+// residency and loses a whole wave where it does.
 Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, int M, int K, int units_cap) {
   const bool res = ro != 0;
   Choice best;
   for (int ks = 1; ks <= std::min(MAX_KS, k_tiles); ++ks) {
     const int kt_max = (k_tiles + ks - 1) / ks;
-    const int smem = smem_bytes(kt_max, ro, M);
+    const int smem = std::max(smem_bytes(2, kt_max, ro, M), kSmemFloor);
     if (smem > 232448) continue;
     const int slice = std::min(kt_max * 256, K);
     const int64_t units = (int64_t)M * (slice / 8);
     if (units_cap > 0 && units > (int64_t)units_cap * kThreads) continue;
-    int per_sm = std::min({233472 / (smem + 1024), TMEM_CTAS, 2048 / kThreads});
-    if (regs > 0) per_sm = std::min(per_sm, 65536 / (((regs + 7) / 8) * 8 * kThreads));
+    const int per_sm = ctas_per_sm(smem, regs);
     if (per_sm < 1) continue;
     const int64_t ctas = (int64_t)row_tiles * ks, slots = (int64_t)per_sm * num_sms;
     const int64_t waves = (ctas + slots - 1) / slots;
@@ -603,8 +633,15 @@ Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, i
       wave += kExchangeUs * (res ? 2.0 : 1.0) + kUnitUs * co_resident * upt;
     }
     const double cost = (double)waves * wave;
-    if (cost < best.cost - 1e-9) best = Choice{ks, kt_max, smem, cost};
+    if (cost < best.cost - 1e-9) best = Choice{ks, kt_max, 2, smem, cost};
   }
+  if (best.ks > 0)
+    for (int st = 3; st <= std::min(MAX_STAGES, best.kt_max); ++st) {
+      const int smem = std::max(smem_bytes(st, best.kt_max, ro, M), kSmemFloor);
+      if (smem > 232448 || ctas_per_sm(smem, regs) < ctas_per_sm(best.smem, regs)) break;
+      best.stages = st;
+      best.smem = smem;
+    }
   return best;
 }
 
@@ -625,6 +662,7 @@ cudaError_t launch_cfg(const DecodeArgs& a, DecodeParams p, const Choice& c, con
   auto kern = k_decode_tc<T, FUSED, RES, BF16OUT, R>;
   const int row_tiles = (int)((a.N + 127) / 128);
   p.kt_max = c.kt_max;
+  p.stages = c.stages;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem);
   if (e != cudaSuccess) return e;
   if (c.ks > 8) {
@@ -737,6 +775,9 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
   p.katoms_w = (int)(a.K / 64);
   p.k_tiles = (int)((a.K + 255) / 256);
   p.st = a.st;
+  const WaitTest wt = wait_test();
+  p.wait_ns = wt.limit_ns;
+  p.hold = wt.hold;
   if (fused)
     return a.x_bf16 ? launch_t<__nv_bfloat16, true>(a, p, tmW, tmX, tmR, num_sms, stream)
                     : launch_t<float, true>(a, p, tmW, tmX, tmR, num_sms, stream);

@@ -68,7 +68,7 @@ constexpr int SF_REGS = 80, CTL_REGS = 56, EPI_REGS = 184;
 static_assert(128 * SF_REGS + 128 * CTL_REGS + 256 * EPI_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment for 128B swizzle");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert((4 * STAGES + 2) * 8 + 8 <= BAR_BYTES, "barrier block");
+static_assert((4 * STAGES + 3) * 8 + 16 + 8 <= BAR_BYTES, "barrier block");
 static_assert(SF_COL % 4 == 0 && SF_BUF % 4 == 0 && SF_COL + STAGES * SF_BUF <= TMEM_COLS,
               "block-scaled MMA scale operands start on 4-column TMEM boundaries");
 
@@ -87,6 +87,8 @@ struct TcParams {
   int b_groups;    // 128-row groups of W = ceil(N / 128)
   int m_blocks, n_blocks, num_tiles, k_tiles;
   int* st;
+  uint64_t wait_ns;   // bound on every mbarrier wait
+  int hold;           // test of the timeout path: the producer loads nothing
 };
 
 // --------------------------------------------------------------- kernel
@@ -117,8 +119,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* sf_full = bars + 3 * STAGES;   // [STAGES] scales in TMEM, all four quadrants -> MMA
   uint64_t* acc_full = bars + 4 * STAGES;
   uint64_t* acc_empty = acc_full + 1;  // the epilogue holds the accumulator in registers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* mma_drain = acc_empty + 1; // every MMA issued has completed (before TMEM is released)
+  WaitState* abort_flag = reinterpret_cast<WaitState*>(mma_drain + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(abort_flag + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -130,7 +133,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(saddr(acc_full), 1);
     mbar_init(saddr(acc_empty), EPI_WARPS);
-    *abort_flag = 0;
+    mbar_init(saddr(mma_drain), 1);
+    abort_flag->abort = 0;
+    abort_flag->limit_ns = p.wait_ns;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 5) {
@@ -206,6 +211,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // the small scale atoms first, on their own barrier: their trip to TMEM
       // overlaps the code tiles' flight
       int g = 0;
+      if (p.hold) goto producer_done;
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
         const int mb = tile % p.m_blocks, nb = tile / p.m_blocks;
         const int ngroups = min(2, p.b_groups - nb * 2);
@@ -231,7 +237,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_2d(saddr(st_base + OFF_B), &tmB, kt * BK_BYTES, nb * BN, bar);
         }
       }
-    producer_done:;
+    producer_done:
+      // the last STAGES stages' copies may still be in flight if a consumer gave
+      // up: let them land before the CTA can exit
+      for (int g2 = max(0, g - STAGES); g2 < g; ++g2) {
+        const uint32_t ph = (uint32_t)((g2 / STAGES) & 1);
+        (void)mbar_drain(saddr(&sf_land[g2 % STAGES]), ph, abort_flag, p.st);
+        (void)mbar_drain(saddr(&full[g2 % STAGES]), ph, abort_flag, p.st);
+      }
     } else if (warp == 5 && lane == 0) {
       // -------------------------------------------------------- MMA issuer
       const uint32_t idesc = idesc_nvf4(BN);
@@ -268,7 +281,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (NUSE == 2 || pass == NPASS - 1) tc_commit(saddr(acc_full));
       }
-    mma_done:;
+    mma_done:
+      // every MMA issued has completed before TMEM can be released
+      tc_commit(saddr(mma_drain));
+      (void)mbar_drain(saddr(mma_drain), 0u, abort_flag, p.st);
     }
   } else {
     regs_inc<EPI_REGS>();
@@ -430,6 +446,9 @@ cudaError_t launch_gemm_impl(const GemmArgs& g, int num_sms, cudaStream_t stream
   p.num_tiles = p.m_blocks * p.n_blocks;
   p.k_tiles = (int)((g.K + BK - 1) / BK);
   p.st = g.st;
+  const WaitTest wt = wait_test();
+  p.wait_ns = wt.limit_ns;
+  p.hold = wt.hold;
   auto kern = res ? (g.y_bf16 ? k_gemm_nvf4<true, MX, true> : k_gemm_nvf4<false, MX, true>)
                   : (g.y_bf16 ? k_gemm_nvf4<true, MX> : k_gemm_nvf4<false, MX>);
   // the register split assumes the launch allocates LAUNCH_REGS per thread

@@ -82,7 +82,7 @@ struct Cfg {
   static constexpr int SMEM = SMEM_NEED > SMEM_MIN ? SMEM_NEED : SMEM_MIN;
   static constexpr int CTAS_PER_SM = (233472 / (SMEM + 1024)) < TMEM_CTAS ? (233472 / (SMEM + 1024)) : TMEM_CTAS;
   static_assert(1023 + STAGES * STAGE + PART_DED + BAR <= SMEM, "layout exceeds the shared-memory request");
-  static_assert((2 * STAGES + 3) * 8 + 8 <= BAR, "barrier block");
+  static_assert((2 * STAGES + 3) * 8 + 16 + 8 <= BAR, "barrier block");
   static_assert(SF_COL % 4 == 0 && SF_BUF % 4 == 0, "block-scaled MMA scale operands start on 4-column TMEM boundaries");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(PART_OWN || PART <= STAGES * STAGE, "partials overlay the stage ring");
@@ -102,6 +102,8 @@ struct SwapParams {
   int M, N, K;
   int katoms_w, k_tiles;
   int* st;
+  uint64_t wait_ns;   // bound on every mbarrier wait
+  int hold;           // test of the timeout path: the producer loads nothing
 };
 
 template <int NP, bool RES, bool BF16OUT>
@@ -117,8 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + C::STAGES;
   uint64_t* acc_full = bars + 2 * C::STAGES;
   uint64_t* sf_full = acc_full + 1;   // [2] a scale buffer written by all four quadrants
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  WaitState* abort_flag = reinterpret_cast<WaitState*>(sf_full + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(abort_flag + 1);
 
   griddep_launch_dependents();   // the next kernel may set itself up; it waits for this one's results
 
@@ -136,7 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(saddr(acc_full), 1);
     mbar_init(saddr(&sf_full[0]), 4);
     mbar_init(saddr(&sf_full[1]), 4);
-    *abort_flag = 0;
+    abort_flag->abort = 0;
+    abort_flag->limit_ns = p.wait_ns;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -165,9 +168,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------- TMA producer
-    int s = 0;
+    int s = 0, issued = 0;
     uint32_t ph = 0;
-    for (int kt = kt0; kt < kt1; ++kt) {
+    for (int kt = kt0; !p.hold && kt < kt1; ++kt, ++issued) {
       if (!mbar_wait(saddr(&empty[s]), ph ^ 1u, abort_flag, p.st)) break;
       const int jmax = min(4, (p.K - kt * 256) / 64);
       const uint32_t sf = (uint32_t)jmax * 512u;
@@ -182,6 +185,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (RES) bulk_load(saddr(sb + C::OFF_SFR), p.sfr + (size_t)kt * 4 * 512, sf, bar);
       if (++s == C::STAGES) { s = 0; ph ^= 1u; }
     }
+    // the last STAGES stages' copies may still be in flight if a consumer gave
+    // up: let them land before the CTA can exit
+    for (int g2 = max(0, issued - C::STAGES); g2 < issued; ++g2)
+      (void)mbar_drain(saddr(&full[g2 % C::STAGES]), (uint32_t)((g2 / C::STAGES) & 1), abort_flag, p.st);
   } else if (warp >= 4) {
     // ------------------------------------------- scales into TMEM (tcgen05.st)
     // Warp w writes TMEM lane quadrant w - 4 of scale buffer g & 1 for the
@@ -261,7 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Owner o = floor(r*ks/128) holds rows [ceil(o*128/ks), ceil((o+1)*128/ks))
   // of the tile, at most ceil(128/ks) rows, and keeps one slot of that many
   // rows per source rank.
-  const bool ok = mbar_wait(saddr(acc_full), 0u, abort_flag, p.st);
+  // the commit after the MMA loop is issued on every path: waiting for it also
+  // waits for every MMA in flight, before TMEM is read and released
+  const bool ok = mbar_drain(saddr(acc_full), 0u, abort_flag, p.st) && !wait_aborted(abort_flag);
   tc_fence_after();
   __syncwarp();     // the cluster barriers below are warp-aligned
   if (!C::PART_OWN) {
@@ -353,6 +362,9 @@ cudaError_t launch_np(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   p.katoms_w = (int)((g.K + 63) / 64);
   p.k_tiles = (int)((g.K + 255) / 256);
   p.st = g.st;
+  const WaitTest wt = wait_test();
+  p.wait_ns = wt.limit_ns;
+  p.hold = wt.hold;
   const int row_tiles = (int)((g.N + 127) / 128);
   // the largest K split whose CTAs are all resident at once (one wave)
   const int fit = std::max(1, (C::CTAS_PER_SM * num_sms) / row_tiles);

@@ -54,6 +54,26 @@ cudaError_t launch_reorder_quant(const void* x, nvfp4_dtype dt, int64_t M, int64
                                  int64_t S, const float* s_ptr, const QOut& q, int* st, int num_sms,
                                  cudaStream_t stream, bool after_stats);
 
+// Offline weight preparation: W_aug = [W' | W'[:, :S]], W'[:, j] = fl32(W[:, perm[j]] *
+// sigma[perm[j]]) (sigma / perm may be null), quantized under s_in or its own
+// computed tensor scale (written to q.s).
+cudaError_t launch_weight_quant(const void* w, nvfp4_dtype dt, int64_t N, int64_t K, int64_t ldw,
+                                const float* sigma, const int32_t* perm, int64_t S, const float* s_in,
+                                const QOut& q, WsHeader* ws, int* st, int num_sms, cudaStream_t stream);
+
+// Bounded-wait settings that the next tensor-core launches carry (process wide,
+// host side): limit_ns bounds every device-side wait; hold != 0 makes the load
+// issuers skip their operand loads, so that the waits run out and the launch
+// reports NVFP4_ERR_TIMEOUT (a test of the timeout path, set through
+// nvfp4_test_wait_fault).
+struct WaitTest {
+  uint64_t limit_ns;
+  int hold;
+};
+WaitTest wait_test();
+// The default bound on a device-side wait (4 s).
+constexpr uint64_t tc_wait_default_ns() { return 4000000000ull; }
+
 // Operands of the decode GEMV / tensor-core GEMM.
 struct GemmArgs {
   const uint8_t* a_codes; const uint8_t* a_scales; const float* a_s;   // M x K

@@ -595,38 +595,85 @@ __device__ __forceinline__ void lds8(const float* p, float v[8]) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Bytes of dynamic shared memory of k_reorder_onepass for `rows` rows per CTA.
+// Bytes of dynamic shared memory of k_reorder_onepass for `rows` rows per CTA:
+// the rows, the permutation (16-bit), gamma in source and in permuted order,
+// one rinv per row, and the 256-entry d and 1/(d s) tables of the block encoder.
 inline size_t onepass_smem_bytes(size_t es, int64_t K, bool has_gamma, int rows) {
   return (size_t)rows * (size_t)K * es + (((size_t)K * 2 + 15) & ~size_t(15)) +
-         (has_gamma ? (size_t)K * es : 0) + (size_t)rows * 4;
+         (has_gamma ? 2 * (size_t)K * es : 0) + (((size_t)rows * 4 + 15) & ~size_t(15)) + 2 * 256 * 4;
+}
+
+// 8 consecutive elements from global memory (16/32-byte aligned) as fp32.
+__device__ __forceinline__ void ldg8(const __nv_bfloat16* p, float v[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+  v[4] = __uint_as_float(u.z << 16); v[5] = __uint_as_float(u.z & 0xFFFF0000u);
+  v[6] = __uint_as_float(u.w << 16); v[7] = __uint_as_float(u.w & 0xFFFF0000u);
+}
+__device__ __forceinline__ void ldg8(const float* p, float v[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Gather reordered block b of a row held in shared memory: v[e] =
+// y'[16 b + e] = fl32(fl32(x[perm[16 b + e]] * ri) * gp[16 b + e]) (gp: gamma in
+// permuted order; no gamma: x[perm[.]]).  Returns the |.| maximum key.
+template <typename T>
+__device__ __forceinline__ uint32_t gather_block(const T* srow, const uint16_t* sperm, const T* sgp, float ri,
+                                                 int b, float v[16]) {
+  uint16_t pv[16];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)   // 16-byte reads of the cached permutation
+    *reinterpret_cast<uint4*>(pv + 8 * j) = reinterpret_cast<const uint4*>(sperm)[b * 2 + j];
+  float g[16];
+  if (sgp != nullptr) {
+    lds8(sgp + b * 16, g);
+    lds8(sgp + b * 16 + 8, g + 8);
+  }
+  uint32_t key = 0u;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float y = load1(srow + pv[i]);
+    if (sgp != nullptr) y = __fmul_rn(__fmul_rn(y, ri), g[i]);
+    v[i] = y;
+    key = max(key, abs_key(y));
+  }
+  return key;
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256) k_reorder_onepass(const T* __restrict__ x, int64_t M, int64_t K,
+__global__ void __launch_bounds__(256, 3) k_reorder_onepass(const T* __restrict__ x, int64_t M, int64_t K,
                                                          int64_t ldx, const T* __restrict__ gamma, float eps,
                                                          const int32_t* __restrict__ perm, int64_t S,
                                                          const float* s_in, QOut q, WsHeader* ws,
                                                          int rows_per_cta, int* st) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ uint32_t redu[32];
-  __shared__ double redd[32];
+  __shared__ uint32_t wkey[8];   // per warp: the |y| maximum of its rows
+  __shared__ uint32_t wbad[8];   // per warp: the |x| maximum (Inf/NaN detection)
   __shared__ float s_sh;
   __shared__ int ok_sh;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row_bytes = K * (int64_t)sizeof(T);   // a multiple of 16 (K % 16 == 0)
   const int64_t rows_bytes = (int64_t)rows_per_cta * row_bytes;
+  const int64_t perm_bytes = (K * 2 + 15) & ~int64_t(15);
   T* srows = reinterpret_cast<T*>(smem);
   uint16_t* sperm = reinterpret_cast<uint16_t*>(smem + rows_bytes);
-  const int64_t perm_bytes = (K * 2 + 15) & ~int64_t(15);
-  T* sgamma = reinterpret_cast<T*>(smem + rows_bytes + perm_bytes);
-  float* srinv = reinterpret_cast<float*>(smem + rows_bytes + perm_bytes + (gamma ? row_bytes : 0));
+  T* sgp = reinterpret_cast<T*>(smem + rows_bytes + perm_bytes);
+  T* sg = sgp + (gamma ? K : 0);   // gamma in source order
+  float* srinv = reinterpret_cast<float*>(smem + rows_bytes + perm_bytes + (gamma ? 2 * row_bytes : 0));
+  float* d_tab = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(srinv) +
+                                          (((int64_t)rows_per_cta * 4 + 15) & ~int64_t(15)));
+  float* inv_tab = d_tab + 256;
   const int64_t G = gridDim.x;
-  int nrows = 0;   // rows of this CTA
+  int nrows = 0;   // rows of this CTA: blockIdx.x + i * G
   while (nrows < rows_per_cta && (int64_t)blockIdx.x + nrows * G < M) ++nrows;
 
-  // 1. every load in flight at once
+  // 1. every row load (and gamma) in flight at once; the permutation meanwhile
   if (gamma)
     for (int64_t c = threadIdx.x; c < row_bytes / 16; c += blockDim.x)
-      cp_async16(reinterpret_cast<uint4*>(sgamma) + c, reinterpret_cast<const uint4*>(gamma) + c);
+      cp_async16(reinterpret_cast<uint4*>(sg) + c, reinterpret_cast<const uint4*>(gamma) + c);
   for (int i = 0; i < nrows; ++i) {
     const T* xr = x + ((int64_t)blockIdx.x + i * G) * ldx;
     T* dst = srows + (int64_t)i * K;
@@ -636,99 +683,163 @@ __global__ void __launch_bounds__(256) k_reorder_onepass(const T* __restrict__ x
   cp_async_commit();
   if (load_perm16(perm, K, sperm)) report_status(st, NVFP4_ERR_INVALID_ARG);
   cp_async_wait_all();
-  __syncthreads();
+  __syncthreads();   // rows, gamma and the permutation are in place
+  if (gamma)         // gamma in the permuted order, for 16-byte reads in the encoder
+    for (int64_t j = threadIdx.x; j < K; j += blockDim.x) sgp[j] = sg[sperm[j]];
 
-  // 2. row factors and this CTA's part of the tensor maximum
+  // 2. per row, one warp: the |x| maximum (exponent), the exact mean square
+  // (k_rms_stats' arithmetic), rinv and the |y| maximum; no block barrier
   const int64_t upr = K >> 3;
-  uint32_t ykey = 0, bad = 0;
-  for (int i = 0; i < nrows; ++i) {
+  uint32_t ykey = 0u, bad = 0u;
+  for (int i = warp; i < nrows; i += 8) {
     const T* sr = srows + (int64_t)i * K;
-    uint32_t key = 0;
-    for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+    uint32_t key = 0u;
+    for (int64_t c8 = lane; c8 < upr; c8 += 32) {
       float v[8];
       lds8(sr + c8 * 8, v);
 #pragma unroll
       for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
     }
-    key = block_max_u32(key, redu);
+    key = warp_max_u32(key);
     bad = max(bad, key);
     if (gamma == nullptr) {
       ykey = max(ykey, key);
       continue;
     }
-    double qsum = 0.0;
+    double qs[4] = {0.0, 0.0, 0.0, 0.0};   // independent partial sums: no serial add chain
     int e = 0;
     if (key != 0u && key < 0x7F800000u) {
       e = ilog2_key(key);
       const double c = pow2_f64(17 - e);  // z = x * 2^(17-e), |z| < 2^18
-      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+      for (int64_t c8 = lane; c8 < upr; c8 += 32) {
         float v[8];
         lds8(sr + c8 * 8, v);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const double z = __dmul_rn((double)v[j], c);
-          qsum = __dadd_rn(qsum, floor(__dmul_rn(z, z)));
+          qs[j & 3] = __dadd_rn(qs[j & 3], floor(__dmul_rn(z, z)));
         }
       }
     }
-    qsum = block_sum_f64(qsum, redd);  // exact: integers with total < 2^53
+    // exact: integers with total < 2^53, so the order of the additions is free
+    double qsum = warp_sum_f64(__dadd_rn(__dadd_rn(qs[0], qs[1]), __dadd_rn(qs[2], qs[3])));
     const double mean = __ddiv_rn(__dmul_rn(qsum, pow2_f64(2 * e - 34)), (double)K);
     const float ri = __double2float_rn(__drcp_rn(__dsqrt_rn(__dadd_rn(mean, (double)eps))));
-    if (threadIdx.x == 0) srinv[i] = ri;
+    if (lane == 0) srinv[i] = ri;
     if (s_in == nullptr) {
-      for (int64_t c8 = threadIdx.x; c8 < upr; c8 += blockDim.x) {
+      for (int64_t c8 = lane; c8 < upr; c8 += 32) {
         float v[8], g[8];
         lds8(sr + c8 * 8, v);
-        lds8(sgamma + c8 * 8, g);
+        lds8(sg + c8 * 8, g);
 #pragma unroll
         for (int j = 0; j < 8; ++j) ykey = max(ykey, abs_key(__fmul_rn(__fmul_rn(v[j], ri), g[j])));
       }
     }
   }
+  ykey = warp_max_u32(ykey);
+  if (lane == 0) {
+    wkey[warp] = ykey;
+    wbad[warp] = bad;
+  }
+  __syncthreads();   // per-warp maxima, srinv and sgp are visible to every thread
 
-  // 3. the tensor scale
-  if (s_in == nullptr) {
-    const uint32_t m = block_max_u32(ykey, redu);
-    if (threadIdx.x == 0) {
+  // 3. the tensor scale: one exchange of the CTA maxima through the workspace
+  if (threadIdx.x == 0) {
+    uint32_t m = 0u, xb = 0u;
+    for (int w = 0; w < 8; ++w) {
+      m = max(m, wkey[w]);
+      xb = max(xb, wbad[w]);
+    }
+    if (xb >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
+    if (s_in == nullptr) {
       if (m != 0u) atomicMax(&ws->amax_bits[0], m);
       __threadfence();
       atomicAdd(&ws->arrive[0], 1u);
       const uint64_t t0 = tc::globaltimer();
       int ok = 1;
       while (ld_acquire_gpu(&ws->arrive[0]) < (uint32_t)G) {
+        __nanosleep(64);   // fewer polls of the shared counter while the others arrive
         if (tc::globaltimer() - t0 > tc::kTimeoutNs) {
           ok = 0;
           report_status(st, NVFP4_ERR_TIMEOUT);
           break;
         }
       }
-      const uint32_t a = atomicAdd(&ws->amax_bits[0], 0u);
+      // every CTA's maximum was added before its arrival was counted
+      const uint32_t a = ld_acquire_gpu(&ws->amax_bits[0]);
       s_sh = ok ? scale_from_key(a, blockIdx.x == 0, st) : 0.0f;
       ok_sh = ok;
-      // the last CTA to leave zeroes the header for the next call
-      __threadfence();
-      if (atomicAdd(&ws->arrive[1], 1u) == (uint32_t)G - 1u) {
-        ws->amax_bits[0] = 0u;
-        ws->arrive[0] = 0u;
-        ws->arrive[1] = 0u;
-        __threadfence();
-      }
+    } else {
+      s_sh = *s_in;
+      ok_sh = 1;
     }
-  } else if (threadIdx.x == 0) {
-    s_sh = *s_in;
-    ok_sh = 1;
   }
-  __syncthreads();   // s_sh, ok_sh and srinv are visible to every thread
+  __syncthreads();
+  if (s_in == nullptr && threadIdx.x == 32) {
+    // leave after this CTA's read above; the last CTA to leave zeroes the
+    // header for the next call (off the other threads' path)
+    __threadfence();
+    if (atomicAdd(&ws->arrive[1], 1u) == (uint32_t)G - 1u) {
+      ws->amax_bits[0] = 0u;
+      ws->arrive[0] = 0u;
+      ws->arrive[1] = 0u;
+      __threadfence();
+    }
+  }
   if (!ok_sh) return;
   const float s = s_sh;
   if (blockIdx.x == 0 && threadIdx.x == 0 && q.s != s_in) *q.s = s;
+  make_scale_tables(s, d_tab, inv_tab);
+  __syncthreads();
 
-  // 4. encode
+  // 4. encode: the CTA's main blocks, then its residue blocks, as one flat list
+  // over all threads (a residue block recomputes its main block's dequantized
+  // values), so that the S residue blocks of a row are not left to a few threads
   const int nb = (int)(K >> 4), nbr = (int)(S >> 4);
-  for (int i = 0; i < nrows; ++i)
-    encode_reordered_row(srows + (int64_t)i * K, sperm, gamma ? sgamma : nullptr, gamma ? srinv[i] : 1.0f, s, q,
-                         (int64_t)blockIdx.x + i * G, nb, nbr, bad);
-  if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
+  const int n_main = nrows * nb, n_all = n_main + nrows * nbr;
+  const T* gp = gamma ? sgp : nullptr;
+  auto task_of = [&](int t, int& i, int& b) {
+    const bool res = t >= n_main;
+    const int u = res ? t - n_main : t;
+    const int per = res ? nbr : nb;
+    i = u / per;
+    b = u - i * per;
+    return res;
+  };
+  auto finish = [&](bool res, int i, int b, const float* v, uint32_t key) {
+    const int64_t row = (int64_t)blockIdx.x + (int64_t)i * G;
+    uint32_t db;
+    float deq[16];
+    const uint64_t codes = quant_block16_tab(v, key, s, d_tab, inv_tab, db, res ? deq : nullptr);
+    if (!res) {
+      store_block16(q, row, b, codes, db);
+    } else {
+      float rv[16];
+      uint32_t rkey = 0u;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        rv[j] = __fsub_rn(v[j], deq[j]);
+        rkey = max(rkey, abs_key(rv[j]));
+      }
+      uint32_t dr;
+      const uint64_t rc = quant_block16_tab(rv, rkey, s, d_tab, inv_tab, dr, nullptr);
+      store_block16(q, row, nb + b, rc, dr);
+    }
+  };
+  // two tasks per iteration: both gathers are issued before either is encoded
+  for (int t = threadIdx.x; t < n_all; t += 2 * blockDim.x) {
+    const int t2 = t + blockDim.x;
+    int i0, b0, i1 = 0, b1 = 0;
+    const bool r0 = task_of(t, i0, b0);
+    const bool has2 = t2 < n_all;
+    const bool r1 = has2 ? task_of(t2, i1, b1) : false;
+    float v0[16], v1[16];
+    const uint32_t k0 = gather_block(srows + (int64_t)i0 * K, sperm, gp, gamma ? srinv[i0] : 1.0f, b0, v0);
+    uint32_t k1 = 0u;
+    if (has2) k1 = gather_block(srows + (int64_t)i1 * K, sperm, gp, gamma ? srinv[i1] : 1.0f, b1, v1);
+    finish(r0, i0, b0, v0, k0);
+    if (has2) finish(r1, i1, b1, v1, k1);
+  }
 }
 
 // ------------------------------------------------------------ launchers

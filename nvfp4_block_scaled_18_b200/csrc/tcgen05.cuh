@@ -7,11 +7,25 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "kernels.h"
 
 namespace nvfp4 {
 namespace tc {
 
-constexpr uint64_t kTimeoutNs = 4000000000ull;   // bound on every mbarrier wait
+constexpr uint64_t kTimeoutNs = tc_wait_default_ns();   // default bound on every mbarrier wait
+
+// A CTA's bounded-wait state, in shared memory: the flag a role raises when it
+// gives up (the other roles then leave their loops at their next wait) and the
+// wait limit of this launch in nanoseconds.
+struct WaitState {
+  int abort;
+  int pad;
+  uint64_t limit_ns;
+};
+__device__ __forceinline__ bool wait_aborted(const WaitState* w) {
+  return *reinterpret_cast<const volatile int*>(&w->abort) != 0;
+}
+__device__ __forceinline__ void wait_raise(WaitState* w) { *reinterpret_cast<volatile int*>(&w->abort) = 1; }
 
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
@@ -69,15 +83,15 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 // Bounded wait: false when this or another role gave up.
 template <bool CLUSTER = false>
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* st) {
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, WaitState* w, int* st) {
   auto poll = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (poll()) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (poll()) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
-      *abort_flag = 1;
+    if (wait_aborted(w)) return false;
+    if (globaltimer() - t0 > w->limit_ns) {
+      wait_raise(w);
       report_status(st, NVFP4_ERR_TIMEOUT);
       return false;
     }
@@ -87,15 +101,33 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
 // warpgroups (setmaxnreg) cannot call a function compiled for one budget.
 // CLUSTER: acquire at cluster scope (arrivals from other CTAs of the cluster).
 template <bool CLUSTER = false>
-__device__ __forceinline__ bool mbar_wait_inline(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* st) {
+__device__ __forceinline__ bool mbar_wait_inline(uint32_t bar, uint32_t parity, WaitState* w, int* st) {
   auto poll = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (poll()) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (poll()) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
-      *abort_flag = 1;
+    if (wait_aborted(w)) return false;
+    if (globaltimer() - t0 > w->limit_ns) {
+      wait_raise(w);
+      report_status(st, NVFP4_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+// Drain: wait for work that completes by itself -- this CTA's own bulk copies
+// and MMAs in flight, or bytes that the peers of a cluster send on every path --
+// whether or not a role has given up, so that nothing lands in this CTA's
+// shared memory or tensor memory after it exits.  Still bounded by the limit.
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, WaitState* w, int* st) {
+  auto poll = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (poll()) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (poll()) return true;
+    if (globaltimer() - t0 > w->limit_ns) {
+      wait_raise(w);
       report_status(st, NVFP4_ERR_TIMEOUT);
       return false;
     }

@@ -288,10 +288,14 @@ def rmsnorm_reorder_quantize(x, gamma=None, eps: float = 1e-5, perm=None, S: int
     return QTensor(codes, scales, s)
 
 
-def augment_weight(w_fp32, perm, S: int):
-    """W_aug = [W[:, perm] | W[:, perm[:S]]] in fp32 ([ARC] s3.1 and s6.3: the
-    weight uses the same channel order as the activation)."""
+def augment_weight(w_fp32, perm, S: int, sigma=None):
+    """W_aug = [W' | W'[:, :S]] with W' = W[:, perm] in fp32 ([ARC] s3.1 and s6.3:
+    the weight uses the same channel order as the activation).  sigma: a
+    per-channel smoothing vector absorbed as W diag(sigma) (OSFP4 page, abstract),
+    W'[:, j] = fl32(W[:, perm[j]] * sigma[perm[j]])."""
     w = _f32(w_fp32)
+    if sigma is not None:
+        w = (w * _f32(sigma)[None, :]).astype(np.float32)   # one IEEE binary32 product per element
     wp = w[:, np.asarray(perm, dtype=np.int64)]
     return np.ascontiguousarray(np.concatenate([wp, wp[:, :S]], axis=1))
 
