@@ -25,7 +25,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC,
           "--expt-relaxed-constexpr"]
 # Files whose arithmetic must round exactly as written (no contraction).
-NO_FMAD = {"quantize.cu", "decode_tc.cu"}
+NO_FMAD = {"quantize.cu", "decode_tc.cu", "weight.cu"}
 
 
 def nvcc() -> str:

@@ -483,7 +483,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_mma_nvf4(tmem + ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + sfw + 4 * j,
                     tmem + sfx + 4 * j, acc);
       }
-      tc_commit(saddr(&empty[s]));
+      // Someone waits for this k-tile's MMAs only if its stage is refilled
+      // (t + NS < nkt) or its scale buffer is reused (t + 2 < nkt); with
+      // NS >= 2 both come down to t + 2 < nkt.  A commit costs tensor-pipe
+      // time, so the last two k-tiles go without one (acc_full covers them).
+      if (t + 2 < nkt) tc_commit(saddr(&empty[s]));
     }
     tc_commit(saddr(acc_full));
   }

@@ -257,7 +257,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_mma_nvf4(tmem + C::ACC_R, dw + (uint64_t)(2 * j), dr + (uint64_t)(2 * j), idesc, tmem + buf + 4 * j,
                       tmem + buf + 32 + 4 * j, acc);
       }
-      tc_commit(saddr(&empty[s]));
+      // waited for only when the stage is refilled (g + STAGES < nkt) or the
+      // scale buffer reused (g + 2 < nkt): both are g + 2 < nkt with STAGES >= 2,
+      // and a commit costs tensor-pipe time (acc_full covers the last two)
+      if (kt + 2 < kt1) tc_commit(saddr(&empty[s]));
       if (++s == C::STAGES) { s = 0; ph ^= 1u; }
     }
     tc_commit(saddr(acc_full));
@@ -366,25 +369,43 @@ cudaError_t launch_np(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   p.wait_ns = wt.limit_ns;
   p.hold = wt.hold;
   const int row_tiles = (int)((g.N + 127) / 128);
-  // the largest K split whose CTAs are all resident at once (one wave)
-  const int fit = std::max(1, (C::CTAS_PER_SM * num_sms) / row_tiles);
-  const int ks = std::max(1, std::min({8, p.k_tiles, fit}));
   auto kern = k_gemv_tc<NP, RES, BF16OUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)ks, (unsigned)row_tiles, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the preceding kernel's tail
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // The largest K split whose clusters are all resident at once (one wave).  A
+  // cluster must fit inside one GPC, so the count of resident clusters comes from
+  // the occupancy query, not from CTAs per SM x SMs; it is cached per split.
+  static int resident[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  int ks = 1;
+  for (int c = std::min(8, p.k_tiles); c > 1; --c) {
+    if (c * row_tiles > C::CTAS_PER_SM * num_sms) continue;
+    if (resident[c] == 0) {
+      attr[0].val.clusterDim.x = (unsigned)c;
+      cfg.gridDim = dim3((unsigned)c, 1, 1);
+      int n = 0;
+      e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      if (e != cudaSuccess) return e;
+      resident[c] = std::max(n, 1);
+    }
+    if (resident[c] >= row_tiles) {
+      ks = c;
+      break;
+    }
+  }
+  attr[0].val.clusterDim.x = (unsigned)ks;
+  cfg.gridDim = dim3((unsigned)ks, (unsigned)row_tiles, 1);
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, tmW, tmX, tmR, p);
 }

@@ -562,19 +562,21 @@ __global__ void __launch_bounds__(256) k_reorder_quant(const T* __restrict__ x, 
   if (bad >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
 }
 
-// One-launch ARCQuant quantizer, for inputs that fit in the shared memory of
-// one wave of CTAs.  The launch is cooperative, so every CTA is resident.
-// Each CTA:
-//   1. loads its rows (rows blockIdx.x + i * gridDim.x) once, with gamma and
-//      the permutation;
-//   2. derives each row's factor rinv and its part of the tensor maximum with
-//      the arithmetic of k_rms_stats (or the |x| maximum of k_amax without
-//      gamma);
-//   3. meets the other CTAs at one exchange of that maximum through the
+// One-launch ARCQuant quantizer, for inputs whose rows fit in the shared
+// memory of one wave of CTAs: one row per warp (or a few).  The launch is
+// cooperative, so every CTA is resident.  Each warp:
+//   1. loads its row with 16-byte loads, all in flight at once, keeps it in
+//      registers and copies it to its row buffer in shared memory, and takes
+//      from the registers the row's |x| maximum, its exact mean square (the
+//      arithmetic of k_rms_stats), rinv and the row's |y| maximum (without
+//      gamma: the |x| maximum);
+//   2. the CTA meets the other CTAs at one exchange of the maximum through the
 //      workspace header (atomics, a bounded wait; the last CTA to leave zeroes
 //      the header again);
-//   4. encodes its rows from shared memory as k_reorder_quant does.
-// So X is read from DRAM once and the result is identical to the two passes.
+//   3. the warp encodes its own row from its row buffer, lanes over the
+//      reordered 16-blocks (residue blocks included).
+// X is read from DRAM once, no block barrier sits inside a row's work, and
+// the result is identical to the two passes.
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned int* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -595,12 +597,14 @@ __device__ __forceinline__ void lds8(const float* p, float v[8]) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Bytes of dynamic shared memory of k_reorder_onepass for `rows` rows per CTA:
-// the rows, the permutation (16-bit), gamma in source and in permuted order,
-// one rinv per row, and the 256-entry d and 1/(d s) tables of the block encoder.
-inline size_t onepass_smem_bytes(size_t es, int64_t K, bool has_gamma, int rows) {
-  return (size_t)rows * (size_t)K * es + (((size_t)K * 2 + 15) & ~size_t(15)) +
-         (has_gamma ? 2 * (size_t)K * es : 0) + (((size_t)rows * 4 + 15) & ~size_t(15)) + 2 * 256 * 4;
+// Shared-memory layout of k_reorder_onepass: the permutation (16-bit), gamma
+// in source and in permuted order, the d and 1/(d s) tables of the block
+// encoder, then rpw row buffers for each of the 8 warps.
+__host__ __device__ inline size_t onepass_fixed_bytes(size_t es, int64_t K, bool has_gamma) {
+  return (((size_t)K * 2 + 15) & ~size_t(15)) + (has_gamma ? 2 * (size_t)K * es : 0) + 2 * 256 * 4;
+}
+inline size_t onepass_smem_bytes(size_t es, int64_t K, bool has_gamma, int rpw) {
+  return onepass_fixed_bytes(es, K, has_gamma) + (size_t)8 * rpw * (size_t)K * es;
 }
 
 // 8 consecutive elements from global memory (16/32-byte aligned) as fp32.
@@ -643,62 +647,81 @@ __device__ __forceinline__ uint32_t gather_block(const T* srow, const uint16_t* 
   return key;
 }
 
+// floor(z^2), z = x 2^(17-e), for a value x of 8 significant bits (bf16) as an
+// exact fp32 computation: for |z| >= 1, z and z^2 (16 bits) are exact in fp32;
+// for |z| < 1 the floor is 0 whatever z rounded to.  (c = 2^(17-e) in fp32,
+// valid for e >= -110; the caller takes the binary64 form below that.)
+__device__ __forceinline__ uint64_t sq_floor_bf16(float x, float c) {
+  const float z = __fmul_rn(x, c);
+  return (uint64_t)floorf(__fmul_rn(z, z));
+}
+
+// Units (8 elements) of a row a lane holds in registers at once.
 template <typename T>
-__global__ void __launch_bounds__(256, 3) k_reorder_onepass(const T* __restrict__ x, int64_t M, int64_t K,
-                                                         int64_t ldx, const T* __restrict__ gamma, float eps,
-                                                         const int32_t* __restrict__ perm, int64_t S,
-                                                         const float* s_in, QOut q, WsHeader* ws,
-                                                         int rows_per_cta, int* st) {
+struct RowChunk {
+  static constexpr int N = sizeof(T) == 2 ? 16 : 8;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256, 2) k_reorder_onepass(const T* __restrict__ x, int64_t M, int64_t K,
+                                                            int64_t ldx, const T* __restrict__ gamma, float eps,
+                                                            const int32_t* __restrict__ perm, int64_t S,
+                                                            const float* s_in, QOut q, WsHeader* ws, int rpw,
+                                                            int* st) {
+  constexpr int NCH = RowChunk<T>::N;   // units per lane loaded at once
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ uint32_t wkey[8];   // per warp: the |y| maximum of its rows
+  __shared__ uint32_t wkey[8];   // per warp: the |y| maximum of its rows (|x| without gamma)
   __shared__ uint32_t wbad[8];   // per warp: the |x| maximum (Inf/NaN detection)
   __shared__ float s_sh;
   __shared__ int ok_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row_bytes = K * (int64_t)sizeof(T);   // a multiple of 16 (K % 16 == 0)
-  const int64_t rows_bytes = (int64_t)rows_per_cta * row_bytes;
-  const int64_t perm_bytes = (K * 2 + 15) & ~int64_t(15);
-  T* srows = reinterpret_cast<T*>(smem);
-  uint16_t* sperm = reinterpret_cast<uint16_t*>(smem + rows_bytes);
-  T* sgp = reinterpret_cast<T*>(smem + rows_bytes + perm_bytes);
-  T* sg = sgp + (gamma ? K : 0);   // gamma in source order
-  float* srinv = reinterpret_cast<float*>(smem + rows_bytes + perm_bytes + (gamma ? 2 * row_bytes : 0));
-  float* d_tab = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(srinv) +
-                                          (((int64_t)rows_per_cta * 4 + 15) & ~int64_t(15)));
+  uint16_t* sperm = reinterpret_cast<uint16_t*>(smem);
+  T* sg = reinterpret_cast<T*>(smem + ((K * 2 + 15) & ~int64_t(15)));   // gamma, source order
+  T* sgp = sg + (gamma ? K : 0);                                         // gamma, permuted order
+  float* d_tab = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(sgp) + (gamma ? row_bytes : 0));
   float* inv_tab = d_tab + 256;
-  const int64_t G = gridDim.x;
-  int nrows = 0;   // rows of this CTA: blockIdx.x + i * G
-  while (nrows < rows_per_cta && (int64_t)blockIdx.x + nrows * G < M) ++nrows;
+  T* wrows = reinterpret_cast<T*>(smem + onepass_fixed_bytes(sizeof(T), K, gamma != nullptr)) +
+             (int64_t)warp * rpw * K;
+  const int64_t W = (int64_t)gridDim.x * 8, wg = (int64_t)blockIdx.x * 8 + warp;   // warps, this warp
+  int nrows = 0;   // rows of this warp: wg + i * W
+  while (nrows < rpw && wg + nrows * W < M) ++nrows;
 
-  // 1. every row load (and gamma) in flight at once; the permutation meanwhile
+  // 0. gamma (source order) and the permutation, shared by the CTA's warps
   if (gamma)
     for (int64_t c = threadIdx.x; c < row_bytes / 16; c += blockDim.x)
       cp_async16(reinterpret_cast<uint4*>(sg) + c, reinterpret_cast<const uint4*>(gamma) + c);
-  for (int i = 0; i < nrows; ++i) {
-    const T* xr = x + ((int64_t)blockIdx.x + i * G) * ldx;
-    T* dst = srows + (int64_t)i * K;
-    for (int64_t c = threadIdx.x; c < row_bytes / 16; c += blockDim.x)
-      cp_async16(reinterpret_cast<uint4*>(dst) + c, reinterpret_cast<const uint4*>(xr) + c);
-  }
   cp_async_commit();
   if (load_perm16(perm, K, sperm)) report_status(st, NVFP4_ERR_INVALID_ARG);
   cp_async_wait_all();
-  __syncthreads();   // rows, gamma and the permutation are in place
-  if (gamma)         // gamma in the permuted order, for 16-byte reads in the encoder
-    for (int64_t j = threadIdx.x; j < K; j += blockDim.x) sgp[j] = sg[sperm[j]];
+  __syncthreads();
 
-  // 2. per row, one warp: the |x| maximum (exponent), the exact mean square
-  // (k_rms_stats' arithmetic), rinv and the |y| maximum; no block barrier
-  const int64_t upr = K >> 3;
+  // 1. per warp, per row: load once (registers and the row buffer), statistics
+  const int64_t upr = K >> 3;                     // 8-element units of a row
+  const int npl = (int)((upr + 31) / 32);         // units per lane
   uint32_t ykey = 0u, bad = 0u;
-  for (int i = warp; i < nrows; i += 8) {
-    const T* sr = srows + (int64_t)i * K;
+  float ri_reg[4] = {1.0f, 1.0f, 1.0f, 1.0f};     // rinv of this warp's rows (rpw <= 4)
+  for (int i = 0; i < nrows; ++i) {
+    const T* xr = x + (wg + i * W) * ldx;
+    T* sr = wrows + (int64_t)i * K;
+    Raw8<T> raw[NCH];
     uint32_t key = 0u;
-    for (int64_t c8 = lane; c8 < upr; c8 += 32) {
-      float v[8];
-      lds8(sr + c8 * 8, v);
+    for (int n0 = 0; n0 < npl; n0 += NCH) {       // load: all of a chunk in flight at once
 #pragma unroll
-      for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
+      for (int n = 0; n < NCH; ++n) {
+        const int64_t c8 = lane + 32 * (int64_t)(n0 + n);
+        if (n0 + n < npl && c8 < upr) raw[n].load(xr + c8 * 8);
+        else raw[n].zero();
+      }
+#pragma unroll
+      for (int n = 0; n < NCH; ++n) {
+        const int64_t c8 = lane + 32 * (int64_t)(n0 + n);
+        if (n0 + n < npl && c8 < upr) raw[n].store_smem(sr + c8 * 8);
+        float v[8];
+        raw[n].get(v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
+      }
     }
     key = warp_max_u32(key);
     bad = max(bad, key);
@@ -706,33 +729,61 @@ __global__ void __launch_bounds__(256, 3) k_reorder_onepass(const T* __restrict_
       ykey = max(ykey, key);
       continue;
     }
-    double qs[4] = {0.0, 0.0, 0.0, 0.0};   // independent partial sums: no serial add chain
+    // the exact sum of floor(z^2), z = x 2^(17-e), from the row buffer, four
+    // independent 16-byte reads at a time
+    uint64_t isum = 0;
     int e = 0;
     if (key != 0u && key < 0x7F800000u) {
       e = ilog2_key(key);
-      const double c = pow2_f64(17 - e);  // z = x * 2^(17-e), |z| < 2^18
-      for (int64_t c8 = lane; c8 < upr; c8 += 32) {
-        float v[8];
-        lds8(sr + c8 * 8, v);
+      const bool fast = sizeof(T) == 2 && e >= -110;
+      const float c32 = fast ? __uint_as_float((uint32_t)(127 + 17 - e) << 23) : 0.0f;
+      const double c64 = pow2_f64(17 - e);
+      for (int n0 = 0; n0 < npl; n0 += 4) {
+        float v[4][8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const double z = __dmul_rn((double)v[j], c);
-          qs[j & 3] = __dadd_rn(qs[j & 3], floor(__dmul_rn(z, z)));
+        for (int n = 0; n < 4; ++n) {
+          const int64_t c8 = lane + 32 * (int64_t)(n0 + n);
+          if (n0 + n < npl && c8 < upr) lds8(sr + c8 * 8, v[n]);
+          else
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[n][j] = 0.0f;
         }
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (fast) {
+              isum += sq_floor_bf16(v[n][j], c32);
+            } else {
+              const double z = __dmul_rn((double)v[n][j], c64);
+              isum += (uint64_t)floor(__dmul_rn(z, z));
+            }
+          }
       }
     }
     // exact: integers with total < 2^53, so the order of the additions is free
-    double qsum = warp_sum_f64(__dadd_rn(__dadd_rn(qs[0], qs[1]), __dadd_rn(qs[2], qs[3])));
+    const double qsum = warp_sum_f64((double)isum);
     const double mean = __ddiv_rn(__dmul_rn(qsum, pow2_f64(2 * e - 34)), (double)K);
     const float ri = __double2float_rn(__drcp_rn(__dsqrt_rn(__dadd_rn(mean, (double)eps))));
-    if (lane == 0) srinv[i] = ri;
+    ri_reg[i & 3] = ri;
     if (s_in == nullptr) {
-      for (int64_t c8 = lane; c8 < upr; c8 += 32) {
-        float v[8], g[8];
-        lds8(sr + c8 * 8, v);
-        lds8(sg + c8 * 8, g);
+      for (int n0 = 0; n0 < npl; n0 += 4) {
+        float v[4][8], g[4][8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) ykey = max(ykey, abs_key(__fmul_rn(__fmul_rn(v[j], ri), g[j])));
+        for (int n = 0; n < 4; ++n) {
+          const int64_t c8 = lane + 32 * (int64_t)(n0 + n);
+          const bool ok = n0 + n < npl && c8 < upr;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[n][j] = g[n][j] = 0.0f;
+          if (ok) {
+            lds8(sr + c8 * 8, v[n]);
+            lds8(sg + c8 * 8, g[n]);
+          }
+        }
+#pragma unroll
+        for (int n = 0; n < 4; ++n)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ykey = max(ykey, abs_key(__fmul_rn(__fmul_rn(v[n][j], ri), g[n][j])));
       }
     }
   }
@@ -741,9 +792,11 @@ __global__ void __launch_bounds__(256, 3) k_reorder_onepass(const T* __restrict_
     wkey[warp] = ykey;
     wbad[warp] = bad;
   }
-  __syncthreads();   // per-warp maxima, srinv and sgp are visible to every thread
+  if (gamma)   // gamma in the permuted order, for 16-byte reads in the encoder
+    for (int64_t j = threadIdx.x; j < K; j += blockDim.x) sgp[j] = sg[sperm[j]];
+  __syncthreads();   // per-warp maxima and sgp are visible to every thread
 
-  // 3. the tensor scale: one exchange of the CTA maxima through the workspace
+  // 2. the tensor scale: one exchange of the CTA maxima through the workspace
   if (threadIdx.x == 0) {
     uint32_t m = 0u, xb = 0u;
     for (int w = 0; w < 8; ++w) {
@@ -757,7 +810,7 @@ __global__ void __launch_bounds__(256, 3) k_reorder_onepass(const T* __restrict_
       atomicAdd(&ws->arrive[0], 1u);
       const uint64_t t0 = tc::globaltimer();
       int ok = 1;
-      while (ld_acquire_gpu(&ws->arrive[0]) < (uint32_t)G) {
+      while (ld_acquire_gpu(&ws->arrive[0]) < (uint32_t)gridDim.x) {
         __nanosleep(64);   // fewer polls of the shared counter while the others arrive
         if (tc::globaltimer() - t0 > tc::kTimeoutNs) {
           ok = 0;
@@ -779,7 +832,7 @@ __global__ void __launch_bounds__(256, 3) k_reorder_onepass(const T* __restrict_
     // leave after this CTA's read above; the last CTA to leave zeroes the
     // header for the next call (off the other threads' path)
     __threadfence();
-    if (atomicAdd(&ws->arrive[1], 1u) == (uint32_t)G - 1u) {
+    if (atomicAdd(&ws->arrive[1], 1u) == gridDim.x - 1u) {
       ws->amax_bits[0] = 0u;
       ws->arrive[0] = 0u;
       ws->arrive[1] = 0u;
@@ -792,22 +845,12 @@ __global__ void __launch_bounds__(256, 3) k_reorder_onepass(const T* __restrict_
   make_scale_tables(s, d_tab, inv_tab);
   __syncthreads();
 
-  // 4. encode: the CTA's main blocks, then its residue blocks, as one flat list
-  // over all threads (a residue block recomputes its main block's dequantized
-  // values), so that the S residue blocks of a row are not left to a few threads
+  // 3. each warp encodes its rows: lanes over the main blocks, then the residue
+  // blocks (a residue block recomputes its main block's dequantized values);
+  // two blocks per iteration, both gathers issued before either is encoded
   const int nb = (int)(K >> 4), nbr = (int)(S >> 4);
-  const int n_main = nrows * nb, n_all = n_main + nrows * nbr;
   const T* gp = gamma ? sgp : nullptr;
-  auto task_of = [&](int t, int& i, int& b) {
-    const bool res = t >= n_main;
-    const int u = res ? t - n_main : t;
-    const int per = res ? nbr : nb;
-    i = u / per;
-    b = u - i * per;
-    return res;
-  };
-  auto finish = [&](bool res, int i, int b, const float* v, uint32_t key) {
-    const int64_t row = (int64_t)blockIdx.x + (int64_t)i * G;
+  auto finish = [&](int64_t row, bool res, int b, const float* v, uint32_t key) {
     uint32_t db;
     float deq[16];
     const uint64_t codes = quant_block16_tab(v, key, s, d_tab, inv_tab, db, res ? deq : nullptr);
@@ -826,19 +869,18 @@ __global__ void __launch_bounds__(256, 3) k_reorder_onepass(const T* __restrict_
       store_block16(q, row, nb + b, rc, dr);
     }
   };
-  // two tasks per iteration: both gathers are issued before either is encoded
-  for (int t = threadIdx.x; t < n_all; t += 2 * blockDim.x) {
-    const int t2 = t + blockDim.x;
-    int i0, b0, i1 = 0, b1 = 0;
-    const bool r0 = task_of(t, i0, b0);
-    const bool has2 = t2 < n_all;
-    const bool r1 = has2 ? task_of(t2, i1, b1) : false;
-    float v0[16], v1[16];
-    const uint32_t k0 = gather_block(srows + (int64_t)i0 * K, sperm, gp, gamma ? srinv[i0] : 1.0f, b0, v0);
-    uint32_t k1 = 0u;
-    if (has2) k1 = gather_block(srows + (int64_t)i1 * K, sperm, gp, gamma ? srinv[i1] : 1.0f, b1, v1);
-    finish(r0, i0, b0, v0, k0);
-    if (has2) finish(r1, i1, b1, v1, k1);
+  for (int i = 0; i < nrows; ++i) {
+    const int64_t row = wg + i * W;
+    const T* sr = wrows + (int64_t)i * K;
+    const float ri = gamma ? ri_reg[i & 3] : 1.0f;
+    const int n_all = nb + nbr;
+    for (int t = lane; t < n_all; t += 32) {
+      const bool res = t >= nb;
+      const int b = res ? t - nb : t;
+      float v[16];
+      const uint32_t k = gather_block(sr, sperm, gp, ri, b, v);
+      finish(row, res, b, v, k);
+    }
   }
 }
 
@@ -1047,20 +1089,19 @@ cudaError_t launch_reorder_onepass_t(const void* x, int64_t M, int64_t K, int64_
                                      float eps, const int32_t* perm, int64_t S, const float* s_in,
                                      const QOut& q, WsHeader* ws, int* st, int num_sms, cudaStream_t stream) {
   constexpr size_t kMaxSmem = 227 * 1024;   // opt-in dynamic shared memory per CTA
-  // the most CTAs per SM (up to 4) whose rows all fit in shared memory together
-  for (int per_sm = 4; per_sm >= 1; --per_sm) {
-    const int64_t g = std::min<int64_t>((int64_t)num_sms * per_sm, M);
-    const int64_t rows = (M + g - 1) / g;
-    if (rows > 4096) continue;
-    const size_t smem = onepass_smem_bytes(sizeof(T), K, gamma != nullptr, (int)rows);
-    if (smem > kMaxSmem) continue;
+  // the fewest rows per warp (up to 4) for which every row fits in the shared
+  // memory of one wave of CTAs
+  for (int rpw = 1; rpw <= 4; ++rpw) {
+    const size_t smem = onepass_smem_bytes(sizeof(T), K, gamma != nullptr, rpw);
+    if (smem > kMaxSmem) break;
     cudaError_t e = cudaFuncSetAttribute(k_reorder_onepass<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_reorder_onepass<T>, 256, smem);
     if (e != cudaSuccess) return e;
-    if ((int64_t)occ * num_sms < g) continue;   // not all resident at once
+    const int64_t g = (M + 8 * rpw - 1) / (8 * rpw);   // CTAs of 8 warps
+    if (occ < 1 || g > (int64_t)occ * num_sms) continue;   // not all resident at once
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)g);
     cfg.blockDim = dim3(256);
@@ -1072,7 +1113,7 @@ cudaError_t launch_reorder_onepass_t(const void* x, int64_t M, int64_t K, int64_
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, k_reorder_onepass<T>, static_cast<const T*>(x), M, K, ldx,
-                           static_cast<const T*>(gamma), eps, perm, S, s_in, q, ws, (int)rows, st);
+                           static_cast<const T*>(gamma), eps, perm, S, s_in, q, ws, rpw, st);
     if (e == cudaErrorCooperativeLaunchTooLarge) {
       (void)cudaGetLastError();
       return cudaErrorNotSupported;   // nothing ran; the two passes do the work

@@ -342,3 +342,30 @@ def test_reorder_unaligned_perm_same_result(orc):
     torch.cuda.synchronize()
     assert st.item() == 0
     assert_same_q(xa, orc.rmsnorm_reorder_quantize(x, gamma, 1e-5, perm, S))
+
+
+@pytest.mark.parametrize("M,K", [(24, 512), (8192, 4096)])   # one launch / two passes
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_rmsnorm_mean_square_extremes(orc, M, K, dtype):
+    """The exact mean square at its edges: rows of subnormal values only, rows
+    where one large element pushes the others' squares below the 2^-34 grain,
+    all-zero rows and ordinary rows, with gamma, both launch forms."""
+    S = 64
+    rng = np.random.default_rng(M + (dtype == torch.float32))
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[0::4] *= np.float32(2.0 ** -130)          # fp32 subnormals (bf16: flush to the smallest normals' grain)
+    x[1::4] *= np.float32(2.0 ** -30)
+    x[1::4, 7] = np.float32(3.0e4)              # one large element per row
+    x[2::4] = 0.0
+    if dtype == torch.bfloat16:
+        x = wl.bf16_values(x)
+    gamma = rng.uniform(0.5, 1.5, K).astype(np.float32)
+    if dtype == torch.bfloat16:
+        gamma = wl.bf16_values(gamma)
+    xa = nv.NVFP4Tensor.empty(M, K + S, nv.SF_TILED)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_rmsnorm_reorder_quantize(to_dev(x, dtype), xa, gamma=to_dev(gamma, dtype), eps=1e-5, S=S,
+                                      workspace=nv.Workspace(M, K), dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, nv.status_string(st.item())
+    assert_same_q(xa, orc.rmsnorm_reorder_quantize(x, gamma, 1e-5, None, S))

@@ -67,9 +67,10 @@ def _operands(orc, M, N, K, seed):
     return x, w
 
 
-@pytest.mark.parametrize("M", [4, 64, 256])
+@pytest.mark.parametrize("M", [8, 64, 256])
 def test_gemm_wait_times_out_and_recovers(orc, M):
-    """M = 4: decode kernel (cluster split of K); 64: few-row kernel; 256: large-M GEMM."""
+    """M = 8: tensor-core decode kernel (cluster split of K); 64: few-row kernel;
+    256: large-M GEMM.  (M <= 4 runs on CUDA cores, which have no such waits.)"""
     N, K = 384, 1024
     x, w = _operands(orc, M, N, K, M)
     qa = run_quantize(to_dev(x, torch.float32), nv.SF_TILED)
@@ -82,7 +83,7 @@ def test_gemm_wait_times_out_and_recovers(orc, M):
     _timed_out_then_recovers(run, orc.gemm(orc.quantize(x), orc.quantize(w)))
 
 
-@pytest.mark.parametrize("M", [4, 64, 256])
+@pytest.mark.parametrize("M", [8, 64, 256])
 def test_residue_gemm_wait_times_out_and_recovers(orc, M):
     N, K = 256, 512
     x, w = _operands(orc, M, N, K, 100 + M)
@@ -103,7 +104,7 @@ def test_residue_gemm_wait_times_out_and_recovers(orc, M):
 def test_fused_decode_wait_times_out_and_recovers(orc, residue):
     """The fused quantize + GEMM decode kernel: its CTAs still exchange the tensor
     maximum and their partial rows with their cluster peers while timing out."""
-    M, N, K = 2, 512, 2048
+    M, N, K = 8, 512, 2048   # the tensor-core decode kernel (M <= 4 runs on CUDA cores)
     x, w = _operands(orc, M, N, K, 7)
     xt = to_dev(x, torch.float32)
     qw = run_quantize(to_dev(w, torch.float32), nv.SF_TILED)
