@@ -251,12 +251,12 @@ class DecodeWorkload:
 
     def run_step(self, step, e2e=False):
         for (M, N, K) in self.calls:
-            if e2e:
-                self.X[(M, K)].copy_(self.Xhost[(M, K)], non_blocking=True)
-            # every call of a step streams its own weight copy
-            self.call(M, N, K, step * len(self.Ms) + self.Ms.index(M))
-            if e2e:
-                self.Yhost[(M, N, K)].copy_(self.Y[(M, N, K)], non_blocking=True)
+            i = step * len(self.Ms) + self.Ms.index(M)   # every call of a step streams its own weight copy
+            if e2e:   # pinned host X -> device, quantize + GEMM, Y -> pinned host: one C-ABI call
+                self.nv.nvfp4_quantize_gemm_host(self.Xhost[(M, K)], self.X[(M, K)], self.QX[(M, K)],
+                                                 self.weight(N, K, i), self.Y[(M, N, K)], self.Yhost[(M, N, K)])
+            else:
+                self.call(M, N, K, i)
 
     def h2d_bytes(self):
         return sum(M * K * 2 for (M, N, K) in self.calls)
@@ -1013,7 +1013,9 @@ def main():
     line.update({"higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
                  "data": "synthetic", "config": config, "roofline": roofline,
                  "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d,
-                         "d2h_bytes_per_step": d2h},
+                         "d2h_bytes_per_step": d2h,
+                         "call": ("nvfp4_quantize_gemm_host (C ABI, pinned host buffers)"
+                                  if args.workload == "decode" else "torch host copies around the C-ABI calls")},
                  "gpu_launches": launches, "clocks": clocks, "detail": detail})
     if args.workload == "decode" and not args.no_prefill and not eager:
         del e2e_graphs

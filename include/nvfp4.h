@@ -155,10 +155,14 @@ nvfp4_status nvfp4_quantize_weight(const void* w, nvfp4_dtype dt, int64_t N, int
  * ARCQuant's K -> K+S compensation is this call with K+S columns
  * (ARCQuant post section 3.1-3.2: "unified GEMM call").
  * Kernel choice (K % 64 == 0 always):
- *   ROWMAJOR scales on both operands, M <= 16: CUDA-core decode GEMV;
+ *   ROWMAJOR scales on both operands, M <= 16: CUDA-core decode GEMV (K split
+ *     across a cluster of up to 8 CTAs when the activations, expanded to 1.25
+ *     bytes per element, do not fit one CTA's shared memory; K up to 71,680
+ *     at M = 16, 35,840 with a residue, twice that for each halving of M,
+ *     else NVFP4_ERR_UNSUPPORTED);
  *   TILED W scales, M <= 16 (A in either layout): tensor-core decode kernel (W
  *     is the 128-row MMA operand, K split across a thread-block cluster of up
- *     to 16 CTAs), K >= 256;
+ *     to 8 CTAs), K >= 256;
  *   TILED scales on both operands, 16 < M <= 128: tensor-core few-row kernel,
  *     K >= 256;
  *   TILED scales, M > 128: tensor-core 128x256-tile GEMM, K >= 256.
@@ -200,6 +204,21 @@ nvfp4_status nvfp4_gemm_residue(const nvfp4_tensor* a, const nvfp4_tensor* r,
 nvfp4_status nvfp4_quantize_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64_t K, int64_t ldx,
                                  const float* scale_in, nvfp4_tensor* q, const nvfp4_tensor* w, void* y,
                                  nvfp4_dtype out_dt, int64_t ldy, int* dev_status, void* stream);
+
+/* nvfp4_quantize_gemm from and to host memory, all on `stream`:
+ *   x_dev <- x_host   (M x K dense host rows copied into rows of stride ldx)
+ *   nvfp4_quantize_gemm(x_dev, ..., y_dev)
+ *   y_host <- y_dev   (M x N: rows of stride ldy copied into dense host rows)
+ * x_host and y_host are host pointers (page-locked memory makes the copies
+ * asynchronous and lets the call be captured in a CUDA graph); x_dev and y_dev
+ * are device buffers the caller owns, with the layouts nvfp4_quantize_gemm
+ * takes.  y_host holds the result once `stream` has reached this point.  Every
+ * argument is checked before the first copy is issued; errors as
+ * nvfp4_quantize_gemm, NVFP4_ERR_CUDA when a copy cannot be issued. */
+nvfp4_status nvfp4_quantize_gemm_host(const void* x_host, void* x_dev, nvfp4_dtype dt, int64_t M, int64_t K,
+                                      int64_t ldx, const float* scale_in, nvfp4_tensor* q,
+                                      const nvfp4_tensor* w, void* y_dev, void* y_host, nvfp4_dtype out_dt,
+                                      int64_t ldy, int* dev_status, void* stream);
 
 /* Number of kernel launches nvfp4_quantize_gemm (residue = 0) or
  * nvfp4_quantize_residue_gemm (residue != 0) makes for these sizes on the

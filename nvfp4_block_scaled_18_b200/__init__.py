@@ -26,10 +26,10 @@ SF_ROWMAJOR, SF_TILED = 0, 1
 EXPORTED_SYMBOLS = ("nvfp4_scales_bytes", "nvfp4_workspace_size", "nvfp4_quantize",
                     "nvfp4_quantize_residue", "nvfp4_rmsnorm_reorder_quantize", "nvfp4_gemm",
                     "nvfp4_gemm_residue", "nvfp4_quantize_gemm", "nvfp4_quantize_residue_gemm",
-                    "nvfp4_quantize_gemm_plan",
+                    "nvfp4_quantize_gemm_plan", "nvfp4_quantize_gemm_host",
                     "nvfp4_rmsnorm_reorder_quantize_noalloc", "nvfp4_mx_quantize",
-                    "nvfp4_mx_scales_bytes", "nvfp4_mx_gemm", "nvfp4_mx_gemm_residue", "nvfp4_quantize_weight", "nvfp4_test_wait_fault", "nvfp4_status_string",
-                    "nvfp4_version")
+                    "nvfp4_mx_scales_bytes", "nvfp4_mx_gemm", "nvfp4_mx_gemm_residue", "nvfp4_quantize_weight",
+                    "nvfp4_test_wait_fault", "nvfp4_status_string", "nvfp4_version")
 NVFP4_NOALLOC_MAX_ROWS = 65536
 
 
@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.nvfp4_gemm.argtypes = [T, T, P, ctypes.c_int, I64, P, P]
         lib.nvfp4_gemm_residue.argtypes = [T, T, T, P, ctypes.c_int, I64, P, P]
         lib.nvfp4_quantize_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, P, T, T, P, ctypes.c_int, I64, P, P]
+        lib.nvfp4_quantize_gemm_host.argtypes = [P, P, ctypes.c_int, I64, I64, I64, P, T, T, P, P, ctypes.c_int,
+                                                 I64, P, P]
         lib.nvfp4_quantize_gemm_plan.argtypes = [I64, I64, I64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         lib.nvfp4_quantize_gemm_plan.restype = ctypes.c_int
         lib.nvfp4_quantize_residue_gemm.argtypes = [P, ctypes.c_int, I64, I64, I64, P, P, T, T, T, P,
@@ -372,6 +374,29 @@ def nvfp4_quantize_gemm(x: torch.Tensor, q: NVFP4Tensor, w: NVFP4Tensor, y: torc
                                    ctypes.byref(qc), ctypes.byref(wc), y.data_ptr(), _out_dtype(y), _ldx(y),
                                    _ptr(dev_status), _stream(stream)),
            "nvfp4_quantize_gemm")
+
+
+def nvfp4_quantize_gemm_host(x_host: torch.Tensor, x_dev: torch.Tensor, q: NVFP4Tensor, w: NVFP4Tensor,
+                             y_dev: torch.Tensor, y_host: torch.Tensor, scale_in: Optional[torch.Tensor] = None,
+                             dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """nvfp4_quantize_gemm between host buffers: x_host (CPU, M x K, dense) is copied
+    into x_dev, the decode linear runs on the device, y_dev is copied into y_host
+    (CPU, M x N, dense); all on the stream.  Pinned host tensors keep it asynchronous."""
+    lib = load_library()
+    M, K = x_dev.shape
+    N = w.rows
+    if x_host.device.type != "cpu" or y_host.device.type != "cpu":
+        raise ValueError("x_host and y_host must be CPU tensors")
+    if tuple(x_host.shape) != (M, K) or x_host.dtype != x_dev.dtype or not x_host.is_contiguous():
+        raise ValueError("x_host must be a dense M x K tensor of x_dev's dtype")
+    if tuple(y_host.shape) != (M, N) or y_host.dtype != y_dev.dtype or not y_host.is_contiguous():
+        raise ValueError("y_host must be a dense M x N tensor of y_dev's dtype")
+    qc, wc = q.c(), w.c()
+    _check(lib.nvfp4_quantize_gemm_host(x_host.data_ptr(), x_dev.data_ptr(), _dtype_code(x_dev), M, K,
+                                        _ldx(x_dev), _ptr(scale_in), ctypes.byref(qc), ctypes.byref(wc),
+                                        y_dev.data_ptr(), y_host.data_ptr(), _out_dtype(y_dev), _ldx(y_dev),
+                                        _ptr(dev_status), _stream(stream)),
+           "nvfp4_quantize_gemm_host")
 
 
 def nvfp4_quantize_residue_gemm(x: torch.Tensor, q: NVFP4Tensor, r: Optional[NVFP4Tensor], w: NVFP4Tensor,

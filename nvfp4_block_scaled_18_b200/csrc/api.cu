@@ -345,6 +345,25 @@ nvfp4_status nvfp4_quantize_gemm(const void* x, nvfp4_dtype dt, int64_t M, int64
                                      dev_status, stream);
 }
 
+nvfp4_status nvfp4_quantize_gemm_host(const void* x_host, void* x_dev, nvfp4_dtype dt, int64_t M, int64_t K,
+                                      int64_t ldx, const float* scale_in, nvfp4_tensor* q,
+                                      const nvfp4_tensor* w, void* y_dev, void* y_host, nvfp4_dtype out_dt,
+                                      int64_t ldy, int* dev_status, void* stream) {
+  if (x_host == nullptr || y_host == nullptr) return NVFP4_ERR_INVALID_ARG;
+  NVFP4_TRY(check_input(x_dev, dt, M, K, ldx));
+  NVFP4_TRY(check_tensor(q, M, K));
+  NVFP4_TRY(check_gemm_operands(q, nullptr, w, y_dev, out_dt, ldy));
+  if (M > 16 || w->sf_layout != NVFP4_SF_TILED || K < 256) return NVFP4_ERR_UNSUPPORTED;
+  if (M * (K / 8) > quant_small_max_units(dt)) return NVFP4_ERR_UNSUPPORTED;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t es = dt_size(dt), oes = dt_size(out_dt), N = (size_t)w->rows;
+  NVFP4_TRY(cuda_status(cudaMemcpy2DAsync(x_dev, (size_t)ldx * es, x_host, (size_t)K * es, (size_t)K * es,
+                                          (size_t)M, cudaMemcpyHostToDevice, s)));
+  NVFP4_TRY(nvfp4_quantize_gemm(x_dev, dt, M, K, ldx, scale_in, q, w, y_dev, out_dt, ldy, dev_status, stream));
+  return cuda_status(cudaMemcpy2DAsync(y_host, N * oes, y_dev, (size_t)ldy * oes, N * oes, (size_t)M,
+                                       cudaMemcpyDeviceToHost, s));
+}
+
 size_t nvfp4_mx_scales_bytes(int64_t rows, int64_t cols, nvfp4_sf_layout layout) {
   if (rows <= 0 || cols <= 0) return 0;
   const int64_t nb = (cols + 31) / 32;

@@ -168,3 +168,21 @@ def test_mx_residue_validation_before_launch(lib):
     assert g(good, good, good, None, good, good, 128, 256, 256, good, 0, 256, None, None) == 1
     assert g(good, good, good + 4, good, good, good, 128, 256, 256, good, 0, 256, None, None) == 2
     assert g(good, good, good, good, good, good, 128, 256, 192, good, 0, 256, None, None) == 3
+
+
+def test_host_io_validation_before_copies(lib):
+    """nvfp4_quantize_gemm_host checks every argument before it issues a copy."""
+    good = 1 << 20
+    q, w = _tensor(4, 1024, good, good, good), _tensor(512, 1024, good, good, good, layout=1)
+    f = lib.nvfp4_quantize_gemm_host
+    assert f(None, good, 1, 4, 1024, 1024, None, ctypes.byref(q), ctypes.byref(w), good, good, 0, 512,
+             None, None) == 1                                                           # null x_host
+    assert f(good, good, 1, 4, 1024, 1024, None, ctypes.byref(q), ctypes.byref(w), good, None, 0, 512,
+             None, None) == 1                                                           # null y_host
+    assert f(good, good + 2, 1, 4, 1024, 1024, None, ctypes.byref(q), ctypes.byref(w), good, good, 0, 512,
+             None, None) == 2                                                           # misaligned x_dev
+    assert f(good, good, 1, 4, 1024, 1024, None, ctypes.byref(q), ctypes.byref(w), good, good, 0, 256,
+             None, None) == 1                                                           # ldy < N
+    q17 = _tensor(17, 1024, good, good, good)
+    assert f(good, good, 1, 17, 1024, 1024, None, ctypes.byref(q17), ctypes.byref(w), good, good, 0, 512,
+             None, None) == 3                                                           # M > 16
