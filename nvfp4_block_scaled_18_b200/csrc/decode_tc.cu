@@ -318,12 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool writer = blockIdx.y == 0;                // this cluster also writes Q(X), Q(R)
     uint32_t key = 0u;
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-      float v[8];
-      raw[i].get(v);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
-    }
+    for (int i = 0; i < R; ++i) key = max(key, raw[i].abs_key_max());
     if (key >= 0x7F800000u) report_status(p.st, NVFP4_ERR_NONFINITE);
     float s;
     if (p.s_in != nullptr) {

@@ -153,6 +153,15 @@ struct Raw8<__nv_bfloat16> {
     v[4] = __uint_as_float(u.z << 16); v[5] = __uint_as_float(u.z & 0xFFFF0000u);
     v[6] = __uint_as_float(u.w << 16); v[7] = __uint_as_float(u.w & 0xFFFF0000u);
   }
+  // max over the 8 elements of abs_key (the fp32 bit pattern of |x|), on the
+  // packed halves: |bf16| bit patterns order like the values, NaN/Inf included
+  __device__ __forceinline__ uint32_t abs_key_max() const {
+    uint32_t m;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(m) : "r"(u.x & 0x7FFF7FFFu), "r"(u.y & 0x7FFF7FFFu));
+    asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(u.z & 0x7FFF7FFFu));
+    asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(u.w & 0x7FFF7FFFu));
+    return max(m << 16, m & 0xFFFF0000u);
+  }
 };
 template <>
 struct Raw8<float> {
@@ -169,6 +178,10 @@ struct Raw8<float> {
   __device__ __forceinline__ void get(float v[8]) const {
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  __device__ __forceinline__ uint32_t abs_key_max() const {
+    return max(max(max(abs_key(a.x), abs_key(a.y)), max(abs_key(a.z), abs_key(a.w))),
+               max(max(abs_key(b.x), abs_key(b.y)), max(abs_key(b.z), abs_key(b.w))));
   }
 };
 

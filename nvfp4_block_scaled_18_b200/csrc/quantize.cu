@@ -80,12 +80,7 @@ __global__ void __launch_bounds__(256) k_amax(const T* __restrict__ x, int64_t M
         else raw[u].zero();
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        float v[8];
-        raw[u].get(v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) key = max(key, abs_key(v[i]));
-      }
+      for (int u = 0; u < kUnroll; ++u) key = max(key, raw[u].abs_key_max());
     }
   } else {
     for (int64_t row = blockIdx.y; row < M; row += gridDim.y) {
@@ -237,13 +232,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
   }
 #pragma unroll
-  for (int i = 0; i < R; ++i) {
-    float v[16];
-    raw[i][0].get(v);
-    raw[i][1].get(v + 8);
-#pragma unroll
-    for (int j = 0; j < 16; ++j) key = max(key, abs_key(v[j]));
-  }
+  for (int i = 0; i < R; ++i) key = max(key, max(raw[i][0].abs_key_max(), raw[i][1].abs_key_max()));
   if (key >= 0x7F800000u) report_status(st, NVFP4_ERR_NONFINITE);
 
   const bool exchange = s_in == nullptr || (RES && sr_in == nullptr);   // uniform
@@ -717,10 +706,7 @@ __global__ void __launch_bounds__(256, 2) k_reorder_onepass(const T* __restrict_
       for (int n = 0; n < NCH; ++n) {
         const int64_t c8 = lane + 32 * (int64_t)(n0 + n);
         if (n0 + n < npl && c8 < upr) raw[n].store_smem(sr + c8 * 8);
-        float v[8];
-        raw[n].get(v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) key = max(key, abs_key(v[j]));
+        key = max(key, raw[n].abs_key_max());
       }
     }
     key = warp_max_u32(key);
