@@ -122,6 +122,36 @@ def test_bf16_output_and_ld(orc):
     assert torch.count_nonzero(big[:, N:]) == 0
 
 
+@pytest.mark.parametrize("M,residue", [(2, False), (4, True), (8, True)])
+def test_k_split_bf16_output_and_ld(orc, M, residue):
+    """Few rows of W and a long K: the M <= 4 kernel splits K over a cluster and the
+    owners sum the peers' partial rows; bf16 output = RNE of the fp32 result, the
+    padding of the strided output rows untouched."""
+    N, K = 40, 4096
+    rng = np.random.default_rng(900 + M)
+    x = (rng.standard_normal((M, K)) * 1.5).astype(np.float32)
+    w = (rng.standard_normal((N, K)) * 0.05).astype(np.float32)
+    qw = run_quantize(to_dev(w, torch.float32))
+    y32 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    big = torch.zeros((M, N + 24), dtype=torch.bfloat16, device="cuda")
+    if residue:
+        q, r = nv.NVFP4Tensor.empty(M, K), nv.NVFP4Tensor.empty(M, K)
+        nv.nvfp4_quantize_residue(to_dev(x, torch.float32), q, r, workspace=nv.Workspace(M, K))
+        nv.nvfp4_gemm_residue(q, r, qw, y32)
+        nv.nvfp4_gemm_residue(q, r, qw, big[:, :N])
+        oq, orr = orc.quantize_residue(x)
+        ref = orc.gemm_residue(oq, orr, orc.quantize(w))
+    else:
+        qx = run_quantize(to_dev(x, torch.float32))
+        nv.nvfp4_gemm(qx, qw, y32)
+        nv.nvfp4_gemm(qx, qw, big[:, :N])
+        ref = orc.gemm(orc.quantize(x), orc.quantize(w))
+    torch.cuda.synchronize()
+    check_y(y32.cpu().numpy(), ref)
+    assert torch.equal(big[:, :N], y32.to(torch.bfloat16))
+    assert torch.count_nonzero(big[:, N:]) == 0
+
+
 def test_exact_sums_are_exact(orc):
     """Power-of-two tensor scales, small K: every partial sum is exactly representable,
     so the GPU result must equal the exact result bit for bit."""
