@@ -583,6 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 constexpr double kFixedUs = 5.0;     // launch-to-exit latency of one wave of CTAs (measured, few k-tiles)
 constexpr double kTileUs = 0.8;      // one k-tile (scale stores, 4 MMAs, 1 commit) per CTA, up to 4 CTAs per SM
 constexpr double kQuantUs = 4.0;     // one-launch quantizer plus the hand-off to the next kernel
+                                     // (with a computed residue scale, plus its second exchange)
 constexpr double kExchangeUs = 1.3;  // fused: one cluster-wide maximum (stores into peers + wait)
 constexpr double kUnitUs = 0.15;     // fused: encoding one 8-element unit per thread, per co-resident CTA
 // A request of at least this many bytes keeps at most TMEM_CTAS CTAs on an SM
@@ -708,7 +709,8 @@ cudaError_t launch_r(const DecodeArgs& a, const DecodeParams& p, const CUtensorM
     if (c2.cost < best->cost - 1e-9) { best = &c2; r = 2; }
     if (c4.cost < best->cost - 1e-9) { best = &c4; r = 4; }
     if (c8.cost < best->cost - 1e-9) { best = &c8; r = 8; }
-    if (best->ks == 0 || best->cost > plain.cost + kQuantUs) return cudaErrorNotSupported;
+    const double quant_us = kQuantUs + (RES && p.sr_in == nullptr ? kExchangeUs : 0.0);
+    if (best->ks == 0 || best->cost > plain.cost + quant_us) return cudaErrorNotSupported;
     switch (r) {
       case 1: return launch_cfg<T, true, RES, BF16OUT, 1>(a, p, *best, tmW, tmX, tmR, stream);
       case 2: return launch_cfg<T, true, RES, BF16OUT, 2>(a, p, *best, tmW, tmX, tmR, stream);
