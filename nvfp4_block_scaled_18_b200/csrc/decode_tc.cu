@@ -586,6 +586,7 @@ constexpr double kQuantUs = 4.0;     // one-launch quantizer plus the hand-off t
                                      // (with a computed residue scale, plus its second exchange)
 constexpr double kExchangeUs = 1.3;  // fused: one cluster-wide maximum (stores into peers + wait)
 constexpr double kUnitUs = 0.15;     // fused: encoding one 8-element unit per thread, per co-resident CTA
+constexpr int kGpcSms = 16;          // SMs per GPC assumed when packing clusters (the smallest GPCs)
 // A request of at least this many bytes keeps at most TMEM_CTAS CTAs on an SM
 // (228 KB per SM, 1 KB reserved per CTA), so tcgen05.alloc never waits for a
 // CTA of another cluster.
@@ -624,7 +625,11 @@ Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, i
     if (units_cap > 0 && units > (int64_t)units_cap * kThreads) continue;
     const int per_sm = ctas_per_sm(smem, regs);
     if (per_sm < 1) continue;
-    const int64_t ctas = (int64_t)row_tiles * ks, slots = (int64_t)per_sm * num_sms;
+    // a cluster must fit inside one GPC: count only the slots that whole
+    // clusters of ks CTAs can fill in GPCs of kGpcSms SMs
+    const int per_gpc = kGpcSms * per_sm;
+    const int64_t ctas = (int64_t)row_tiles * ks,
+                  slots = (int64_t)per_sm * num_sms * ((per_gpc / ks) * ks) / per_gpc;
     const int64_t waves = (ctas + slots - 1) / slots;
     double wave = kFixedUs + kTileUs * kt_max;
     if (units_cap > 0) {
