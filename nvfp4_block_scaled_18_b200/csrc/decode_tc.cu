@@ -141,8 +141,18 @@ struct DecodeParams {
 // stays below 1/d, so the quotient is exact.
 __device__ __forceinline__ int div_magic(int u, uint32_t m) { return (int)__umulhi((uint32_t)u, m); }
 
-__host__ __device__ constexpr int smem_bytes(int stages, int kt_max, int ro, int M) {
-  return 1024 + stages * WSTAGE + kt_max * (b_tile(ro) + SF_TILE) + part_bytes(M) + BAR_BYTES;
+// Fused mode encodes the activation operand of all its k-tiles up front, and
+// plain mode loads all of them at once (kt_max B tiles after the ring); plain
+// mode with the 32-row X+R operand (ro = 16) streams each k-tile's B tile
+// through the ring with its W tile instead (a stage is W_TILE + SFW_BYTES + B
+// tile), since kt_max of its 4 KB tiles would leave one CTA per SM.
+__host__ __device__ constexpr bool streams_b(int ro, bool fused) { return !fused && ro == 16; }
+__host__ __device__ constexpr int stage_bytes(int ro, bool fused) {
+  return streams_b(ro, fused) ? WSTAGE + b_tile(ro) : WSTAGE;
+}
+__host__ __device__ constexpr int smem_bytes(int stages, int kt_max, int ro, int M, bool fused) {
+  return 1024 + stages * stage_bytes(ro, fused) + kt_max * ((streams_b(ro, fused) ? 0 : b_tile(ro)) + SF_TILE) +
+         part_bytes(M) + BAR_BYTES;
 }
 
 template <typename T, bool FUSED, int RES, bool BF16OUT, int R>
@@ -153,11 +163,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int KT = p.kt_max;
   const int NS = p.stages;                                          // W ring depth
-  uint8_t* xcodes = smem + NS * WSTAGE;                             // KT x 2 KB
   constexpr int BT = b_tile(RES);                                   // B tile bytes per k-tile
+  constexpr bool STREAM = streams_b(RES, FUSED);                    // B tiles travel with the W stages
+  constexpr int SSTRIDE = stage_bytes(RES, FUSED);                  // ring stage: W (+ B tile)
   constexpr int OPR = operand_rows(RES);                            // rows of X (and of R)
+  uint8_t* xcodes = smem + NS * SSTRIDE;                            // KT B tiles (unless STREAM)
   uint8_t* rcodes = xcodes + RES * 128;                             // R rows of each B tile
-  uint8_t* sfxp = xcodes + KT * BT;                                 // KT x 512 B activation scales
+  uint8_t* sfxp = xcodes + (STREAM ? 0 : KT * BT);                  // KT x 512 B activation scales
   uint8_t* sfrp = sfxp + RES * 4;                                   // R scales: rows RES..
   const int pitch = part_pitch(p.M);
   float* part = reinterpret_cast<float*>(sfxp + KT * SF_TILE);      // pushed partial rows
@@ -221,13 +233,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool peers_running = false; // this thread has waited for the peers' start-up arrivals
 
   auto w_chunks = [&](int kt) { return min(4, (p.K - kt * 256) / 64); };   // K = 64 chunks in k-tile kt
-  auto load_w = [&](int kt, int s) {
+  auto load_w = [&](int kt, int s) {   // the stage's W tile and scale atoms (STREAM: and its B tile)
     const uint32_t sf = (uint32_t)w_chunks(kt) * 512u;
-    uint8_t* sb = smem + s * WSTAGE;
+    uint8_t* sb = smem + s * SSTRIDE;
     const uint32_t bar = saddr(&full[s]);
-    mbar_expect_tx(bar, (uint32_t)W_TILE + sf);
+    mbar_expect_tx(bar, (uint32_t)W_TILE + sf + (STREAM ? (uint32_t)BT : 0u));
     tma_load_2d(saddr(sb), &tmW, kt * 128, rt * 128, bar);
     bulk_load(saddr(sb + W_TILE), p.sfw + ((size_t)rt * p.katoms_w + kt * 4) * 512, sf, bar);
+    if (STREAM) {
+      tma_load_2d(saddr(sb + WSTAGE), &tmX, kt * 128, 0, bar);
+      if (RES) tma_load_2d(saddr(sb + WSTAGE + RES * 128), &tmR, kt * 128, 0, bar);
+    }
   };
 
   if (warp == 0 && lane == 0) {
@@ -262,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pre = p.hold ? 0 : min(nkt, NS);   // every stage of the ring is loaded at once
   int issued = pre;   // W stages loaded (warp 0 lane 0)
   if (warp == 0 && lane == 0) {
-    if (!FUSED) {
+    if (!FUSED && !STREAM) {
       mbar_expect_tx(saddr(x_full), (uint32_t)(nkt * BT));
       for (int t = 0; t < nkt; ++t) {
         tma_load_2d(saddr(xcodes + t * BT), &tmX, (kt0 + t) * 128, 0, saddr(x_full));
@@ -403,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // flight if a consumer gave up: let them land before the CTA can exit
     for (int g2 = max(0, issued - NS); g2 < issued; ++g2)
       (void)mbar_drain(saddr(&full[g2 % NS]), (uint32_t)((g2 / NS) & 1), abort_flag, p.st);
-    if (!FUSED) (void)mbar_drain(saddr(x_full), 0u, abort_flag, p.st);
+    if (!FUSED && !STREAM) (void)mbar_drain(saddr(x_full), 0u, abort_flag, p.st);
   } else if (warp >= 4) {
     // ------------------------------------------- scales into TMEM (tcgen05.st)
     // Warp w writes TMEM lane quadrant w - 4 of scale buffer t & 1 for the
@@ -416,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // is still the current one of its barrier).
     const uint32_t quad = (uint32_t)((warp - 4) * 32) << 16;
     auto write_tile = [&](int t, int s) {
-      const uint8_t* sb = smem + s * WSTAGE;
+      const uint8_t* sb = smem + s * SSTRIDE;
       uint32_t r[32];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -462,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------- MMA issuer
     bool ok = true;
-    if (!FUSED) ok = mbar_wait(saddr(x_full), 0u, abort_flag, p.st);
+    if (!FUSED && !STREAM) ok = mbar_wait(saddr(x_full), 0u, abort_flag, p.st);
     const uint32_t idesc = idesc_nvf4(RES == 16 ? 2 * NP : NP);
     for (int t = 0; ok && t < nkt; ++t) {
       const int s = t % NS;
@@ -470,9 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(saddr(&sf_full[t & 1]), (uint32_t)((t >> 1) & 1), abort_flag, p.st)) break;
       tc_fence_after();
       const int kt = kt0 + t, jmax = w_chunks(kt);
-      const uint8_t* sb = smem + s * WSTAGE;
+      const uint8_t* sb = smem + s * SSTRIDE;
       const uint32_t sfw = SF_COL + (uint32_t)(t & 1) * SF_BUF, sfx = sfw + SFX_OFF;
-      const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(xcodes + t * BT));
+      const uint64_t dw = desc_sw128(saddr(sb)), dx = desc_sw128(saddr(STREAM ? sb + WSTAGE : xcodes + t * BT));
       for (int j = 0; j < jmax; ++j) {
         const uint32_t acc = (t > 0 || j > 0) ? 1u : 0u;
         tc_mma_nvf4(tmem + ACC, dw + (uint64_t)(2 * j), dx + (uint64_t)(2 * j), idesc, tmem + sfw + 4 * j,
@@ -618,7 +634,7 @@ Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, i
   Choice best;
   for (int ks = 1; ks <= std::min(MAX_KS, k_tiles); ++ks) {
     const int kt_max = (k_tiles + ks - 1) / ks;
-    const int smem = std::max(smem_bytes(2, kt_max, ro, M), kSmemFloor);
+    const int smem = std::max(smem_bytes(2, kt_max, ro, M, units_cap > 0), kSmemFloor);
     if (smem > 232448) continue;
     const int slice = std::min(kt_max * 256, K);
     const int64_t units = (int64_t)M * (slice / 8);
@@ -642,7 +658,7 @@ Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, i
   }
   if (best.ks > 0)
     for (int st = 3; st <= std::min(MAX_STAGES, best.kt_max); ++st) {
-      const int smem = std::max(smem_bytes(st, best.kt_max, ro, M), kSmemFloor);
+      const int smem = std::max(smem_bytes(st, best.kt_max, ro, M, units_cap > 0), kSmemFloor);
       if (smem > 232448 || ctas_per_sm(smem, regs) < ctas_per_sm(best.smem, regs)) break;
       best.stages = st;
       best.smem = smem;
