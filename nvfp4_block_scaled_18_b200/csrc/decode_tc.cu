@@ -135,6 +135,7 @@ struct DecodeParams {
   int* st;
   uint64_t wait_ns;     // bound on every mbarrier wait
   int hold;             // test of the timeout path: no W tile is loaded
+  int prefetch;         // prefetch W into L2 before the dependency wait
 };
 
 // u / d for u < 2^16, d < 2^16 with m = ceil(2^32 / d): the error u*(m - 2^32/d)/2^32
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
 
-  if (warp == 0 && lane == 0) {
+  if (p.prefetch && warp == 0 && lane == 0) {
     // warm L2 with this CTA's W tiles and scale atoms while the preceding kernel finishes
     for (int kt = kt0; kt < kt1; ++kt) {
       prefetch_l2_tile_2d(&tmW, kt * 128, rt * 128);
@@ -800,6 +801,7 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, int num_sms, cudaStream_t stre
   const WaitTest wt = wait_test();
   p.wait_ns = wt.limit_ns;
   p.hold = wt.hold;
+  p.prefetch = prefetch_w(a.N, a.K) ? 1 : 0;
   if (fused)
     return a.x_bf16 ? launch_t<__nv_bfloat16, true>(a, p, tmW, tmX, tmR, num_sms, stream)
                     : launch_t<float, true>(a, p, tmW, tmX, tmR, num_sms, stream);

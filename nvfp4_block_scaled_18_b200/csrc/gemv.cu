@@ -143,6 +143,7 @@ struct GemvLayout {
 struct GemvParams {
   GemmArgs g;
   int ks, rows_per_cta, pairs;
+  int prefetch;   // prefetch the W rows into L2 before the dependency wait
 };
 
 template <int MT, int RL, bool RES, bool BF16OUT>
@@ -166,8 +167,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_gemv(const GemvParams p) {
   const int xpitch = L.slice_pairs * 64, dpitch = L.slice_pairs * 4;
 
   // warm L2 with this CTA's W rows while the preceding kernel finishes
-  for (int r = r0 + (int)threadIdx.x; r < r1; r += kThreads)
-    prefetch_l2_bulk(g.w_codes + (int64_t)r * cpitch + k0 / 2, (uint32_t)chunks * 16u);
+  if (p.prefetch)
+    for (int r = r0 + (int)threadIdx.x; r < r1; r += kThreads)
+      prefetch_l2_bulk(g.w_codes + (int64_t)r * cpitch + k0 / 2, (uint32_t)chunks * 16u);
   griddep_wait();   // everything below may read the preceding kernel's results
 
   // ---- expand the activation (and residue) slice: int8 2 v(c) and fp32 scales
@@ -671,7 +673,7 @@ cudaError_t launch_t(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   auto kern = k_gemv<MT, RL, RES, BF16OUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem);
   if (e != cudaSuccess) return e;
-  const GemvParams p{g, c.ks, c.rows_per_cta, (int)(g.K / 64)};
+  const GemvParams p{g, c.ks, c.rows_per_cta, (int)(g.K / 64), prefetch_w(g.N, g.K) ? 1 : 0};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)c.ks, (unsigned)((g.N + c.rows_per_cta - 1) / c.rows_per_cta), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -104,6 +104,7 @@ struct SwapParams {
   int* st;
   uint64_t wait_ns;   // bound on every mbarrier wait
   int hold;           // test of the timeout path: the producer loads nothing
+  int prefetch;       // prefetch W into L2 before the dependency wait
 };
 
 template <int NP, bool RES, bool BF16OUT>
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0 && lane == 0) {
+  if (p.prefetch && warp == 0 && lane == 0) {
     // warm L2 with this CTA's W tiles and scale atoms while the preceding kernel finishes
     for (int kt = kt0; kt < kt1; ++kt) {
       prefetch_l2_tile_2d(&tmW, kt * 128, rt * 128);
@@ -368,6 +369,7 @@ cudaError_t launch_np(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   const WaitTest wt = wait_test();
   p.wait_ns = wt.limit_ns;
   p.hold = wt.hold;
+  p.prefetch = prefetch_w(g.N, g.K) ? 1 : 0;
   const int row_tiles = (int)((g.N + 127) / 128);
   auto kern = k_gemv_tc<NP, RES, BF16OUT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);

@@ -74,6 +74,13 @@ WaitTest wait_test();
 // The default bound on a device-side wait (4 s).
 constexpr uint64_t tc_wait_default_ns() { return 4000000000ull; }
 
+// The decode-sized kernels ask L2 to prefetch their W before their dependency
+// wait, so that W streams while the preceding kernel finishes.  Beyond about a
+// third of L2 (126 MB) the prefetched W and the W the preceding kernel is still
+// streaming evict each other, so larger W is not prefetched.
+constexpr int64_t kPrefetchMaxBytes = 40ll << 20;
+inline bool prefetch_w(int64_t N, int64_t K) { return N * K / 16 * 9 <= kPrefetchMaxBytes; }
+
 // Operands of the decode GEMV / tensor-core GEMM.
 struct GemmArgs {
   const uint8_t* a_codes; const uint8_t* a_scales; const float* a_s;   // M x K
