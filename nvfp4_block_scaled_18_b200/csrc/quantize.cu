@@ -197,11 +197,13 @@ __global__ void __launch_bounds__(256) k_quant(const T* __restrict__ x, int64_t 
 // identical to the multi-launch path.
 
 constexpr int kQC = 8;              // CTAs per cluster (portable cluster size)
+constexpr int kQCWide = 16;         // CTAs per cluster for the largest inputs (non-portable size)
 constexpr int kQThreads = 512;      // threads per CTA
-constexpr int kQUnitsPerChunk = kQC * kQThreads;   // 16-element blocks per chunk of the cluster
+constexpr int kQUnitsPerChunk = kQC * kQThreads;   // 16-element blocks per chunk of an 8-CTA cluster
 
-// Block u (16 elements) of this thread's i-th chunk.  Grid: exactly one cluster.
-template <typename T, int R, bool RES>
+// Block u (16 elements) of this thread's i-th chunk.  Grid: exactly one cluster
+// of QC CTAs.
+template <typename T, int R, bool RES, int QC>
 __global__ void __launch_bounds__(kQThreads, 1)
     k_quant_cluster(const T* __restrict__ x, int M, int K, int64_t ldx, const float* s_in,
                     const float* sr_in, QOut q, QOut r, int* st) {
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   uint32_t key = 0u;
 #pragma unroll
   for (int i = 0; i < R; ++i) {
-    const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
+    const int u = (i * QC + (int)rank) * kQThreads + (int)threadIdx.x;
     if (u < U) {
       const int row = u / nb, b = u - row * nb;
       const T* src = x + (int64_t)row * ldx + (int64_t)b * 16;
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
   uint32_t rkey = 0u;
 #pragma unroll
   for (int i = 0; i < R; ++i) {
-    const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
+    const int u = (i * QC + (int)rank) * kQThreads + (int)threadIdx.x;
     const bool act = u < U;
     const int row = act ? u / nb : 0, b = act ? u - row * nb : 0;
     float v[16], deq[16];
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
     if (reporter) *r.s = s_r;
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-      const int u = (i * kQC + (int)rank) * kQThreads + (int)threadIdx.x;
+      const int u = (i * QC + (int)rank) * kQThreads + (int)threadIdx.x;
       if (u >= U) continue;
       const int row = u / nb, b = u - row * nb;
       float v[16], deq[16], rv[16];
@@ -879,26 +881,53 @@ int64_t quant_small_max_units(nvfp4_dtype dt) {
   return 2 * (int64_t)kQUnitsPerChunk * (dt == NVFP4_BF16 ? 8 : 4);
 }
 
-template <typename T, int R, bool RES>
-cudaError_t launch_quant_cluster_r(const void* x, int64_t M, int64_t K, int64_t ldx, const float* s_in,
-                                   const float* sr_in, const QOut& q, const QOut& r, int* st,
-                                   cudaStream_t stream) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kQC, 1, 1);
+template <int QC>
+void quant_cluster_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, cudaStream_t stream) {
+  cfg = cudaLaunchConfig_t{};
+  cfg.gridDim = dim3(QC, 1, 1);
   cfg.blockDim = dim3(kQThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kQC;
+  attr[0].val.clusterDim.x = QC;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the preceding kernel's tail
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k_quant_cluster<T, R, RES>, static_cast<const T*>(x), (int)M, (int)K, ldx,
+}
+
+template <typename T, int R, bool RES, int QC = kQC>
+cudaError_t launch_quant_cluster_r(const void* x, int64_t M, int64_t K, int64_t ldx, const float* s_in,
+                                   const float* sr_in, const QOut& q, const QOut& r, int* st,
+                                   cudaStream_t stream) {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  quant_cluster_config<QC>(cfg, attr, stream);
+  return cudaLaunchKernelEx(&cfg, k_quant_cluster<T, R, RES, QC>, static_cast<const T*>(x), (int)M, (int)K, ldx,
                             s_in, sr_in, q, r, st);
+}
+
+// Whether a 16-CTA cluster of this instance can be resident on the device
+// (the cluster must fit in one GPC); queried once per instance.
+template <typename T, int R, bool RES>
+bool wide_cluster_fits() {
+  static int fits = -1;
+  if (fits < 0) {
+    auto kern = k_quant_cluster<T, R, RES, kQCWide>;
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+      cudaLaunchConfig_t cfg;
+      cudaLaunchAttribute attr[2];
+      quant_cluster_config<kQCWide>(cfg, attr, nullptr);
+      cfg.numAttrs = 1;   // the cluster dimension only
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    }
+    (void)cudaGetLastError();   // a refused query leaves no error for the next launch
+    fits = n >= 1 ? 1 : 0;
+  }
+  return fits == 1;
 }
 
 template <typename T, bool RES>
@@ -911,6 +940,9 @@ cudaError_t launch_quant_cluster_t(const void* x, int64_t M, int64_t K, int64_t 
   if (chunks <= 2) return launch_quant_cluster_r<T, 2, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
   if (chunks <= 4) return launch_quant_cluster_r<T, 4, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
   if constexpr (sizeof(T) == 2) {
+    // twice the CTAs (16 SMs of one GPC) rather than twice the blocks per thread
+    if (chunks <= 8 && wide_cluster_fits<T, 4, RES>())
+      return launch_quant_cluster_r<T, 4, RES, kQCWide>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
     if (chunks <= 8) return launch_quant_cluster_r<T, 8, RES>(x, M, K, ldx, s_in, sr_in, q, r, st, stream);
   }
   return cudaErrorNotSupported;
