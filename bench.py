@@ -169,7 +169,7 @@ def replica_throughput(work: float, ms: float, world: int, scale: float):
 
 # DRAM traffic / algorithmic bytes of k_decode_tc from its ncu capture (None once the kernel
 # changes after the capture)
-DECODE_TRAFFIC_RATIO = 33.103616e6 / (4096 * 14336 * 9 / 16 + 1 * 14336 * (2 + 9 / 16) + 4 * 1 * 4096)
+DECODE_TRAFFIC_RATIO = 33.103104e6 / (4096 * 14336 * 9 / 16 + 1 * 14336 * (2 + 9 / 16) + 4 * 1 * 4096)
 
 
 def decode_bytes(M, N, K):
