@@ -385,23 +385,15 @@ cudaError_t launch_np(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap the preceding kernel's tail
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  // The largest K split whose clusters are all resident at once (one wave).  A
-  // cluster must fit inside one GPC, so the count of resident clusters comes from
-  // the occupancy query, not from CTAs per SM x SMs; it is cached per split.
-  static int resident[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+  // The largest K split whose clusters all fit at once (one wave).  A cluster
+  // must fit inside one GPC, so count only the slots that whole clusters of c
+  // CTAs fill in GPCs of 16 SMs (the smaller GPCs), not CTAs per SM x SMs.
+  constexpr int kGpcSms = 16;
+  const int per_gpc = kGpcSms * C::CTAS_PER_SM;
   int ks = 1;
   for (int c = std::min(8, p.k_tiles); c > 1; --c) {
-    if (c * row_tiles > C::CTAS_PER_SM * num_sms) continue;
-    if (resident[c] == 0) {
-      attr[0].val.clusterDim.x = (unsigned)c;
-      cfg.gridDim = dim3((unsigned)c, 1, 1);
-      int n = 0;
-      e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
-      if (e != cudaSuccess) return e;
-      resident[c] = std::max(n, 1);
-    }
-    if (resident[c] >= row_tiles) {
+    const int64_t slots = (int64_t)C::CTAS_PER_SM * num_sms * ((per_gpc / c) * c) / per_gpc;
+    if ((int64_t)c * row_tiles <= slots) {
       ks = c;
       break;
     }
