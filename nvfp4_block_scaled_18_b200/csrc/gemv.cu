@@ -6,8 +6,7 @@
 // The small-M CUDA-core kernel of the ReSET summary (section "CUDA kernel
 // optimisation") is the prior art this follows; the layout below is our own.
 //
-// Two kernels share the arithmetic below.  M <= 4 (k_gemv), where the W stream
-// bounds the time:
+// Two kernels share the arithmetic below.  M <= 8 (k_gemv):
 //   row-step = 1024 K-elements of one W row: 512 code bytes + 64 scale bytes.
 //              The 32 lanes of a warp take consecutive 16-byte code chunks
 //              (32 elements, two blocks) of the same row, so every copy of a
@@ -27,7 +26,7 @@
 //              butterfly (V values over 32 lanes in V - 1 + 5 - log2 V
 //              shuffles), scaled by 1/4 s_a s_w (the two doubled operands),
 //              with the residue term s_r s_w folded in before the reduction.
-// 4 < M <= 16 (k_gemv_lanes), where the dp4a rate bounds the time: one W row
+// 8 < M <= 16 (k_gemv_lanes), where the dp4a rate bounds the time: one W row
 // per lane, activations read at one address by the whole warp (see below).
 // Math (both): W codes become int8 values 2 v(c) by a byte-permute table; a
 // 16-element block dot is 4 dp4a (exact in int32, |dot| <= 2304); the block
@@ -406,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_gemv(const GemvParams p) {
 }
 
 // ------------------------------------------------------------------------
-// 4 < M <= 16: one W row per lane.  A CTA of 8 warps takes 32 rows of W; K is
+// 8 < M <= 16: one W row per lane.  A CTA of 8 warps takes 32 rows of W; K is
 // split into 8 contiguous ranges, one per warp.  Each lane streams its row (32
 // code bytes + 4 scale bytes per 64-element step) through a 6-deep per-warp
 // cp.async ring together with the activation codes of the same step, which
@@ -707,7 +706,7 @@ cudaError_t launch_gemv(const GemmArgs& g, int num_sms, cudaStream_t stream) {
   if (g.M <= 1) return launch_m<1, 2>(g, num_sms, stream);
   if (g.M <= 2) return launch_m<2, 2>(g, num_sms, stream);
   if (g.M <= 4) return launch_m<4, 2>(g, num_sms, stream);
-  if (g.M <= 8) return launch_lanes_m<8>(g, stream);
+  if (g.M <= 8) return launch_m<8, 2>(g, num_sms, stream);
   return launch_lanes_m<16>(g, stream);
 }
 
