@@ -632,6 +632,15 @@ int ctas_per_sm(int smem, int regs) {
 // residency and loses a whole wave where it does.
 Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, int M, int K, int units_cap) {
   const bool res = ro != 0;
+  // waves of ks-CTA clusters with `per_sm` CTAs per SM: a cluster must fit
+  // inside one GPC, so count only the slots that whole clusters fill in GPCs
+  // of kGpcSms SMs
+  auto waves_of = [&](int ks, int per_sm) {
+    const int per_gpc = kGpcSms * per_sm;
+    const int64_t ctas = (int64_t)row_tiles * ks,
+                  slots = (int64_t)per_sm * num_sms * ((per_gpc / ks) * ks) / per_gpc;
+    return slots > 0 ? (ctas + slots - 1) / slots : int64_t(1) << 40;
+  };
   Choice best;
   for (int ks = 1; ks <= std::min(MAX_KS, k_tiles); ++ks) {
     const int kt_max = (k_tiles + ks - 1) / ks;
@@ -642,12 +651,8 @@ Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, i
     if (units_cap > 0 && units > (int64_t)units_cap * kThreads) continue;
     const int per_sm = ctas_per_sm(smem, regs);
     if (per_sm < 1) continue;
-    // a cluster must fit inside one GPC: count only the slots that whole
-    // clusters of ks CTAs can fill in GPCs of kGpcSms SMs
-    const int per_gpc = kGpcSms * per_sm;
-    const int64_t ctas = (int64_t)row_tiles * ks,
-                  slots = (int64_t)per_sm * num_sms * ((per_gpc / ks) * ks) / per_gpc;
-    const int64_t waves = (ctas + slots - 1) / slots;
+    const int64_t ctas = (int64_t)row_tiles * ks, slots = (int64_t)per_sm * num_sms;
+    const int64_t waves = waves_of(ks, per_sm);
     double wave = kFixedUs + kTileUs * kt_max;
     if (units_cap > 0) {
       const double upt = (double)((units + kThreads - 1) / kThreads) * (res ? 2.0 : 1.0);
@@ -657,13 +662,28 @@ Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, i
     const double cost = (double)waves * wave;
     if (cost < best.cost - 1e-9) best = Choice{ks, kt_max, 2, smem, cost};
   }
-  if (best.ks > 0)
-    for (int st = 3; st <= std::min(MAX_STAGES, best.kt_max); ++st) {
-      const int smem = std::max(smem_bytes(st, best.kt_max, ro, M, units_cap > 0), kSmemFloor);
-      if (smem > 232448 || ctas_per_sm(smem, regs) < ctas_per_sm(best.smem, regs)) break;
-      best.stages = st;
-      best.smem = smem;
+  // A ring that holds every W tile of the CTA, if the CTAs still fit in as
+  // many waves (measured: all tiles in flight at once gains; a partly deeper
+  // ring with fewer CTAs per SM can lose); else a deeper ring only while it
+  // keeps the same number of CTAs per SM.
+  if (best.ks > 0) {
+    const int64_t waves = waves_of(best.ks, ctas_per_sm(best.smem, regs));
+    const int all = best.kt_max;
+    const int smem_all = std::max(smem_bytes(all, all, ro, M, units_cap > 0), kSmemFloor);
+    const int per_sm_all = ctas_per_sm(smem_all, regs);
+    if (all > 2 && all <= MAX_STAGES && smem_all <= 232448 && per_sm_all >= 1 &&
+        waves_of(best.ks, per_sm_all) <= waves) {
+      best.stages = all;
+      best.smem = smem_all;
+    } else {
+      for (int st = 3; st <= std::min(MAX_STAGES, best.kt_max); ++st) {
+        const int smem = std::max(smem_bytes(st, best.kt_max, ro, M, units_cap > 0), kSmemFloor);
+        if (smem > 232448 || ctas_per_sm(smem, regs) < ctas_per_sm(best.smem, regs)) break;
+        best.stages = st;
+        best.smem = smem;
+      }
     }
+  }
   return best;
 }
 
