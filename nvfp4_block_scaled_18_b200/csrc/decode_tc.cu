@@ -624,13 +624,14 @@ int ctas_per_sm(int smem, int regs) {
 
 // Cluster split of K for a kernel instance with `regs` registers per thread:
 // waves of resident CTAs cost a fixed latency plus the per-CTA time of their
-// k-tiles and, fused (units_cap > 0), the cluster-wide maxima and the encoding
+// k-tiles and, fused (units_cap > 0), the `exchanges` cluster-wide maxima and the encoding
 // of the CTA's activation slice (every unit of which must fit in units_cap
 // register arrays per thread).  The smaller split wins ties.  The W ring then
 // takes as many stages (up to the CTA's k-tiles) as keep the same number of
 // CTAs per SM: measured, a deeper ring gains a little where it costs no
 // residency and loses a whole wave where it does.
-Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, int M, int K, int units_cap) {
+Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, int M, int K, int units_cap,
+                    int exchanges) {
   const bool res = ro != 0;
   // waves of ks-CTA clusters with `per_sm` CTAs per SM: a cluster must fit
   // inside one GPC, so count only the slots that whole clusters fill in GPCs
@@ -657,7 +658,7 @@ Choice choose_split(int row_tiles, int k_tiles, int ro, int num_sms, int regs, i
     if (units_cap > 0) {
       const double upt = (double)((units + kThreads - 1) / kThreads) * (res ? 2.0 : 1.0);
       const double co_resident = (double)std::min<int64_t>(per_sm, (std::min(ctas, slots) + num_sms - 1) / num_sms);
-      wave += kExchangeUs * (res ? 2.0 : 1.0) + kUnitUs * co_resident * upt;
+      wave += kExchangeUs * exchanges + kUnitUs * co_resident * upt;
     }
     const double cost = (double)waves * wave;
     if (cost < best.cost - 1e-9) best = Choice{ks, kt_max, 2, smem, cost};
@@ -735,17 +736,19 @@ cudaError_t launch_r(const DecodeArgs& a, const DecodeParams& p, const CUtensorM
   const int M = (int)a.M, K = (int)a.K;
   // the same kernel on NVFP4 operands: the split for the plain instance
   const Choice plain = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<float, false, RES, BF16OUT, 0>(),
-                                    M, K, 0);
+                                    M, K, 0, 0);
   if constexpr (!FUSED) {
     if (plain.ks == 0) return cudaErrorNotSupported;
     return launch_cfg<float, false, RES, BF16OUT, 0>(a, p, plain, tmW, tmX, tmR, stream);
   } else {
     // fused: the register-array size with the cheapest split; not worth it
     // (cudaErrorNotSupported) when quantizing separately is estimated faster
-    const Choice c1 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 1>(), M, K, 1);
-    const Choice c2 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 2>(), M, K, 2);
-    const Choice c4 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 4>(), M, K, 4);
-    const Choice c8 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 8>(), M, K, 8);
+    // one cluster-wide maximum per tensor scale not given
+    const int ex = (p.s_in == nullptr ? 1 : 0) + (RES && p.sr_in == nullptr ? 1 : 0);
+    const Choice c1 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 1>(), M, K, 1, ex);
+    const Choice c2 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 2>(), M, K, 2, ex);
+    const Choice c4 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 4>(), M, K, 4, ex);
+    const Choice c8 = choose_split(row_tiles, p.k_tiles, RES, num_sms, regs_of<T, true, RES, BF16OUT, 8>(), M, K, 8, ex);
     const Choice* best = &c1;
     int r = 1;
     if (c2.cost < best->cost - 1e-9) { best = &c2; r = 2; }

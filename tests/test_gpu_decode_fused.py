@@ -79,8 +79,12 @@ def test_fused_resserve_shapes(orc, N, K):
         assert err <= REL_FRO_TOL, (M, err)
 
 
+# (3, 100, 320) and (4, 300, 4160): a ragged last k-tile, so the CTAs of a
+# cluster encode slices of two widths; M = 3: the last warp holding units is
+# only partly filled
 @pytest.mark.parametrize("M,N,K", [(1, 1, 256), (3, 100, 320), (16, 200, 4224), (5, 130, 512), (16, 4000, 1088),
-                                   (2, 513, 14336), (9, 128, 27648)])
+                                   (2, 513, 14336), (9, 128, 27648), (4, 300, 4096), (1, 260, 16384),
+                                   (4, 300, 4160)])
 @pytest.mark.parametrize("residue", [False, True])
 @pytest.mark.parametrize("layout", [T, RM])
 def test_fused_ragged(orc, M, N, K, residue, layout):

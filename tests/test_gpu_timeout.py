@@ -101,10 +101,13 @@ def test_residue_gemm_wait_times_out_and_recovers(orc, M):
 
 
 @pytest.mark.parametrize("residue", [False, True])
-def test_fused_decode_wait_times_out_and_recovers(orc, residue):
+@pytest.mark.parametrize("M,K", [(8, 2048), (16, 2048)])
+def test_fused_decode_wait_times_out_and_recovers(orc, residue, M, K):
     """The fused quantize + GEMM decode kernel: its CTAs still exchange the tensor
-    maximum and their partial rows with their cluster peers while timing out."""
-    M, N, K = 8, 512, 2048   # the tensor-core decode kernel (M <= 4 runs on CUDA cores)
+    maxima and their partial rows with their cluster peers while timing out
+    (M = 8: X and R share one 16-row operand; M = 16: a 32-row operand)."""
+    N = 512   # the tensor-core decode kernel (M <= 4 runs on CUDA cores)
+    assert nv.nvfp4_quantize_gemm_plan(M, N, K, x_dtype=torch.float32, residue=residue) == 1
     x, w = _operands(orc, M, N, K, 7)
     xt = to_dev(x, torch.float32)
     qw = run_quantize(to_dev(w, torch.float32), nv.SF_TILED)
