@@ -590,12 +590,12 @@ __device__ __forceinline__ void lds8(const float* p, float v[8]) {
 
 // Shared-memory layout of k_reorder_onepass: the permutation (16-bit), gamma
 // in source and in permuted order, the d and 1/(d s) tables of the block
-// encoder, then rpw row buffers for each of the 8 warps.
+// encoder, then rpw row buffers for each of the CTA's wpc warps (4..8).
 __host__ __device__ inline size_t onepass_fixed_bytes(size_t es, int64_t K, bool has_gamma) {
   return (((size_t)K * 2 + 15) & ~size_t(15)) + (has_gamma ? 2 * (size_t)K * es : 0) + 2 * 256 * 4;
 }
-inline size_t onepass_smem_bytes(size_t es, int64_t K, bool has_gamma, int rpw) {
-  return onepass_fixed_bytes(es, K, has_gamma) + (size_t)8 * rpw * (size_t)K * es;
+inline size_t onepass_smem_bytes(size_t es, int64_t K, bool has_gamma, int rpw, int wpc) {
+  return onepass_fixed_bytes(es, K, has_gamma) + (size_t)wpc * rpw * (size_t)K * es;
 }
 
 // 8 consecutive elements from global memory (16/32-byte aligned) as fp32.
@@ -666,6 +666,7 @@ __global__ void __launch_bounds__(256, 2) k_reorder_onepass(const T* __restrict_
   __shared__ float s_sh;
   __shared__ int ok_sh;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpc = (int)(blockDim.x >> 5);   // warps of this CTA, 4..8
   const int64_t row_bytes = K * (int64_t)sizeof(T);   // a multiple of 16 (K % 16 == 0)
   uint16_t* sperm = reinterpret_cast<uint16_t*>(smem);
   T* sg = reinterpret_cast<T*>(smem + ((K * 2 + 15) & ~int64_t(15)));   // gamma, source order
@@ -674,7 +675,7 @@ __global__ void __launch_bounds__(256, 2) k_reorder_onepass(const T* __restrict_
   float* inv_tab = d_tab + 256;
   T* wrows = reinterpret_cast<T*>(smem + onepass_fixed_bytes(sizeof(T), K, gamma != nullptr)) +
              (int64_t)warp * rpw * K;
-  const int64_t W = (int64_t)gridDim.x * 8, wg = (int64_t)blockIdx.x * 8 + warp;   // warps, this warp
+  const int64_t W = (int64_t)gridDim.x * wpc, wg = (int64_t)blockIdx.x * wpc + warp;   // warps, this warp
   int nrows = 0;   // rows of this warp: wg + i * W
   while (nrows < rpw && wg + nrows * W < M) ++nrows;
 
@@ -787,7 +788,7 @@ __global__ void __launch_bounds__(256, 2) k_reorder_onepass(const T* __restrict_
   // 2. the tensor scale: one exchange of the CTA maxima through the workspace
   if (threadIdx.x == 0) {
     uint32_t m = 0u, xb = 0u;
-    for (int w = 0; w < 8; ++w) {
+    for (int w = 0; w < wpc; ++w) {
       m = max(m, wkey[w]);
       xb = max(xb, wbad[w]);
     }
@@ -1107,22 +1108,42 @@ cudaError_t launch_reorder_onepass_t(const void* x, int64_t M, int64_t K, int64_
                                      float eps, const int32_t* perm, int64_t S, const float* s_in,
                                      const QOut& q, WsHeader* ws, int* st, int num_sms, cudaStream_t stream) {
   constexpr size_t kMaxSmem = 227 * 1024;   // opt-in dynamic shared memory per CTA
-  // the fewest rows per warp (up to 4) for which every row fits in the shared
-  // memory of one wave of CTAs
+  // The fewest rows per warp (up to 4) for which every row fits in the shared
+  // memory of one wave of CTAs.  The kernel is bound by instruction issue, so
+  // its time follows the busiest SM: the warps per CTA (4..8) are the ones
+  // that put the fewest rows on any SM (2048 rows on 148 SMs: 7 warps, 14
+  // rows per SM, where 8 warps leave 16 on most SMs and 8 on the rest).
+  auto set_smem = [](size_t smem) {
+    return cudaFuncSetAttribute(k_reorder_onepass<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  };
+  cudaError_t e = cudaSuccess;
   for (int rpw = 1; rpw <= 4; ++rpw) {
-    const size_t smem = onepass_smem_bytes(sizeof(T), K, gamma != nullptr, rpw);
-    if (smem > kMaxSmem) break;
-    cudaError_t e = cudaFuncSetAttribute(k_reorder_onepass<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    int wpc = 0;
+    int64_t g = 0, best_load = INT64_MAX;
+    for (int w = 8; w >= 4; --w) {
+      const size_t smem = onepass_smem_bytes(sizeof(T), K, gamma != nullptr, rpw, w);
+      if (smem > kMaxSmem) continue;
+      e = set_smem(smem);
+      if (e != cudaSuccess) return e;
+      int occ = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_reorder_onepass<T>, 32 * w, smem);
+      if (e != cudaSuccess) return e;
+      const int64_t gw = (M + (int64_t)w * rpw - 1) / ((int64_t)w * rpw);   // CTAs of w warps
+      if (occ < 1 || gw > (int64_t)occ * num_sms) continue;                 // not all resident at once
+      const int64_t load = (gw + num_sms - 1) / num_sms * w;                // warps on the busiest SM
+      if (load < best_load) {
+        best_load = load;
+        wpc = w;
+        g = gw;
+      }
+    }
+    if (wpc == 0) continue;
+    const size_t smem = onepass_smem_bytes(sizeof(T), K, gamma != nullptr, rpw, wpc);
+    e = set_smem(smem);
     if (e != cudaSuccess) return e;
-    int occ = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_reorder_onepass<T>, 256, smem);
-    if (e != cudaSuccess) return e;
-    const int64_t g = (M + 8 * rpw - 1) / (8 * rpw);   // CTAs of 8 warps
-    if (occ < 1 || g > (int64_t)occ * num_sms) continue;   // not all resident at once
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)g);
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(32 * wpc);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
