@@ -4,10 +4,11 @@
 // Y^T = W X^T with W (N x K, NVFP4, TILED scales) as the 128-row A operand of
 // tcgen05.mma.kind::mxf4nvf4.block_scale.block16 and the activation rows
 // (padded to 16) as the B operand.  With a residue R (ResServe abstract: FP4
-// base plus FP4 residue, combined on-chip) X and R are stacked into one
-// 32-row B operand (rows 0-15 X, 16-31 R): each MMA then produces both
-// products side by side in one accumulator, for the same instruction count as
-// the plain case, and Y = s_x s_w acc[:, 0:16] + s_r s_w acc[:, 16:32].
+// base plus FP4 residue, combined on-chip) X and R are stacked into one B
+// operand, R's rows starting at row ro: ro = 8 for M <= 8 (one 16-row
+// operand, the plain case's instructions), else ro = 16 (a 32-row operand).
+// Each MMA then produces both products side by side in one accumulator, and
+// Y = s_x s_w acc[:, 0:M] + s_r s_w acc[:, ro:ro+M].
 //
 // Fused mode (nvfp4_quantize_gemm): the kernel reads X in bf16/fp32 and
 // quantizes it itself.  The ks CTAs of a cluster split K; together they cover
@@ -21,8 +22,8 @@
 // Plain mode (nvfp4_gemm): X codes arrive by TMA, X scales are gathered.
 //
 // Activation scales sit in shared memory compactly: per k-tile and K=64 chunk,
-// the 4 block scales of each of the 32 operand rows (X rows 0-15, R rows
-// 16-31).  In TMEM they take the layout of a scale atom (lane l, column c:
+// the 4 block scales of each of the 32 operand rows (X rows from 0, R rows
+// from ro).  In TMEM they take the layout of a scale atom (lane l, column c:
 // row 32c + l), with rows 32 and up absent (zero).  The scale operands of a
 // block-scaled MMA start on a 4-column TMEM boundary: each K=64 MMA reads one
 // atom's 4 columns.  With a residue, each CTA pushes s_x s_w acc_x + s_r s_w
