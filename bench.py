@@ -786,6 +786,8 @@ def reference_arm(args):
 def profile_case(case: str) -> int:
     """A handful of launches of one kernel, inputs just above L2, for ncu:
     decode   -- nvfp4_quantize_gemm, M=1, (N,K)=(4096,14336), 5 weight copies (147 MB)
+    decode_res -- nvfp4_quantize_residue_gemm (computed residue scale), M=4, (N,K)=(5120,5120)
+                (ResServe decode), Student-t activations, 12 weight copies (177 MB)
     prefill  -- nvfp4_gemm, M=8192, (N,K)=(14336,4096) (A 19 MB, W 33 MB, Y 470 MB)
     quantize -- nvfp4_quantize of the 8192x4096 bf16 prefill activations (67 MB)
     reorder  -- nvfp4_rmsnorm_reorder_quantize of the same activations, S=256
@@ -814,6 +816,20 @@ def profile_case(case: str) -> int:
         y = torch.empty((M, N), device=dev)
         for i in range(10):
             nv.nvfp4_quantize_gemm(x, qx, ws[i % 5], y)
+    elif case == "decode_res":
+        M, N, K = 4, 5120, 5120
+        w = torch.from_numpy(wl.weights_normal(N, K)).to(dev)
+        ws = []
+        for _ in range(12):
+            q = nv.NVFP4Tensor.empty(N, K, nv.SF_TILED, device=dev)
+            nv.nvfp4_quantize(w, q, workspace=nv.Workspace(N, K, dev))
+            ws.append(q)
+        x = wl.to_bf16(wl.resserve_x(M, K)).to(dev)
+        qx = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev)
+        rx = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev)
+        y = torch.empty((M, N), device=dev)
+        for i in range(12):
+            nv.nvfp4_quantize_residue_gemm(x, qx, rx, ws[i], y)
     elif case == "prefill":
         M, N, K = 8192, 14336, 4096
         qa = nv.NVFP4Tensor.empty(M, K, nv.SF_TILED, device=dev)
@@ -914,8 +930,8 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="decode: launch every step directly on the stream (no CUDA graphs) and skip the "
                          "per-call detail; for profilers that cannot follow graph replays")
-    ap.add_argument("--profile-case", choices=["decode", "prefill", "quantize", "reorder", "mxgemm", "arcquant", "gemv", "gemv_tc",
-                                               "mxquant"],
+    ap.add_argument("--profile-case", choices=["decode", "decode_res", "prefill", "quantize", "reorder", "mxgemm", "arcquant",
+                                               "gemv", "gemv_tc", "mxquant"],
                     help="run a few launches of one kernel on a small case (for ncu captures) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
