@@ -244,8 +244,8 @@ nvfp4_status nvfp4_quantize_residue_gemm(const void* x, nvfp4_dtype dt, int64_t 
 #define NVFP4_NOALLOC_MAX_ROWS 65536
 
 /* nvfp4_rmsnorm_reorder_quantize without a caller workspace, for callers that
- * cannot allocate device memory (code running during CUDA graph capture, hosts
- * that own every allocation, paths that must never call the allocator).  The
+ * cannot allocate device memory (hosts that own every allocation, paths that
+ * must never call the allocator).  The
  * method's pages have no counterpart: this is a deployment variant of the
  * fused quantizer above, with identical results.
  * Its scratch (reduction cells + one fp32 per row) is a device array inside the
@@ -256,7 +256,7 @@ nvfp4_status nvfp4_quantize_residue_gemm(const void* x, nvfp4_dtype dt, int64_t 
  * `stream`, so calls ordered on one stream are safe, while calls that may
  * overlap on the GPU (unordered streams) race on it.  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture begins.
+ * device current.
  * It calls no allocation routine.  Other arguments and errors as
  * nvfp4_rmsnorm_reorder_quantize. */
 nvfp4_status nvfp4_rmsnorm_reorder_quantize_noalloc(const void* x, nvfp4_dtype dt, int64_t M, int64_t K,

@@ -2,10 +2,9 @@
 // quantize entry point for callers that cannot allocate device memory.
 //
 // The regular entry point takes a caller-owned workspace (reduction cells and
-// one fp32 rinv per row).  Some callers cannot provide one: code that runs
-// while a CUDA graph is being captured (allocation is not capturable), plugins
-// embedded in a host framework that owns every device allocation, and
-// real-time paths that must never call the allocator.  This variant keeps the
+// one fp32 rinv per row).  Some callers cannot provide one: plugins embedded
+// in a host framework that owns every device allocation, and real-time paths
+// that must never call the allocator.  This variant keeps the
 // same scratch in a file-scope device array that lives as long as the library
 // is loaded, so it allocates nothing at all.
 //
@@ -18,8 +17,7 @@
 //    on the call's stream at the start of each call, and calls that overlap on
 //    the GPU (different streams without ordering) race on it;
 //  * the first call on a device resolves the array's device address with
-//    cudaGetSymbolAddress while that device is current; make that first call
-//    before any stream capture begins.
+//    cudaGetSymbolAddress while that device is current.
 #include <cuda_runtime.h>
 
 #include <mutex>

@@ -2,9 +2,9 @@
 called through the C ABI, gives the same codes, scales and tensor scale as the
 regular entry point with a caller workspace, on two calls in a row.
 
-It exists for callers that cannot allocate device memory (capture-time code,
-hosts that own every allocation); its scratch is a device array inside the
-library.  This file is collected last so a failure here leaves the rest of the
+It exists for callers that cannot allocate device memory (hosts that own
+every allocation, paths that must never call the allocator); its scratch is a
+device array inside the library.  This file is collected last so a failure here leaves the rest of the
 suite already run."""
 import ctypes
 
