@@ -69,14 +69,19 @@ __global__ void __launch_bounds__(256) k_amax(const T* __restrict__ x, int64_t M
   const int64_t upr = K >> 3;
   uint32_t key = 0;
   if (ldx == K) {
+    // Each CTA streams one contiguous, equal share of the units (boundaries
+    // on 32-unit lines), so no partly filled last round of the grid leaves
+    // the read stream short of CTAs.
     const int64_t units = M * upr;
     const int64_t cta = (int64_t)(blockIdx.y * gridDim.x + blockIdx.x), ctas = (int64_t)gridDim.x * gridDim.y;
-    for (int64_t base = cta * 256 * kUnroll; base < units; base += ctas * 256 * kUnroll) {
+    const int64_t u0 = (units * cta / ctas) & ~int64_t(31);
+    const int64_t u1 = cta + 1 == ctas ? units : (units * (cta + 1) / ctas) & ~int64_t(31);
+    for (int64_t base = u0; base < u1; base += 256 * kUnroll) {
       Raw8<T> raw[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int64_t i = base + u * 256 + threadIdx.x;
-        if (i < units) raw[u].load(x + i * 8);
+        if (i < u1) raw[u].load(x + i * 8);
         else raw[u].zero();
       }
 #pragma unroll
