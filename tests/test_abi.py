@@ -186,3 +186,48 @@ def test_host_io_validation_before_copies(lib):
     q17 = _tensor(17, 1024, good, good, good)
     assert f(good, good, 1, 17, 1024, 1024, None, ctypes.byref(q17), ctypes.byref(w), good, good, 0, 512,
              None, None) == 3                                                           # M > 16
+
+
+def test_weight_residue_noalloc_validation_before_launch(lib):
+    """nvfp4_quantize_weight, nvfp4_quantize_residue and the allocation-free fused
+    quantizer reject bad arguments on the host, before any CUDA call."""
+    good = 1 << 20
+    N, K, S = 32, 256, 32
+    wa = _tensor(N, K + S, good, good, good)
+    f = lib.nvfp4_quantize_weight
+
+    def weight(w=good, K=K, S=S, sigma=None, perm=good, t=wa, ws=good, dt=1):
+        return f(w, dt, N, K, K, sigma, perm, S, None, ctypes.byref(t), ws, 1 << 20, None, None)
+
+    assert weight(w=None) == 1                                    # null W
+    assert weight(K=250) == 1                                     # K % 16
+    assert weight(S=24) == 1                                      # S % 16
+    assert weight(S=K + 16) == 1                                  # S > K
+    assert weight(sigma=good + 2) == 2                            # misaligned sigma
+    assert weight(perm=good + 2) == 2                             # misaligned perm
+    assert weight(t=_tensor(N, K, good, good, good)) == 1         # W_aug must have K + S columns
+    assert weight(ws=None) == 7                                   # computed scale needs a workspace
+    assert weight(dt=9) == 1                                      # bad dtype
+
+    M = 4
+    q, r = _tensor(M, K, good, good, good), _tensor(M, K, good, good, good)
+    g = lib.nvfp4_quantize_residue
+    assert g(good, 1, M, K, K, None, None, ctypes.byref(q), None, good, 1 << 20, None, None) == 1   # no r
+    r_bad = _tensor(M + 1, K, good, good, good)
+    assert g(good, 1, M, K, K, None, None, ctypes.byref(q), ctypes.byref(r_bad), good, 1 << 20, None,
+             None) == 1                                           # r of another shape
+    assert g(good, 1, M, K, K, None, None, ctypes.byref(q), ctypes.byref(r), None, 0, None, None) == 7
+
+    h = lib.nvfp4_rmsnorm_reorder_quantize_noalloc
+    xa = _tensor(M, K + S, good, good, good)
+
+    def noalloc(x=good, M=M, t=xa, gamma=None, eps=1e-5, ldx=K):
+        return h(x, 1, M, K, ldx, gamma, ctypes.c_float(eps), None, S, None, ctypes.byref(t), None, None)
+
+    big = _tensor(65537, K + S, good, good, good)
+    assert noalloc(M=65537, t=big) == 7                           # beyond the built-in scratch
+    assert noalloc(x=None) == 1
+    assert noalloc(x=good + 8) == 2                               # x not 16-byte aligned
+    assert noalloc(ldx=K + 4) == 2                                # row stride not 16-byte aligned
+    assert noalloc(t=_tensor(M, K, good, good, good)) == 1        # X_aug must have K + S columns
+    assert noalloc(gamma=good, eps=-1.0) == 1                     # negative eps
